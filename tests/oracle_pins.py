@@ -1,0 +1,356 @@
+"""Pins that tie the CPU oracle to something other than itself.
+
+Each ``pin_*`` takes an oracle module ``orc`` (the real one, or a deliberately
+mutated copy in ``test_oracle_mutants.py``) and raises AssertionError when the
+oracle disagrees with:
+
+* closed-form hand cases (``tests/golden/hand_cases.json``);
+* the exact RMS invariant of a normalised row, mean(y^2) = ms / (ms + eps);
+* power-of-two scaling of the input (exact in 16-bit);
+* ``torch.nn.functional.rms_norm`` in float64 (an independent library routine);
+* torch's bf16 and numpy's float16 addition (the residual write-back);
+* torch's / numpy's format conversions, the e4m3 -> fp16 bit reinterpretation
+  from "MI210 LLM Stack - Optimizing 310B MoE Inference on 2x AMD MI210
+  (gfx90a)" (insight 4), and brute-force nearest-value search (the codecs);
+* properties every per-token e4m3 row must have.
+
+Operators: "vllm.kernels.aiter_ops" (rms_no_var_16bit_only,
+rms_add_no_var_16bit_only) and the fused residual + RMSNorm + FP8 pass of
+"Custom CUDA kernels juice Llama 3.1 405B on AMD MI300X, skipping Nvidia
+lock-in".
+"""
+from __future__ import annotations
+
+import bisect
+import math
+from decimal import Decimal
+
+import numpy as np
+import torch
+
+import synth
+from tests.cmp_util import bits16, ulp16
+
+ALL16 = np.arange(65536, dtype=np.uint32).astype(np.uint16)
+
+
+def _nan16(b, dtype):
+    if dtype == "bf16":
+        return ((b & 0x7F80) == 0x7F80) & ((b & 0x7F) != 0)
+    return ((b & 0x7C00) == 0x7C00) & ((b & 0x3FF) != 0)
+
+
+def _close(got, want_strs, rel=4e-16):
+    for g, w in zip(got, want_strs):
+        w = float(Decimal(w))
+        assert abs(g - w) <= rel * abs(w) + 1e-300, (g, w)
+
+
+def _nearest_even(sorted_vals, sorted_codes, v):
+    """Brute force: nearest representable value; a tie goes to the code whose
+    last bit (the significand's last bit) is 0."""
+    i = bisect.bisect_left(sorted_vals, v)
+    cands = [j for j in (i - 1, i) if 0 <= j < len(sorted_vals)]
+    best = min(abs(sorted_vals[j] - v) for j in cands)
+    ties = [j for j in cands if abs(sorted_vals[j] - v) == best]
+    if len(ties) == 1:
+        return sorted_codes[ties[0]]
+    even = [j for j in ties if (sorted_codes[j] & 1) == 0]
+    assert len(even) == 1
+    return sorted_codes[even[0]]
+
+
+def _bits(orc, values, dtype):
+    return orc.encode16(np.asarray(values, dtype=np.float64), dtype)
+
+
+# ---------------------------------------------------------------- codecs
+
+def pin_bf16_decode(orc, golden=None):
+    got = orc.decode16(ALL16, "bf16")
+    ref = torch.from_numpy(ALL16.view(np.int16).copy()).view(torch.bfloat16).double().numpy()
+    nan = _nan16(ALL16, "bf16")
+    assert np.isnan(got[nan]).all()
+    np.testing.assert_array_equal(got[~nan], ref[~nan])
+    assert np.array_equal(np.signbit(got[~nan]), np.signbit(ref[~nan]))
+
+
+def pin_f16_decode(orc, golden=None):
+    got = orc.decode16(ALL16, "fp16")
+    ref = ALL16.view(np.float16).astype(np.float64)
+    nan = _nan16(ALL16, "fp16")
+    assert np.isnan(got[nan]).all()
+    np.testing.assert_array_equal(got[~nan], ref[~nan])
+    assert np.array_equal(np.signbit(got[~nan]), np.signbit(ref[~nan]))
+
+
+def pin_e4m3_decode_bit_trick(orc, golden=None):
+    # h = ((u & 0x80) << 8) | ((u & 0x7f) << 7) is an fp16 holding exactly
+    # 2^-8 times the e4m3 value, for normals and subnormals alike.
+    u = np.arange(256, dtype=np.uint16)
+    h = ((u & 0x80) << 8) | ((u & 0x7F) << 7)
+    trick = h.astype(np.uint16).view(np.float16).astype(np.float64) * 256.0
+    got = orc.decode_e4m3(u.astype(np.uint8))
+    nan_codes = (u & 0x7F) == 0x7F
+    assert np.isnan(got[nan_codes]).all()
+    np.testing.assert_array_equal(got[~nan_codes], trick[~nan_codes])
+    assert np.array_equal(np.signbit(got[~nan_codes]), np.signbit(trick[~nan_codes]))
+    ref = torch.from_numpy(u.astype(np.uint8)).view(torch.float8_e4m3fn).double().numpy()
+    np.testing.assert_array_equal(got[~nan_codes], ref[~nan_codes])
+
+
+def pin_e4m3_encode(orc, golden=None):
+    u = np.arange(256, dtype=np.uint8)
+    finite = (u & 0x7F) != 0x7F
+    np.testing.assert_array_equal(orc.encode_e4m3(orc.decode_e4m3(u[finite])), u[finite])
+    pos = u[u < 0x7F]
+    pv = torch.from_numpy(pos.copy()).view(torch.float8_e4m3fn).double().numpy()
+    order = np.argsort(pv)
+    sv, sc = list(pv[order]), [int(c) for c in pos[order]]
+    rng = np.random.default_rng(7)
+    mids = [(sv[k] + sv[k + 1]) / 2 for k in range(len(sv) - 1)]
+    vals = np.concatenate([rng.uniform(0, 448, 2000), 2.0 ** rng.uniform(-12, 9, 2000),
+                           np.array(mids)])
+    got = orc.encode_e4m3(vals)
+    for v, g in zip(vals, got):
+        assert int(g) == _nearest_even(sv, sc, float(v)), v
+    np.testing.assert_array_equal(orc.encode_e4m3(-vals), got | 0x80)
+    big = np.array([448.0, 449.0, 463.9, 464.0, 480.0, 1e6, math.inf])
+    np.testing.assert_array_equal(orc.encode_e4m3(big), np.full(7, 0x7E))
+    np.testing.assert_array_equal(orc.encode_e4m3(-big), np.full(7, 0xFE))
+    assert orc.encode_e4m3(np.array([336.0]))[0] == 0x7A  # tie 320|352 -> 320
+    assert orc.encode_e4m3(np.array([math.nan]))[0] == 0x7F
+    # against torch's own cast on float32-exact, in-range values
+    v = np.clip(np.concatenate([rng.normal(0, 50, 5000), rng.normal(0, 0.01, 2000)]),
+                -448, 448).astype(np.float32)
+    ref = torch.from_numpy(v).to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+    np.testing.assert_array_equal(orc.encode_e4m3(v.astype(np.float64)), ref)
+
+
+def pin_f16_encode(orc, golden=None):
+    rng = np.random.default_rng(3)
+    v = np.concatenate([
+        rng.normal(0, 1, 20000), rng.normal(0, 1e-5, 5000), rng.uniform(6e4, 7e4, 2000),
+        np.array([65519.99, 65520.0, 65520.01, 2.0 ** -25, 2.0 ** -25 * 1.0000001,
+                  3 * 2.0 ** -26, 0.0]),
+    ])
+    v = np.concatenate([v, -v])
+    with np.errstate(over="ignore"):
+        ref = v.astype(np.float16).view(np.uint16)  # numpy rounds binary64 -> fp16 directly
+    np.testing.assert_array_equal(orc.encode16(v, "fp16"), ref)
+    h = orc.encode16(np.array([1 + 2 ** -11, 1 + 3 * 2 ** -11, 2.0 ** -25, 3 * 2.0 ** -25,
+                               65520.0, 65519.0, -1e300]), "fp16")
+    assert list(h) == [0x3C00, 0x3C02, 0x0000, 0x0002, 0x7C00, 0x7BFF, 0xFC00]
+
+
+def pin_bf16_encode(orc, golden=None):
+    rng = np.random.default_rng(5)
+    v32 = np.concatenate([
+        rng.normal(0, 1, 20000), rng.normal(0, 1e-39, 3000),
+        np.array([3.3895313892515355e38, 3.39e38, 3.4028234e38]),
+    ]).astype(np.float32)
+    v32 = np.concatenate([v32, -v32])
+    ref = torch.from_numpy(v32).to(torch.bfloat16).view(torch.int16).numpy().view(np.uint16)
+    np.testing.assert_array_equal(orc.encode16(v32.astype(np.float64), "bf16"), ref)
+    b = orc.encode16(np.array([1 + 2 ** -8, 1 + 3 * 2 ** -8, 1 + 2 ** -8 + 2 ** -30]), "bf16")
+    assert list(b) == [0x3F80, 0x3F82, 0x3F81]
+
+
+def pin_encode16_brute_force(orc, golden=None):
+    """Doubles that are not float32-exact, against a brute-force nearest search."""
+    for dtype in ("bf16", "fp16"):
+        if dtype == "bf16":
+            allv = torch.from_numpy(ALL16.view(np.int16).copy()).view(torch.bfloat16).double().numpy()
+        else:
+            allv = ALL16.view(np.float16).astype(np.float64)
+        finite = np.isfinite(allv) & (ALL16 < 0x8000)
+        idx = np.argsort(allv[finite])
+        sv = list(allv[finite][idx])
+        sc = [int(c) for c in ALL16[finite][idx]]
+        rng = np.random.default_rng(13)
+        hi = 3.3e38 if dtype == "bf16" else 65000.0
+        v = np.concatenate([np.exp(rng.uniform(-30, math.log(hi), 1500)),
+                            rng.uniform(0.5, 4, 1000) + rng.uniform(-1e-12, 1e-12, 1000)])
+        k = rng.integers(0, len(sv) - 1, 500)
+        v = np.concatenate([v, (np.array(sv)[k] + np.array(sv)[k + 1]) / 2])
+        got = orc.encode16(v, dtype)
+        for x, g in zip(v, got):
+            assert int(g) == _nearest_even(sv, sc, float(x)), (dtype, x, hex(g))
+
+
+# ---------------------------------------------------------------- operators
+
+def pin_rms_norm_hand_cases(orc, golden):
+    for dtype in ("bf16", "fp16"):
+        for case in golden["rms_norm"]:
+            x = _bits(orc, [case["x"]], dtype)
+            w = None if case["w"] is None else _bits(orc, case["w"], dtype)
+            out, y = orc.rms_norm(x, w, dtype, case["eps"], want_y=True)
+            _close(y[0], case["y"])
+            if dtype == "bf16" and "bf16_out" in case:
+                assert [int(v) for v in out[0]] == [int(s, 16) for s in case["bf16_out"]]
+
+
+def pin_fused_hand_cases(orc, golden):
+    for dtype in ("bf16", "fp16"):
+        for case in golden["fused_add_rms_norm"]:
+            if "x_bits" in case:
+                if case["dtype"] != dtype:
+                    continue
+                x = np.array([[int(s, 16) for s in case["x_bits"]]], np.uint16)
+                r = np.array([[int(s, 16) for s in case["r_bits"]]], np.uint16)
+                r_out, _ = orc.fused_add_rms_norm(x, r, None, dtype, 1e-6)
+                assert [int(v) for v in r_out[0]] == [int(s, 16) for s in case["r_out_bits"]]
+                continue
+            x = _bits(orc, [case["x"]], dtype)
+            r = _bits(orc, [case["r"]], dtype)
+            r_out, out, y = orc.fused_add_rms_norm(x, r, None, dtype, case["eps"], want_y=True)
+            np.testing.assert_array_equal(orc.decode16(r_out, dtype)[0], case["r_out"])
+            _close(y[0], case["y"])
+
+
+def pin_fp8_hand_cases(orc, golden):
+    for dtype in ("bf16", "fp16"):
+        for case in golden["fused_add_rms_norm_fp8"]:
+            x = _bits(orc, [case["x"]], dtype)
+            r = _bits(orc, [case["r"]], dtype)
+            w = None if case["w"] is None else _bits(orc, case["w"], dtype)
+            _, q, scale = orc.fused_add_rms_norm_fp8(x, r, w, dtype, case["eps"])
+            assert [int(c) for c in q[0]] == [int(s, 16) for s in case["q_bits"]]
+            assert scale[0] == np.float32(float(case["scale"]))
+
+
+def _rows(T, H, dtype, seed, var=1.0):
+    g = torch.Generator().manual_seed(seed)
+    return bits16(synth.normal((T, H), var, g, "cpu").to(synth.to_dtype(dtype)))
+
+
+def pin_rms_invariant(orc, golden=None):
+    """With w = 1: mean(y^2) = ms / (ms + eps), exactly in closed form."""
+    for dtype in ("bf16", "fp16"):
+        for eps in (0.0, 1e-6, 0.5):
+            x = _rows(16, 1000, dtype, 1)
+            _, y = orc.rms_norm(x, None, dtype, eps, want_y=True)
+            xv = torch.from_numpy(x.view(np.int16).copy()).view(synth.to_dtype(dtype)).double().numpy()
+            ms = (xv * xv).mean(axis=1)
+            lhs = np.sqrt((y * y).mean(axis=1))
+            rhs = np.sqrt(ms / (ms + np.float64(np.float32(eps))))
+            np.testing.assert_allclose(lhs, rhs, rtol=1e-14)
+
+
+def pin_power_of_two_scaling(orc, golden=None):
+    for dtype in ("bf16", "fp16"):
+        tdt = synth.to_dtype(dtype)
+        g = torch.Generator().manual_seed(2)
+        xf = synth.normal((8, 512), 1.0, g, "cpu")
+        xf = torch.sign(xf) * xf.abs().clamp_min(0.01)  # keep 2^-3 x a normal number
+        x = bits16(xf.to(tdt))
+        w = _rows(1, 512, dtype, 3)[0]
+        xv = torch.from_numpy(x.view(np.int16).copy()).view(tdt).double()
+        wv = torch.from_numpy(w.view(np.int16).copy()).view(tdt).double().numpy()
+        for k in (-3, 4):
+            a = 2.0 ** k
+            xs = bits16((xv * a).to(tdt))  # exact: power-of-two scaling of normals
+            assert np.array_equal(orc.decode16(xs, dtype), xv.numpy() * a)
+            np.testing.assert_array_equal(orc.rms_norm(xs, w, dtype, 0.0),
+                                          orc.rms_norm(x, w, dtype, 0.0))
+            eps = 1e-2
+            _, y1 = orc.rms_norm(xs, w, dtype, eps, want_y=True)
+            xn = xv.numpy()
+            ms = (xn * xn).mean(axis=1, keepdims=True)
+            expect = a * xn / np.sqrt(a * a * ms + np.float64(np.float32(eps))) * wv
+            np.testing.assert_allclose(y1, expect, rtol=1e-14, atol=0)
+
+
+def pin_torch_rms_norm_float64(orc, golden=None):
+    for dtype in ("bf16", "fp16"):
+        for with_w in (True, False):
+            wl = synth.make_inputs("sweep", "rms_norm", dtype, 33, 2048)
+            w = wl.weight if with_w else None
+            _, y = orc.rms_norm(bits16(wl.x), None if w is None else bits16(w), dtype,
+                                wl.eps, want_y=True)
+            ref = torch.nn.functional.rms_norm(
+                wl.x.double(), (2048,), None if w is None else w.double(),
+                eps=float(np.float32(wl.eps))).numpy()
+            np.testing.assert_allclose(y, ref, rtol=1e-13, atol=1e-300)
+
+
+def pin_residual_library_addition(orc, golden=None):
+    """r' = RNE16(x + r) against torch's bf16 and numpy's float16 addition over
+    bit patterns that include subnormals, ties and large exponent gaps."""
+    rng = np.random.default_rng(17)
+    pats = np.concatenate([rng.integers(0, 65536, 3000),
+                           np.array([0x0001, 0x8001, 0x3F80, 0x3B80, 0x3F81, 0x0400, 0x7BFF])])
+    pats = pats.astype(np.uint16)
+    xs = np.repeat(pats, 32)
+    rs = rng.choice(pats, xs.size).astype(np.uint16)
+    for dtype in ("bf16", "fp16"):
+        if dtype == "bf16":
+            tx = torch.from_numpy(xs.view(np.int16).copy()).view(torch.bfloat16)
+            tr = torch.from_numpy(rs.view(np.int16).copy()).view(torch.bfloat16)
+            ok = (torch.isfinite(tx) & torch.isfinite(tr)).numpy()
+            ref = (tx + tr).view(torch.int16).numpy().view(np.uint16)[ok]
+        else:
+            fx, fr = xs.view(np.float16), rs.view(np.float16)
+            ok = np.isfinite(fx) & np.isfinite(fr)
+            with np.errstate(over="ignore"):
+                ref = (fx[ok] + fr[ok]).view(np.uint16)
+        x2, r2 = xs[ok].reshape(1, -1), rs[ok].reshape(1, -1)
+        r_out, _ = orc.fused_add_rms_norm(x2, r2, None, dtype, 1e-6)
+        got = r_out[0]
+        nan_ref = _nan16(ref, dtype)
+        assert (_nan16(got, dtype) == nan_ref).all()
+        np.testing.assert_array_equal(got[~nan_ref], ref[~nan_ref])
+
+
+def pin_fused_equals_norm_of_written_back(orc, golden=None):
+    for dtype in ("bf16", "fp16"):
+        wl = synth.make_inputs("decode", "fused_add_rms_norm", dtype, 64, 4096)
+        x, r, w = bits16(wl.x), bits16(wl.residual), bits16(wl.weight)
+        r_out, out = orc.fused_add_rms_norm(x, r, w, dtype, wl.eps)
+        np.testing.assert_array_equal(out, orc.rms_norm(r_out, w, dtype, wl.eps))
+        # the same output computed from torch's own rounded sum
+        rs = bits16(wl.x + wl.residual)
+        np.testing.assert_array_equal(out, orc.rms_norm(rs, w, dtype, wl.eps))
+
+
+def pin_fp8_row_properties(orc, golden=None):
+    for dtype in ("bf16", "fp16"):
+        wl = synth.make_inputs("outlier", "fused_add_rms_norm_fp8", dtype, 64, 16384)
+        x, r, w = bits16(wl.x), bits16(wl.residual), bits16(wl.weight)
+        r_out, q, scale, y = orc.fused_add_rms_norm_fp8(x, r, w, dtype, wl.eps, want_y=True)
+        r2, out16 = orc.fused_add_rms_norm(x, r, w, dtype, wl.eps)
+        np.testing.assert_array_equal(r_out, r2)
+        # y agrees with float64 torch on the written-back residual
+        tdt = synth.to_dtype(dtype)
+        rt = torch.from_numpy(r_out.view(np.int16).copy()).view(tdt).double()
+        yt = torch.nn.functional.rms_norm(rt, (16384,), wl.weight.double(),
+                                          eps=float(np.float32(wl.eps))).numpy()
+        np.testing.assert_allclose(y, yt, rtol=1e-13, atol=1e-300)
+        # every non-zero row reaches the largest code and never a NaN code
+        assert ((q == 0x7E) | (q == 0xFE)).any(axis=1).all()
+        assert not ((q & 0x7F) == 0x7F).any()
+        amax = np.abs(yt).max(axis=1)
+        np.testing.assert_allclose(scale, amax / 448.0, rtol=2 ** -24)
+        # dequantised codes lie within half an e4m3 step of y
+        deq = torch.from_numpy(q.copy()).view(torch.float8_e4m3fn).double().numpy() \
+            * (amax / 448.0)[:, None]
+        half_step = np.maximum(np.abs(yt) * 2.0 ** -4, 2.0 ** -10 * (amax / 448.0)[:, None])
+        assert (np.abs(deq - yt) <= half_step * (1 + 1e-9)).all()
+        # the codes depend only on x*w / max|x*w|, not on eps or the rms
+        _, q_eps, _ = orc.fused_add_rms_norm_fp8(x, r, w, dtype, 0.5)
+        np.testing.assert_array_equal(q_eps, q)
+        # the 16-bit output of the same row is RNE16(y), per torch's rounding of y
+        assert ulp16(out16, bits16(torch.from_numpy(yt).to(tdt))).max() <= 1
+
+
+def pin_zero_rows(orc, golden=None):
+    x = np.zeros((3, 64), np.uint16)
+    r_out, q, scale = orc.fused_add_rms_norm_fp8(x, x, None, "bf16", 1e-6)
+    assert (q == 0).all() and (scale == 0).all() and (r_out == 0).all()
+    assert (orc.rms_norm(x, None, "fp16", 1e-6) == 0).all()
+    _, y = orc.rms_norm(x, None, "bf16", 0.0, want_y=True)
+    assert np.isnan(y).all()  # 0/0 with eps = 0
+
+
+PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

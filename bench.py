@@ -1,0 +1,487 @@
+#!/usr/bin/env python3
+"""Benchmark of the fused add + RMSNorm (+FP8) path on B200.
+
+One step = one pass of the whole path over one batch: the prefill workload
+[8192 x 3840] bf16 (x ~ Student-t(3) clipped to +-1e3, residual ~ N(0,16),
+weight = 1 + N(0,0.1), eps 1e-6) through
+  1. fused_add_rms_norm       (residual write-back + bf16 output), and
+  2. fused_add_rms_norm_fp8   (residual write-back + per-token e4m3 + scale).
+Metric: algorithmic HBM GB/s of the step (bytes every element must move,
+weight counted once per launch), its fraction of the HBM roofline, and rows/s.
+
+Timing: W untimed warm-up steps, then K steps bracketed by a barrier and a
+device synchronize, timed with CUDA events on the launching stream; per-kernel
+durations from event pairs around each launch. L2: launches rotate over
+buffer sets totalling >= 4x the L2 size, so no launch reads data the previous
+launches left in L2. Under torchrun each rank runs an independent replica
+(no collective on the data path; the path has no exchange step) and rank 0
+prints the max-over-ranks time.
+
+`--impl reference` times the fp64 CPU oracle (the reference arm; host cores).
+Usage: python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import statistics
+import sys
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+import synth  # noqa: E402
+
+METRIC = "fused add+RMSNorm(+FP8) HBM GB/s and % of B200 peak; rows/sec"
+NOMINAL_HBM_GBS = 8000.0
+FALLBACK_HBM_GBS = 6650.0
+T_PREFILL, H_PREFILL = 8192, 3840
+PROFILE_SUMMARY = os.path.join(ROOT, "profiles",
+                               "ncu_fused_add_rms_norm_prefill_bf16_8192x3840.md")
+
+
+def op_bytes(op: str, T: int, H: int, esize: int = 2) -> int:
+    """Algorithmic bytes of one launch: what each element must move once."""
+    if op == "rms_norm":
+        return 2 * esize * H * T + esize * H          # read x, write out; weight
+    if op == "fused_add_rms_norm":
+        return 4 * esize * H * T + esize * H          # read x, r; write r, out; weight
+    return (3 * esize + 1) * H * T + 4 * T + esize * H  # read x, r; write r, q, scale; weight
+
+
+STEP_OPS = ("fused_add_rms_norm", "fused_add_rms_norm_fp8")
+
+
+def step_bytes(T: int, H: int) -> int:
+    return sum(op_bytes(op, T, H) for op in STEP_OPS)
+
+
+def csrc_digest() -> str:
+    h = hashlib.sha256()
+    d = os.path.join(ROOT, "residual_add_rmsnorm_rms_b200", "csrc")
+    for name in sorted(os.listdir(d)):
+        with open(os.path.join(d, name), "rb") as f:
+            h.update(name.encode() + f.read())
+    return h.hexdigest()[:16]
+
+
+def measured_peak():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            j = json.load(f)
+        return float(j["hbm_gbs"]), "measured (MEASURED_PEAKS.json hbm_gbs, torch copy)"
+    except (OSError, KeyError, ValueError):
+        return FALLBACK_HBM_GBS, "fallback (6.65 TB/s earlier pool measurement)"
+
+
+def ncu_traffic():
+    """DRAM bytes per launch of the dominant kernel from the committed ncu
+    summary, or None when the kernels changed since it was captured."""
+    try:
+        text = open(PROFILE_SUMMARY).read()
+    except OSError:
+        return None
+    vals = {}
+    for line in text.splitlines():
+        if ":" in line and line.strip().startswith("- "):
+            k, v = line.strip()[2:].split(":", 1)
+            vals[k.strip()] = v.strip().strip("`")
+    if vals.get("csrc_digest") != csrc_digest():
+        return None
+    try:
+        return int(vals["dram_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """SM clock and clock-event (throttle) reasons of this process's GPU,
+    polled through NVML from a background thread every few milliseconds while
+    the timed region runs (read-only queries; no GPU setting is changed)."""
+
+    REASONS = (("hw_slowdown", "nvmlClocksEventReasonHwSlowdown"),
+               ("hw_thermal_slowdown", "nvmlClocksEventReasonHwThermalSlowdown"),
+               ("sw_thermal_slowdown", "nvmlClocksEventReasonSwThermalSlowdown"),
+               ("sw_power_cap", "nvmlClocksEventReasonSwPowerCap"),
+               ("hw_power_brake_slowdown", "nvmlClocksEventReasonHwPowerBrakeSlowdown"))
+
+    def __init__(self, device, period_s: float = 0.005):
+        import threading
+        self.period = period_s
+        self.samples = []
+        self.max_mhz = None
+        self._stop = threading.Event()
+        self._thread = None
+        self.err = None
+        try:
+            import pynvml
+            pynvml.nvmlInit()
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            if not uuid.startswith("GPU-"):
+                uuid = "GPU-" + uuid
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.masks = [(n, getattr(pynvml, c)) for n, c in self.REASONS if hasattr(pynvml, c)]
+        except Exception as e:  # no NVML: report no clocks rather than guess
+            self.nv = None
+            self.err = f"{type(e).__name__}: {e}"
+
+    def _poll(self):
+        nv = self.nv
+        while not self._stop.is_set():
+            try:
+                mhz = nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM)
+                bits = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                self.samples.append((mhz, bits))
+            except Exception as e:
+                self.err = f"{type(e).__name__}: {e}"
+                return
+            self._stop.wait(self.period)
+
+    def start(self):
+        import threading
+        if self.nv is None:
+            return
+        self._thread = threading.Thread(target=self._poll, daemon=True)
+        self._thread.start()
+
+    def stop(self):
+        if self._thread is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0,
+                    "error": self.err}
+        self._stop.set()
+        self._thread.join(timeout=2)
+        mhz = [m for m, _ in self.samples]
+        reasons = sorted({n for _, b in self.samples for n, m in self.masks if b & m})
+        return {"sm_mhz": statistics.median(mhz) if mhz else None, "sm_max_mhz": self.max_mhz,
+                "reasons": reasons, "samples": len(mhz), "source": "NVML, polled every 5 ms"}
+
+
+def dist_setup():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if torch.cuda.is_available():
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    return world, rank, local
+
+
+def max_over_ranks(value: float, world: int, device) -> float:
+    if world == 1:
+        return value
+    import torch.distributed as dist
+    t = torch.tensor([value], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(world: int):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+
+def oracle_step_sample(rows: int, threads: int, seed_inputs=None):
+    """Runs the oracle over `rows` rows of the prefill workload (both ops of a
+    step); returns (seconds, rows, bytes)."""
+    import oracle
+    if seed_inputs is None:
+        wl = synth.make_inputs("prefill", "fused_add_rms_norm", "bf16", rows, H_PREFILL)
+        seed_inputs = (wl.x, wl.residual, wl.weight, wl.eps)
+    x, r, w, eps = seed_inputs
+    xb = x.contiguous().view(torch.int16).numpy()
+    rb = r.contiguous().view(torch.int16).numpy()
+    wb = w.contiguous().view(torch.int16).numpy()
+    t0 = time.perf_counter()
+    oracle.fused_add_rms_norm(xb, rb, wb, "bf16", eps, threads=threads)
+    oracle.fused_add_rms_norm_fp8(xb, rb, wb, "bf16", eps, threads=threads)
+    dt = time.perf_counter() - t0
+    return dt, rows, step_bytes(rows, H_PREFILL)
+
+
+def cpu_baseline(target_cpu_s: float = 15.0):
+    import oracle
+    cores = oracle.usable_cores()
+    probe_rows = 64
+    wl = synth.make_inputs("prefill", "fused_add_rms_norm", "bf16", T_PREFILL, H_PREFILL)
+    probe = (wl.x[:probe_rows], wl.residual[:probe_rows], wl.weight, wl.eps)
+    dt, _, _ = oracle_step_sample(probe_rows, 1, probe)
+    per_row = dt / probe_rows
+    rows = int(max(probe_rows, min(T_PREFILL, target_cpu_s / per_row)))
+    sample = (wl.x[:rows], wl.residual[:rows], wl.weight, wl.eps)
+    dt, rows, nbytes = oracle_step_sample(rows, cores, sample)
+    return {"value": round(nbytes / dt / 1e9, 4), "unit": "GB/s", "cores": cores,
+            "kind": "oracle",
+            "rows_per_s": round(rows / dt, 2),
+            "sample": f"first {rows} of {T_PREFILL} rows of the prefill batch, both ops of a step, "
+                      f"fp64 C oracle on {cores} host threads, {dt:.2f} s wall"}
+
+
+def run_reference(args, world, rank):
+    """The reference arm: the fp64 CPU oracle timed on the host cores."""
+    if rank != 0:
+        return
+    import oracle
+    cores = oracle.usable_cores()
+    rows = args.reference_rows
+    wl = synth.make_inputs("prefill", "fused_add_rms_norm", "bf16", rows, H_PREFILL)
+    inp = (wl.x, wl.residual, wl.weight, wl.eps)
+    for _ in range(args.warmup):
+        oracle_step_sample(rows, cores, inp)
+    total = 0.0
+    for _ in range(args.steps):
+        dt, _, _ = oracle_step_sample(rows, cores, inp)
+        total += dt
+    nbytes = step_bytes(rows, H_PREFILL) * args.steps
+    value = nbytes / total / 1e9
+    sample = (f"{rows} of {T_PREFILL} rows of the prefill batch per step, both ops, fp64 C oracle "
+              f"on {cores} host threads")
+    line = {
+        "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
+        "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(total / args.steps * 1e3, 3), "higher_is_better": True,
+        "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "rows_per_s": round(rows * args.steps / total, 2),
+        "config": {"workload": f"prefill fused_add_rms_norm + fused_add_rms_norm_fp8, bf16, "
+                               f"{T_PREFILL}x{H_PREFILL} (row sample of {rows})",
+                   "T": rows, "H": H_PREFILL},
+        "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores,
+                         "kind": "oracle", "sample": sample},
+        "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+        "gpu_launches": 0,
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ----------------------------------------------------------------------------- GPU arm
+
+class Sets:
+    """Rotating device buffer sets for the two ops of a step."""
+
+    def __init__(self, wl, n_sets, device):
+        T, H = wl.T, wl.H
+        self.w = wl.weight.to(device)
+        self.sets = []
+        for _ in range(n_sets):
+            self.sets.append({
+                "x": wl.x.to(device),
+                "r": wl.residual.to(device).clone(),
+                "out": torch.empty(T, H, dtype=wl.dtype, device=device),
+                "q": torch.empty(T, H, dtype=torch.float8_e4m3fn, device=device),
+                "scale": torch.empty(T, dtype=torch.float32, device=device),
+            })
+
+
+def set_bytes(T, H):
+    return 2 * T * H * 3 + T * H + 4 * T
+
+
+def run_ours(args, world, rank, local):
+    import residual_add_rmsnorm_rms_b200 as rn
+    if not torch.cuda.is_available():
+        raise SystemExit("bench.py needs a CUDA device for --impl ours")
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    T, H = T_PREFILL, H_PREFILL
+    wl = synth.make_inputs("prefill", "fused_add_rms_norm", "bf16", T, H, device=device)
+    eps = wl.eps
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    n_sets = max(2, math.ceil(4 * l2 / set_bytes(T, H)) + 1)
+    S = Sets(wl, n_sets, device)
+    stream = torch.cuda.current_stream(device)
+    w = S.w
+
+    def launch(i, k):
+        # launch k (0: bf16 output, 1: fp8) of step i uses its own buffer set
+        s = S.sets[(2 * i + k) % n_sets]
+        if k == 0:
+            rn.fused_add_rms_norm(s["out"], s["x"], s["r"], w, eps, stream=stream)
+        else:
+            rn.fused_add_rms_norm_fp8(s["q"], s["scale"], s["x"], s["r"], w, eps, stream=stream)
+
+    for i in range(args.warmup):
+        launch(i, 0)
+        launch(i, 1)
+    torch.cuda.synchronize(device)
+
+    K = args.steps
+    # Pass A (the headline): K steps, events only at the two ends.
+    clocks = ClockSampler(device)
+    e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize(device)
+    clocks.start()
+    e_start.record(stream)
+    for i in range(K):
+        launch(i, 0)
+        launch(i, 1)
+    e_end.record(stream)
+    torch.cuda.synchronize(device)
+    clk = clocks.stop()
+    barrier(world)
+    total_ms = max_over_ranks(e_start.elapsed_time(e_end), world, device)
+
+    # Pass B: the same K steps with an event pair around every launch, for
+    # the per-kernel durations (the roofline of the dominant kernel).
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
+    barrier(world)
+    torch.cuda.synchronize(device)
+    for i in range(K):
+        ev[i][0].record(stream)
+        launch(i, 0)
+        ev[i][1].record(stream)
+        launch(i, 1)
+        ev[i][2].record(stream)
+    torch.cuda.synchronize(device)
+    barrier(world)
+    k0 = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K)]
+    k1 = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]
+    passb_ms = ev[0][0].elapsed_time(ev[K - 1][2])
+
+    # end to end through the public API with host buffers: pinned H2D of each
+    # launch's inputs, the two launches, D2H of every output, all timed.
+    e2e = run_e2e(args, rn, wl, S, device, stream)
+    del S
+    torch.cuda.empty_cache()
+
+    b_step = step_bytes(T, H)
+    value = b_step * K * world / (total_ms / 1e3) / 1e9
+    peak, peak_src = measured_peak()
+    dom_bytes = op_bytes("fused_add_rms_norm", T, H)
+    dom_ms = statistics.mean(k0)
+    achieved = dom_bytes / (dom_ms / 1e3) / 1e9
+    fp8_ms = statistics.mean(k1)
+    traffic = ncu_traffic()
+    cpu = cpu_baseline() if (rank == 0 and world == 1 and not args.no_cpu_baseline) else None
+    if rank != 0:
+        return
+    line = {
+        "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
+        "steps": K, "warmup": args.warmup, "ms_per_step": round(total_ms / K, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic",
+        "rows_per_s": round(T * K * world / (total_ms / 1e3), 1),
+        "frac_of_nominal_8tbs": round(value / world / NOMINAL_HBM_GBS, 4),
+        "frac_of_measured_peak": round(value / world / peak, 4),
+        "config": {
+            "workload": f"prefill: fused_add_rms_norm (bf16 out) + fused_add_rms_norm_fp8 "
+                        f"(e4m3 + per-token scale), bf16 [{T} x {H}]",
+            "T": T, "H": H, "eps": eps,
+            "inputs": "x ~ Student-t(3) clipped +-1e3, residual ~ N(0,16), weight 1+N(0,0.1)",
+            "l2": f"rotating {n_sets} buffer sets ({n_sets * set_bytes(T, H) / 1e6:.0f} MB, "
+                  f">= 4x L2 of {l2 / 1e6:.0f} MB); no L2 flush",
+            "bytes_per_step": b_step,
+            "plans": {op: rn.plan_launch(op, torch.bfloat16, T, H) for op in STEP_OPS},
+        },
+        "per_kernel_pass_ms_per_step": round(passb_ms / K, 5),
+        "per_kernel_ms": {"fused_add_rms_norm": round(dom_ms, 5),
+                          "fused_add_rms_norm_fp8": round(fp8_ms, 5)},
+        "per_kernel_gbs": {"fused_add_rms_norm": round(achieved, 1),
+                           "fused_add_rms_norm_fp8": round(
+                               op_bytes("fused_add_rms_norm_fp8", T, H) / (fp8_ms / 1e3) / 1e9, 1)},
+        "roofline": {"bound": "hbm", "kernel": "fused_add_rms_norm", "achieved": round(achieved, 1),
+                     "peak": peak, "peak_source": peak_src, "unit": "GB/s",
+                     "frac": round(achieved / peak, 4),
+                     "frac_of_nominal_8tbs": round(achieved / NOMINAL_HBM_GBS, 4),
+                     "algorithmic_bytes_per_launch": dom_bytes,
+                     "traffic": traffic},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": 2 * K,
+        "clocks": clk,
+    }
+    print(json.dumps(line), flush=True)
+
+
+def run_e2e(args, rn, wl, S, device, stream):
+    T, H = wl.T, wl.H
+    pin = lambda t: t.cpu().pin_memory()  # noqa: E731
+    hx, hr = pin(wl.x), pin(wl.residual)
+    outs = {
+        "r0": torch.empty(T, H, dtype=wl.dtype).pin_memory(),
+        "out": torch.empty(T, H, dtype=wl.dtype).pin_memory(),
+        "r1": torch.empty(T, H, dtype=wl.dtype).pin_memory(),
+        "q": torch.empty(T, H, dtype=torch.uint8).pin_memory(),
+        "scale": torch.empty(T, dtype=torch.float32).pin_memory(),
+    }
+    a, b = S.sets[0], S.sets[1]
+    w = S.w
+    h2d = 4 * hx.numel() * 2
+    d2h = sum(t.numel() * t.element_size() for t in outs.values())
+
+    def step():
+        a["x"].copy_(hx, non_blocking=True)
+        a["r"].copy_(hr, non_blocking=True)
+        b["x"].copy_(hx, non_blocking=True)
+        b["r"].copy_(hr, non_blocking=True)
+        rn.fused_add_rms_norm(a["out"], a["x"], a["r"], w, wl.eps, stream=stream)
+        rn.fused_add_rms_norm_fp8(b["q"], b["scale"], b["x"], b["r"], w, wl.eps, stream=stream)
+        outs["r0"].copy_(a["r"], non_blocking=True)
+        outs["out"].copy_(a["out"], non_blocking=True)
+        outs["r1"].copy_(b["r"], non_blocking=True)
+        outs["q"].copy_(b["q"].view(torch.uint8), non_blocking=True)
+        outs["scale"].copy_(b["scale"], non_blocking=True)
+
+    n = max(3, min(args.steps, 10))
+    for _ in range(2):
+        step()
+    torch.cuda.synchronize(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(n):
+        step()
+    e1.record(stream)
+    torch.cuda.synchronize(device)
+    ms = e0.elapsed_time(e1) / n
+    return {"value": round(step_bytes(T, H) / (ms / 1e3) / 1e9, 3), "unit": "GB/s",
+            "ms_per_step": round(ms, 4), "steps": n,
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+            "how": "pinned host buffers; per step H2D of x and residual for each of the two "
+                   "launches, both launches through the C ABI, D2H of residual, out, q, scale"}
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true",
+                    help="skip the oracle timing (for profiler runs)")
+    ap.add_argument("--reference-rows", type=int, default=1024,
+                    help="rows of the prefill batch per reference (oracle) step")
+    args = ap.parse_args()
+    if args.warmup < 3 and args.impl == "ours" and not args.no_cpu_baseline:
+        print("warning: fewer than 3 warm-up steps", file=sys.stderr)
+    world, rank, local = dist_setup()
+    if world != args.gpus:
+        args.gpus = world if world > 1 else args.gpus
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,199 @@
+/*
+ * rmsnorm_b200.h -- C ABI of the B200 (sm_100a) RMSNorm library.
+ *
+ * Three operators over a dense [T x H] matrix of 16-bit activations (fp16 or
+ * bf16), each accumulating in fp32:
+ *
+ *   rn_rms_norm               out = x / sqrt(mean(x^2) + eps) * weight
+ *   rn_fused_add_rms_norm     residual := x + residual (rounded to the 16-bit
+ *                             dtype and written back), out = rms_norm(residual)
+ *   rn_fused_add_rms_norm_fp8 the fused pass with a per-token dynamic cast to
+ *                             OCP FP8 e4m3fn instead of a 16-bit output
+ *
+ * Sources. The operators and their eligibility rules are those of the AITER
+ * wrappers in "vllm.kernels.aiter_ops": rms_no_var_16bit_only and
+ * rms_add_no_var_16bit_only accept only fp16/bf16 activations, a weight of the
+ * same dtype or None, no variance-size override, and inputs whose flattening
+ * to 2-D is free (flatten_to_2d_is_free). The single-pass residual + RMSNorm
+ * + FP8 fusion is the first kernel of "Custom CUDA kernels juice Llama 3.1
+ * 405B on AMD MI300X, skipping Nvidia lock-in". The pages name the operators
+ * without writing the formula; the library computes textbook RMSNorm (eps
+ * inside the square root, weight applied after normalising).
+ *
+ * Common conventions for every entry point:
+ *
+ *  - Memory. Every data pointer is a DEVICE pointer on the current CUDA
+ *    device. The caller owns and allocates all memory; the library allocates
+ *    nothing, keeps no pointer after returning, and has no global state
+ *    besides rn_force_plan's test override and the thread-local error text.
+ *  - Views. A tensor is described by rn_tensor (pointer, dtype, sizes and
+ *    strides in ELEMENTS). It must flatten to a dense [T x H] matrix for free:
+ *    the last stride is 1 and each leading dimension of size != 1 has the
+ *    stride equal to the product of the sizes after it. This is the
+ *    flatten_to_2d_is_free rule of "vllm.kernels.aiter_ops", applied to 1-D
+ *    and 2-D views as well (so padded 2-D rows are rejected too, matching the
+ *    docstring's "dense 2D inputs" and its rejection of a strided last dim).
+ *    H = sizes[ndim-1], T = numel / H. 1 <= ndim <= RN_MAX_DIMS.
+ *  - weight. NULL (the descriptor pointer) means "no weight" (all ones);
+ *    otherwise a 1-D view of H elements, stride 1, same dtype as x.
+ *  - variance_size must be -1 (None); any other value is rejected with
+ *    RN_ERR_VARIANCE_SIZE, as the AITER predicates reject an override.
+ *  - eps must be finite and >= 0. The kernels use it as the given float.
+ *  - Streams. Work is enqueued on `stream` (a cudaStream_t; NULL = legacy
+ *    default stream) and the call returns without waiting. Validation errors
+ *    return synchronously and launch nothing; a failed launch returns
+ *    RN_ERR_CUDA (text in rn_last_cuda_error()).
+ *  - T == 0 (with a valid H >= 1) is a no-op returning RN_OK; H == 0 is
+ *    RN_ERR_SHAPE.
+ *  - Aliasing. out may be exactly x (same pointer and extent: in place).
+ *    Every other overlap between a written buffer (out, residual, q, scale)
+ *    and any other operand is RN_ERR_ALIAS.
+ *  - Alignment. Data pointers must be aligned to their element size
+ *    (RN_ERR_LAYOUT otherwise). The fast vectorised kernels additionally need
+ *    16-byte aligned 16-bit rows (H % 8 == 0 and 16-byte aligned bases) and an
+ *    8-byte aligned q; other inputs run a correct scalar kernel.
+ *  - Numerics (on the GPU): sum of squares in fp32, inv = 1 / sqrt(ss/H + eps)
+ *    with IEEE sqrt and division, y = (v * w) * inv (the 16-bit product v * w
+ *    is exact in fp32), one rounding to nearest-even to the output type.
+ *    Squares or products beyond the fp32 range (|v| > ~1.8e19, bf16 only)
+ *    are outside the supported input range.
+ */
+#ifndef RMSNORM_B200_H
+#define RMSNORM_B200_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define RN_MAX_DIMS 8
+
+/* Exported symbols (the library is built with hidden default visibility). */
+#if defined(__GNUC__)
+#define RN_API __attribute__((visibility("default")))
+#else
+#define RN_API
+#endif
+
+typedef enum {
+    RN_OK = 0,
+    RN_ERR_NULL = 1,          /* a required descriptor, data, sizes or strides pointer is NULL */
+    RN_ERR_DTYPE = 2,         /* x not fp16/bf16; out/residual dtype != x; q not E4M3; scale not F32 */
+    RN_ERR_WEIGHT_DTYPE = 3,  /* weight dtype != x dtype */
+    RN_ERR_SHAPE = 4,         /* bad ndim, negative size, H == 0, [T x H] mismatch, weight not [H], scale not [T] */
+    RN_ERR_LAYOUT = 5,        /* flattening to dense 2-D is not free, or a pointer misaligned for its dtype */
+    RN_ERR_ALIAS = 6,         /* forbidden overlap between operands */
+    RN_ERR_VARIANCE_SIZE = 7, /* variance_size != -1 */
+    RN_ERR_EPS = 8,           /* eps negative, NaN or infinite */
+    RN_ERR_CUDA = 9,          /* a CUDA runtime call failed */
+    RN_ERR_CONFIG = 10        /* rn_force_plan / rn_plan_launch: unsupported request */
+} rn_status;
+
+typedef enum {
+    RN_F16 = 0,   /* IEEE binary16 */
+    RN_BF16 = 1,  /* bfloat16 */
+    RN_E4M3 = 2,  /* OCP FP8 e4m3fn (1 byte; largest finite 448; NaN = S.1111.111) */
+    RN_F32 = 3    /* IEEE binary32 */
+} rn_dtype;
+
+/* A strided view of caller-owned device memory. Strides are in elements. */
+typedef struct {
+    void* data;
+    int32_t dtype;          /* rn_dtype */
+    int32_t ndim;           /* 1 .. RN_MAX_DIMS */
+    const int64_t* sizes;   /* ndim entries, >= 0 */
+    const int64_t* strides; /* ndim entries, in elements */
+} rn_tensor;
+
+/* rms_norm: out = RNE16(x / sqrt(mean(x^2) + eps) * weight), per row.
+ * out, x: [T x H] fp16/bf16 (same dtype). weight: [H] or NULL.
+ * "vllm.kernels.aiter_ops", rms_no_var_16bit_only. */
+RN_API rn_status rn_rms_norm(const rn_tensor* out, const rn_tensor* x,
+                      const rn_tensor* weight, float eps, int64_t variance_size,
+                      void* stream);
+
+/* fused_add_rms_norm: residual := RNE16(x + residual) (in place), then
+ * out = RNE16(residual / sqrt(mean(residual^2) + eps) * weight), normalising
+ * the rounded values that were written back.
+ * out, x, residual: [T x H], same 16-bit dtype; residual is read and written.
+ * "vllm.kernels.aiter_ops", rms_add_no_var_16bit_only. */
+RN_API rn_status rn_fused_add_rms_norm(const rn_tensor* out, const rn_tensor* x,
+                                const rn_tensor* residual, const rn_tensor* weight,
+                                float eps, int64_t variance_size, void* stream);
+
+/* fused_add_rms_norm_fp8: residual := RNE16(x + residual) (in place); per row
+ * y = residual / sqrt(mean(residual^2) + eps) * weight (fp32, not rounded),
+ * scale[t] = max|y| / 448 (fp32) and q = e4m3fn(round-to-nearest-even,
+ * saturating to +-448)(y / scale). A row whose max|y| is 0 gets scale 0 and
+ * all-zero codes. Dequantise with q * scale[t].
+ * q: [T x H] RN_E4M3 (row-major, 1 byte per element). scale: T elements of
+ * RN_F32 (any shape with numel T, dense). x, residual: as above.
+ * The residual + RMSNorm + FP8 single pass of "Custom CUDA kernels juice
+ * Llama 3.1 405B on AMD MI300X, skipping Nvidia lock-in". */
+RN_API rn_status rn_fused_add_rms_norm_fp8(const rn_tensor* q, const rn_tensor* scale,
+                                    const rn_tensor* x, const rn_tensor* residual,
+                                    const rn_tensor* weight, float eps,
+                                    int64_t variance_size, void* stream);
+
+/* Static text for a status code (never NULL). */
+RN_API const char* rn_status_string(rn_status status);
+
+/* Text of the last RN_ERR_CUDA returned on the calling thread ("" if none). */
+RN_API const char* rn_last_cuda_error(void);
+
+/* ---- launch planning (introspection; no memory is touched) ------------- */
+
+typedef enum { RN_OP_RMS_NORM = 0, RN_OP_FUSED_ADD = 1, RN_OP_FUSED_ADD_FP8 = 2 } rn_op;
+typedef enum { RN_KERNEL_VECTOR = 0, RN_KERNEL_SCALAR = 1 } rn_kernel;
+
+typedef struct {
+    int32_t kernel;             /* rn_kernel */
+    int32_t threads_per_row;    /* threads cooperating on one row */
+    int32_t vectors_per_thread; /* 16-byte vectors each thread holds per row */
+    int32_t rows_per_cta;       /* rows in flight per thread block */
+    int32_t block_threads;      /* threads per block */
+    int32_t smem_bytes;         /* dynamic shared memory per block */
+    int64_t grid;               /* blocks launched */
+} rn_plan;
+
+/* The launch shape the library would use for `op` on a [T x H] problem of
+ * `dtype` (RN_F16/RN_BF16); `vector_ok` says whether the operands meet the
+ * vector kernel's alignment (see Alignment above). Pure host logic: needs no
+ * GPU. Honours rn_force_plan. Returns RN_ERR_SHAPE for H < 1 or T < 0. */
+RN_API rn_status rn_plan_launch(int32_t op, int32_t dtype, int64_t T, int64_t H,
+                         int32_t vector_ok, rn_plan* plan);
+
+/* Dry run: performs every check of the entry point named by `op` (for
+ * RN_OP_RMS_NORM and RN_OP_FUSED_ADD `out_or_q` is `out`; for
+ * RN_OP_FUSED_ADD_FP8 it is `q`; `scale` and `residual` are ignored by the
+ * ops that take none) and returns the status that call would return, without
+ * touching memory, calling CUDA or launching. When it returns RN_OK and the
+ * problem is not empty, `plan` (nullable) receives the launch shape. Pure host
+ * logic: usable without a GPU. */
+RN_API rn_status rn_validate(int32_t op, const rn_tensor* out_or_q, const rn_tensor* scale,
+                      const rn_tensor* x, const rn_tensor* residual, const rn_tensor* weight,
+                      float eps, int64_t variance_size, rn_plan* plan);
+
+/* Test hook: force the vector kernel's (threads_per_row, vectors_per_thread)
+ * for every later call in the process; (0, 0) restores automatic choice.
+ * threads_per_row must be a power of two <= 32 or a multiple of 32 <= 1024,
+ * and vectors_per_thread one of the compiled widths (see
+ * rn_supported_vectors_per_thread); otherwise RN_ERR_CONFIG. A forced shape
+ * that cannot cover a row (threads_per_row * vectors_per_thread * 8 < H) or
+ * exceeds the kernel's block limit falls back to the scalar kernel. Not
+ * thread-safe with concurrent launches; meant for tests and tuning. */
+RN_API rn_status rn_force_plan(int32_t threads_per_row, int32_t vectors_per_thread);
+
+/* Writes up to `cap` compiled vectors_per_thread values into `out` and
+ * returns how many exist. */
+RN_API int32_t rn_supported_vectors_per_thread(int32_t* out, int32_t cap);
+
+/* Library version, "major.minor.patch". */
+RN_API const char* rn_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* RMSNORM_B200_H */

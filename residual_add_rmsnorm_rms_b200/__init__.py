@@ -1,0 +1,232 @@
+"""B200 (sm_100a) RMSNorm library: rms_norm, fused_add_rms_norm and
+fused_add_rms_norm_fp8 over dense 16-bit activations.
+
+This module is a thin ctypes binding over the C ABI declared in
+``include/rmsnorm_b200.h`` (``librmsnorm_b200.so``, built in-tree by
+``python residual_add_rmsnorm_rms_b200/build.py``). It only marshals torch
+tensors into ``rn_tensor`` descriptors and passes the current CUDA stream;
+every step of the computation runs in the library's CUDA kernels. There is no
+CPU or PyTorch fallback: if the shared library is missing, importing this
+package raises.
+
+Operators as wrapped in "vllm.kernels.aiter_ops" (rms_no_var_16bit_only,
+rms_add_no_var_16bit_only, flatten_to_2d_is_free); the fp8 variant is the
+residual + RMSNorm + FP8 single pass of "Custom CUDA kernels juice Llama 3.1
+405B on AMD MI300X, skipping Nvidia lock-in".
+"""
+from __future__ import annotations
+
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "RmsNormError", "rms_norm", "fused_add_rms_norm", "fused_add_rms_norm_fp8",
+    "plan_launch", "validate", "force_plan", "supported_vectors_per_thread", "status_string",
+    "LIB_PATH", "lib", "RnTensor", "RnPlan", "STATUS", "OPS",
+]
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "librmsnorm_b200.so")
+
+STATUS = {
+    0: "RN_OK", 1: "RN_ERR_NULL", 2: "RN_ERR_DTYPE", 3: "RN_ERR_WEIGHT_DTYPE", 4: "RN_ERR_SHAPE",
+    5: "RN_ERR_LAYOUT", 6: "RN_ERR_ALIAS", 7: "RN_ERR_VARIANCE_SIZE", 8: "RN_ERR_EPS",
+    9: "RN_ERR_CUDA", 10: "RN_ERR_CONFIG",
+}
+OPS = {"rms_norm": 0, "fused_add_rms_norm": 1, "fused_add_rms_norm_fp8": 2}
+_DTYPES = {torch.float16: 0, torch.bfloat16: 1, torch.float8_e4m3fn: 2, torch.float32: 3,
+           torch.uint8: 2}
+
+
+class RnTensor(ctypes.Structure):
+    _fields_ = [
+        ("data", ctypes.c_void_p),
+        ("dtype", ctypes.c_int32),
+        ("ndim", ctypes.c_int32),
+        ("sizes", ctypes.POINTER(ctypes.c_int64)),
+        ("strides", ctypes.POINTER(ctypes.c_int64)),
+    ]
+
+
+class RnPlan(ctypes.Structure):
+    _fields_ = [
+        ("kernel", ctypes.c_int32),
+        ("threads_per_row", ctypes.c_int32),
+        ("vectors_per_thread", ctypes.c_int32),
+        ("rows_per_cta", ctypes.c_int32),
+        ("block_threads", ctypes.c_int32),
+        ("smem_bytes", ctypes.c_int32),
+        ("grid", ctypes.c_int64),
+    ]
+
+    def as_dict(self):
+        return {k: getattr(self, k) for k, _ in self._fields_}
+
+
+class RmsNormError(RuntimeError):
+    def __init__(self, status: int, what: str):
+        self.status = status
+        self.name = STATUS.get(status, str(status))
+        super().__init__(f"{what}: {self.name} ({status_string(status)})")
+
+
+def _load():
+    if not os.path.exists(LIB_PATH):
+        raise ImportError(
+            f"{LIB_PATH} is missing: build it with `python residual_add_rmsnorm_rms_b200/build.py` "
+            "(this package has no CPU fallback)")
+    L = ctypes.CDLL(LIB_PATH)
+    P = ctypes.POINTER(RnTensor)
+    F, I64, VP = ctypes.c_float, ctypes.c_int64, ctypes.c_void_p
+    L.rn_rms_norm.argtypes = [P, P, P, F, I64, VP]
+    L.rn_fused_add_rms_norm.argtypes = [P, P, P, P, F, I64, VP]
+    L.rn_fused_add_rms_norm_fp8.argtypes = [P, P, P, P, P, F, I64, VP]
+    for f in (L.rn_rms_norm, L.rn_fused_add_rms_norm, L.rn_fused_add_rms_norm_fp8):
+        f.restype = ctypes.c_int
+    L.rn_status_string.argtypes = [ctypes.c_int]
+    L.rn_status_string.restype = ctypes.c_char_p
+    L.rn_last_cuda_error.argtypes = []
+    L.rn_last_cuda_error.restype = ctypes.c_char_p
+    L.rn_plan_launch.argtypes = [ctypes.c_int32, ctypes.c_int32, I64, I64, ctypes.c_int32,
+                                 ctypes.POINTER(RnPlan)]
+    L.rn_plan_launch.restype = ctypes.c_int
+    L.rn_validate.argtypes = [ctypes.c_int32, P, P, P, P, P, F, I64, ctypes.POINTER(RnPlan)]
+    L.rn_validate.restype = ctypes.c_int
+    L.rn_force_plan.argtypes = [ctypes.c_int32, ctypes.c_int32]
+    L.rn_force_plan.restype = ctypes.c_int
+    L.rn_supported_vectors_per_thread.argtypes = [ctypes.POINTER(ctypes.c_int32), ctypes.c_int32]
+    L.rn_supported_vectors_per_thread.restype = ctypes.c_int32
+    L.rn_version.argtypes = []
+    L.rn_version.restype = ctypes.c_char_p
+    return L
+
+
+lib = _load()
+
+
+def status_string(status: int) -> str:
+    return lib.rn_status_string(int(status)).decode()
+
+
+def describe(t: torch.Tensor | None):
+    """(RnTensor, keepalive) for a tensor; (None, None) for None."""
+    if t is None:
+        return None, None
+    n = t.dim()
+    sizes = (ctypes.c_int64 * max(n, 1))(*t.shape)
+    strides = (ctypes.c_int64 * max(n, 1))(*t.stride())
+    dt = _DTYPES.get(t.dtype, -1)
+    d = RnTensor(t.data_ptr() if t.numel() else 0, dt, n, sizes, strides)
+    return d, (sizes, strides)
+
+
+def _ref(d):
+    return None if d is None else ctypes.byref(d)
+
+
+def _vs(variance_size) -> int:
+    return -1 if variance_size is None else int(variance_size)
+
+
+def _device_and_stream(tensors, stream):
+    dev = None
+    for t in tensors:
+        if t is None:
+            continue
+        if not t.is_cuda:
+            raise ValueError("all operands must be CUDA tensors (the library takes device pointers)")
+        if dev is None:
+            dev = t.device
+        elif t.device != dev:
+            raise ValueError("operands are on different devices")
+    if stream is None:
+        stream = torch.cuda.current_stream(dev)
+    return dev, (stream.cuda_stream if hasattr(stream, "cuda_stream") else stream)
+
+
+def _check(status: int, what: str):
+    if status != 0:
+        err = RmsNormError(status, what)
+        if status == 9:
+            err.args = (err.args[0] + ": " + lib.rn_last_cuda_error().decode(),)
+        raise err
+
+
+def rms_norm(out: torch.Tensor, x: torch.Tensor, weight: torch.Tensor | None, eps: float,
+             variance_size=None, stream=None) -> None:
+    """out = x / sqrt(mean(x^2) + eps) * weight over the last dim (C ABI rn_rms_norm)."""
+    dev, s = _device_and_stream((out, x, weight), stream)
+    do, ko = describe(out)
+    dx, kx = describe(x)
+    dw, kw = describe(weight)
+    with torch.cuda.device(dev):
+        st = lib.rn_rms_norm(_ref(do), _ref(dx), _ref(dw), eps, _vs(variance_size), s)
+    _check(st, "rn_rms_norm")
+
+
+def fused_add_rms_norm(out: torch.Tensor, x: torch.Tensor, residual: torch.Tensor,
+                       weight: torch.Tensor | None, eps: float, variance_size=None,
+                       stream=None) -> None:
+    """residual += x (rounded, in place); out = rms_norm(residual) (C ABI rn_fused_add_rms_norm)."""
+    dev, s = _device_and_stream((out, x, residual, weight), stream)
+    do, ko = describe(out)
+    dx, kx = describe(x)
+    dr, kr = describe(residual)
+    dw, kw = describe(weight)
+    with torch.cuda.device(dev):
+        st = lib.rn_fused_add_rms_norm(_ref(do), _ref(dx), _ref(dr), _ref(dw), eps,
+                                       _vs(variance_size), s)
+    _check(st, "rn_fused_add_rms_norm")
+
+
+def fused_add_rms_norm_fp8(q: torch.Tensor, scale: torch.Tensor, x: torch.Tensor,
+                           residual: torch.Tensor, weight: torch.Tensor | None, eps: float,
+                           variance_size=None, stream=None) -> None:
+    """residual += x (in place); q, scale = per-token e4m3 cast of rms_norm(residual)
+    (C ABI rn_fused_add_rms_norm_fp8). q: float8_e4m3fn (or uint8) [T, H]; scale: float32 [T]."""
+    dev, s = _device_and_stream((q, scale, x, residual, weight), stream)
+    dq, kq = describe(q)
+    dsc, ks = describe(scale)
+    dx, kx = describe(x)
+    dr, kr = describe(residual)
+    dw, kw = describe(weight)
+    with torch.cuda.device(dev):
+        st = lib.rn_fused_add_rms_norm_fp8(_ref(dq), _ref(dsc), _ref(dx), _ref(dr), _ref(dw), eps,
+                                           _vs(variance_size), s)
+    _check(st, "rn_fused_add_rms_norm_fp8")
+
+
+def plan_launch(op: str, dtype: torch.dtype, T: int, H: int, vector_ok: bool = True) -> dict:
+    """The launch shape the library picks (pure host logic; no GPU needed)."""
+    p = RnPlan()
+    st = lib.rn_plan_launch(OPS[op], _DTYPES[dtype], T, H, int(vector_ok), ctypes.byref(p))
+    _check(st, "rn_plan_launch")
+    return p.as_dict()
+
+
+def validate(op: str, out_or_q, x, residual=None, weight=None, eps: float = 1e-6,
+             variance_size=None, scale=None):
+    """Dry run of an entry point on tensor METADATA (no memory is touched, no
+    CUDA call): returns (status_name, plan dict). Works for CPU tensors too."""
+    keep = []
+    descs = []
+    for t in (out_or_q, scale, x, residual, weight):
+        d, k = describe(t)
+        keep.append(k)
+        descs.append(d)
+    p = RnPlan()
+    st = lib.rn_validate(OPS[op], *[_ref(d) for d in descs], eps, _vs(variance_size),
+                         ctypes.byref(p))
+    return STATUS.get(st, str(st)), p.as_dict()
+
+
+def force_plan(threads_per_row: int, vectors_per_thread: int) -> None:
+    """Test/tuning hook: force the vector kernel's shape; (0, 0) restores auto."""
+    _check(lib.rn_force_plan(threads_per_row, vectors_per_thread), "rn_force_plan")
+
+
+def supported_vectors_per_thread() -> list[int]:
+    buf = (ctypes.c_int32 * 64)()
+    n = lib.rn_supported_vectors_per_thread(buf, 64)
+    return list(buf[:n])

@@ -1,0 +1,432 @@
+// rmsnorm_api.cpp -- the C ABI of include/rmsnorm_b200.h: argument
+// validation (the eligibility rules of the AITER wrappers in
+// "vllm.kernels.aiter_ops": 16-bit activations, matching weight dtype or
+// None, no variance-size override, free flattening to dense 2-D), aliasing
+// rules, launch planning and the launch itself. Pure host code.
+#include <cmath>
+#include <cstdint>
+#include <cstdio>
+#include <cstring>
+
+#include <atomic>
+
+#include <cuda_runtime_api.h>
+
+#include "../../include/rmsnorm_b200.h"
+#include "rn_internal.h"
+
+namespace {
+
+thread_local char g_cuda_error[256] = "";
+std::atomic<int> g_force_tpr{0};
+std::atomic<int> g_force_vpt{0};
+
+int elem_size(int32_t dt) {
+    switch (dt) {
+        case RN_F16:
+        case RN_BF16: return 2;
+        case RN_E4M3: return 1;
+        case RN_F32: return 4;
+        default: return 0;
+    }
+}
+
+struct Flat {
+    char* ptr = nullptr;
+    int64_t T = 0, H = 0, numel = 0;
+    int esize = 0;
+    int64_t bytes() const { return numel * esize; }
+};
+
+// flatten_to_2d_is_free ("vllm.kernels.aiter_ops"), applied to every rank:
+// unit last stride; each leading dim of size != 1 has the dense stride.
+rn_status flatten(const rn_tensor* t, Flat* f) {
+    if (t->ndim < 1 || t->ndim > RN_MAX_DIMS) return RN_ERR_SHAPE;
+    if (!t->sizes || !t->strides) return RN_ERR_NULL;
+    const int n = t->ndim;
+    int64_t numel = 1;
+    for (int i = 0; i < n; ++i) {
+        if (t->sizes[i] < 0) return RN_ERR_SHAPE;
+        if (t->sizes[i] != 0 && numel > INT64_MAX / t->sizes[i]) return RN_ERR_SHAPE;
+        numel *= t->sizes[i];
+    }
+    const int64_t H = t->sizes[n - 1];
+    if (H == 0) return RN_ERR_SHAPE;
+    if (numel > 0) {
+        if (t->strides[n - 1] != 1) return RN_ERR_LAYOUT;
+        int64_t expected = H;
+        for (int i = n - 2; i >= 0; --i) {
+            if (t->sizes[i] != 1 && t->strides[i] != expected) return RN_ERR_LAYOUT;
+            expected *= t->sizes[i];
+        }
+    }
+    f->ptr = static_cast<char*>(t->data);
+    f->H = H;
+    f->numel = numel;
+    f->T = numel / H;
+    f->esize = elem_size(t->dtype);
+    return RN_OK;
+}
+
+bool overlap(const Flat& a, const Flat& b) {
+    if (a.bytes() == 0 || b.bytes() == 0) return false;
+    const uintptr_t a0 = reinterpret_cast<uintptr_t>(a.ptr), a1 = a0 + a.bytes();
+    const uintptr_t b0 = reinterpret_cast<uintptr_t>(b.ptr), b1 = b0 + b.bytes();
+    return a0 < b1 && b0 < a1;
+}
+
+bool same_extent(const Flat& a, const Flat& b) { return a.ptr == b.ptr && a.bytes() == b.bytes(); }
+
+bool aligned(const void* p, uintptr_t n) { return (reinterpret_cast<uintptr_t>(p) % n) == 0; }
+
+int clamp_rpc(int rpc, int tpr, int64_t T) {
+    if (rpc < 1) rpc = 1;
+    if (tpr > 32 && rpc > 15) rpc = 15;  // named barriers 1..15, one per row group
+    if (T > 0 && rpc > T) {
+        // Keep sub-warp groups whole-warp: a warp never straddles two CTAs.
+        const int64_t min_rpc = tpr < 32 ? 32 / tpr : 1;
+        rpc = static_cast<int>(T < min_rpc ? min_rpc : T);
+        if (tpr < 32) rpc = static_cast<int>(((rpc + min_rpc - 1) / min_rpc) * min_rpc);
+    }
+    return rpc;
+}
+
+bool vpt_compiled(int vpt) {
+    for (int i = 0; i < rn::kNumVpt; ++i)
+        if (rn::kVptList[i] == vpt) return true;
+    return false;
+}
+
+bool tpr_valid(int tpr) {
+    if (tpr >= 1 && tpr <= 32) return (tpr & (tpr - 1)) == 0;
+    return tpr > 32 && tpr <= 1024 && tpr % 32 == 0;
+}
+
+// Smallest legal threads-per-row that covers nvec vectors at width vpt.
+int tpr_for(int64_t nvec, int vpt) {
+    const int64_t need = (nvec + vpt - 1) / vpt;
+    if (need <= 32) {
+        int t = 1;
+        while (t < need) t <<= 1;
+        return t;
+    }
+    return static_cast<int>(((need + 31) / 32) * 32);
+}
+
+void fill_vector_plan(int tpr, int vpt, int64_t T, rn_plan* p) {
+    // Aim for ~256-thread blocks: several rows per block for narrow rows.
+    int rpc = tpr >= 256 ? 1 : 256 / tpr;
+    rpc = clamp_rpc(rpc, tpr, T);
+    p->kernel = RN_KERNEL_VECTOR;
+    p->threads_per_row = tpr;
+    p->vectors_per_thread = vpt;
+    p->rows_per_cta = rpc;
+    p->block_threads = tpr * rpc;
+    const int wpr = tpr / 32;
+    p->smem_bytes = wpr > 1 ? static_cast<int32_t>(2 * rpc * wpr * sizeof(float) * 2) : 0;
+    p->grid = T > 0 ? (T + rpc - 1) / rpc : 0;
+}
+
+void fill_scalar_plan(int64_t T, rn_plan* p) {
+    p->kernel = RN_KERNEL_SCALAR;
+    p->threads_per_row = 256;
+    p->vectors_per_thread = 0;
+    p->rows_per_cta = 1;
+    p->block_threads = 256;
+    p->smem_bytes = 0;
+    p->grid = T;
+}
+
+// Automatic choice of (threads per row, vectors per thread) for the vector
+// kernel. Candidates cover the row with at most 1/16 idle slots and respect
+// the per-width block limit; among them, many rows favour wide per-thread
+// work (fewer threads per row: fewer cross-warp steps), few rows favour more
+// threads per row (more parallelism and bytes in flight per row).
+bool auto_vector_plan(int64_t T, int64_t H, rn_plan* p) {
+    const int64_t nvec = H / 8;
+    const int64_t kFillThreads = 148LL * 1024;  // one full wave of resident threads
+    int best_tpr = 0, best_vpt = 0;
+    double best_score = -1e300;
+    for (int i = 0; i < rn::kNumVpt; ++i) {
+        const int vpt = rn::kVptList[i];
+        const int tpr = tpr_for(nvec, vpt);
+        if (tpr > rn::max_block_for_vpt(vpt)) continue;
+        const int64_t slots = static_cast<int64_t>(tpr) * vpt;
+        const double idle = static_cast<double>(slots - nvec) / static_cast<double>(slots);
+        if (idle > 1.0 / 16) continue;
+        const double threads = static_cast<double>(T) * tpr;
+        double score;
+        if (threads >= 4.0 * kFillThreads) {
+            // Plenty of rows: prefer 4..8 vectors per thread.
+            score = -(vpt < 4 ? (4 - vpt) : (vpt > 8 ? (vpt - 8) : 0)) * 1.0 - idle * 8;
+        } else {
+            // Few rows: prefer the most threads per row (latency-bound).
+            score = static_cast<double>(tpr) / 1024.0 - idle * 8 - (vpt > 8 ? 1 : 0);
+        }
+        if (score > best_score) {
+            best_score = score;
+            best_tpr = tpr;
+            best_vpt = vpt;
+        }
+    }
+    if (!best_tpr) return false;
+    fill_vector_plan(best_tpr, best_vpt, T, p);
+    return true;
+}
+
+rn_status plan_impl(int64_t T, int64_t H, bool vector_ok, rn_plan* p) {
+    if (H < 1 || T < 0) return RN_ERR_SHAPE;
+    std::memset(p, 0, sizeof *p);
+    if (!vector_ok || H % 8 != 0) {
+        fill_scalar_plan(T, p);
+        return RN_OK;
+    }
+    const int ftpr = g_force_tpr.load(), fvpt = g_force_vpt.load();
+    if (ftpr && fvpt) {
+        const int64_t nvec = H / 8;
+        if (static_cast<int64_t>(ftpr) * fvpt >= nvec && ftpr <= rn::max_block_for_vpt(fvpt)) {
+            fill_vector_plan(ftpr, fvpt, T, p);
+        } else {
+            fill_scalar_plan(T, p);
+        }
+        return RN_OK;
+    }
+    if (!auto_vector_plan(T, H, p)) fill_scalar_plan(T, p);
+    return RN_OK;
+}
+
+struct Common {
+    Flat x, out, res, q, scale, w;
+    bool has_w = false;
+    int dt = 0;
+};
+
+rn_status check_weight(const rn_tensor* weight, int32_t xdt, int64_t H, Common* c) {
+    if (!weight) return RN_OK;
+    if (weight->dtype != xdt) return RN_ERR_WEIGHT_DTYPE;
+    if (weight->ndim != 1) return RN_ERR_SHAPE;
+    Flat f;
+    rn_status st = flatten(weight, &f);
+    if (st != RN_OK) return st;
+    if (f.numel != H) return RN_ERR_SHAPE;
+    c->w = f;
+    c->has_w = true;
+    return RN_OK;
+}
+
+rn_status check_scalars(float eps, int64_t variance_size) {
+    if (variance_size != -1) return RN_ERR_VARIANCE_SIZE;
+    if (!std::isfinite(eps) || eps < 0.f) return RN_ERR_EPS;
+    return RN_OK;
+}
+
+bool is16(int32_t dt) { return dt == RN_F16 || dt == RN_BF16; }
+
+// Descriptor-level checks of one call, in the documented order: NULL
+// descriptors, variance_size and eps, dtypes, weight dtype, shapes and
+// layouts. Fills `c`.
+rn_status check_descriptors(int op, const rn_tensor* o, const rn_tensor* sc, const rn_tensor* x,
+                            const rn_tensor* r, const rn_tensor* w, float eps,
+                            int64_t variance_size, Common* c) {
+    if (!o || !x || (op != rn::kRmsNorm && !r) || (op == rn::kFusedAddFp8 && !sc))
+        return RN_ERR_NULL;
+    rn_status st = check_scalars(eps, variance_size);
+    if (st != RN_OK) return st;
+    if (!is16(x->dtype)) return RN_ERR_DTYPE;
+    if (op != rn::kRmsNorm && r->dtype != x->dtype) return RN_ERR_DTYPE;
+    if (op == rn::kFusedAddFp8) {
+        if (o->dtype != RN_E4M3 || sc->dtype != RN_F32) return RN_ERR_DTYPE;
+    } else if (o->dtype != x->dtype) {
+        return RN_ERR_DTYPE;
+    }
+    if (w && w->dtype != x->dtype) return RN_ERR_WEIGHT_DTYPE;
+    c->dt = x->dtype == RN_BF16 ? rn::kBF16 : rn::kF16;
+    if ((st = flatten(x, &c->x)) != RN_OK) return st;
+    Flat* of = op == rn::kFusedAddFp8 ? &c->q : &c->out;
+    if ((st = flatten(o, of)) != RN_OK) return st;
+    if (of->T != c->x.T || of->H != c->x.H) return RN_ERR_SHAPE;
+    if (op != rn::kRmsNorm) {
+        if ((st = flatten(r, &c->res)) != RN_OK) return st;
+        if (c->res.T != c->x.T || c->res.H != c->x.H) return RN_ERR_SHAPE;
+    }
+    if (op == rn::kFusedAddFp8) {
+        // scale: T fp32 values, dense (e.g. [T] or [T x 1]); unused when T == 0.
+        if (c->x.T > 0) {
+            if ((st = flatten(sc, &c->scale)) != RN_OK) return st;
+            if (c->scale.numel != c->x.T) return RN_ERR_SHAPE;
+        } else if (sc->ndim < 1 || sc->ndim > RN_MAX_DIMS) {
+            return RN_ERR_SHAPE;
+        }
+    }
+    return check_weight(w, x->dtype, c->x.H, c);
+}
+
+// Pointer-level checks (NULL data, element alignment, aliasing) and the plan.
+// Only called for T > 0.
+rn_status check_pointers_and_plan(int op, const Common& c, rn_plan* plan) {
+    const int64_t T = c.x.T, H = c.x.H;
+    if (!c.x.ptr || (op != rn::kFusedAddFp8 && !c.out.ptr)) return RN_ERR_NULL;
+    if (op != rn::kRmsNorm && !c.res.ptr) return RN_ERR_NULL;
+    if (op == rn::kFusedAddFp8 && (!c.q.ptr || !c.scale.ptr)) return RN_ERR_NULL;
+    if (c.has_w && !c.w.ptr) return RN_ERR_NULL;
+    if (!aligned(c.x.ptr, 2) || (c.out.ptr && !aligned(c.out.ptr, 2)) ||
+        (c.res.ptr && !aligned(c.res.ptr, 2)) || (c.has_w && !aligned(c.w.ptr, 2)) ||
+        (c.scale.ptr && !aligned(c.scale.ptr, 4)))
+        return RN_ERR_LAYOUT;
+    // Aliasing: written buffers must not overlap each other or any input,
+    // except out == x exactly (in place) for the 16-bit-output ops.
+    Flat written[3];
+    int nw = 0;
+    if (op == rn::kFusedAddFp8) {
+        written[nw++] = c.res;
+        written[nw++] = c.q;
+        written[nw++] = c.scale;
+    } else {
+        written[nw++] = c.out;
+        if (op == rn::kFusedAdd) written[nw++] = c.res;
+    }
+    for (int i = 0; i < nw; ++i) {
+        for (int j = i + 1; j < nw; ++j)
+            if (overlap(written[i], written[j])) return RN_ERR_ALIAS;
+        const bool is_out = (op != rn::kFusedAddFp8 && i == 0);
+        if (overlap(written[i], c.x) && !(is_out && same_extent(written[i], c.x)))
+            return RN_ERR_ALIAS;
+        if (c.has_w && overlap(written[i], c.w)) return RN_ERR_ALIAS;
+    }
+    if (op != rn::kRmsNorm && overlap(c.res, c.x)) return RN_ERR_ALIAS;
+
+    bool vector_ok = (H % 8 == 0) && aligned(c.x.ptr, 16) && (!c.has_w || aligned(c.w.ptr, 16));
+    if (op != rn::kFusedAddFp8) vector_ok = vector_ok && aligned(c.out.ptr, 16);
+    if (op != rn::kRmsNorm) vector_ok = vector_ok && aligned(c.res.ptr, 16);
+    if (op == rn::kFusedAddFp8) vector_ok = vector_ok && aligned(c.q.ptr, 8);
+    rn_status st = plan_impl(T, H, vector_ok, plan);
+    if (st != RN_OK) return st;
+    if (plan->grid > 0x7fffffffLL) plan->grid = 0x7fffffffLL;  // grid-stride loops cover the rest
+    return RN_OK;
+}
+
+// All checks of one call; *launch_needed is false for the T == 0 no-op.
+rn_status prepare(int op, const rn_tensor* o, const rn_tensor* sc, const rn_tensor* x,
+                  const rn_tensor* r, const rn_tensor* w, float eps, int64_t variance_size,
+                  Common* c, rn_plan* plan, bool* launch_needed) {
+    *launch_needed = false;
+    std::memset(plan, 0, sizeof *plan);
+    rn_status st = check_descriptors(op, o, sc, x, r, w, eps, variance_size, c);
+    if (st != RN_OK) return st;
+    if (c->x.T == 0) return RN_OK;
+    st = check_pointers_and_plan(op, *c, plan);
+    if (st != RN_OK) return st;
+    *launch_needed = true;
+    return RN_OK;
+}
+
+rn_status run(int op, const rn_tensor* o, const rn_tensor* sc, const rn_tensor* x,
+              const rn_tensor* r, const rn_tensor* w, float eps, int64_t variance_size,
+              void* stream) {
+    Common c;
+    rn_plan plan;
+    bool launch_needed;
+    rn_status st = prepare(op, o, sc, x, r, w, eps, variance_size, &c, &plan, &launch_needed);
+    if (st != RN_OK || !launch_needed) return st;
+    rn::Args a;
+    a.x = c.x.ptr;
+    a.residual = c.res.ptr;
+    a.weight = c.has_w ? c.w.ptr : nullptr;
+    a.out = c.out.ptr;
+    a.q = reinterpret_cast<uint8_t*>(c.q.ptr);
+    a.scale = reinterpret_cast<float*>(c.scale.ptr);
+    a.T = c.x.T;
+    a.H = c.x.H;
+    a.eps = eps;
+    const rn::Launch l{plan.kernel, plan.threads_per_row, plan.vectors_per_thread,
+                       plan.rows_per_cta, plan.block_threads, plan.smem_bytes, plan.grid};
+    const cudaError_t e = rn::launch(op, c.dt, a, l, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) {
+        std::snprintf(g_cuda_error, sizeof g_cuda_error, "%s: %s", cudaGetErrorName(e),
+                      cudaGetErrorString(e));
+        return RN_ERR_CUDA;
+    }
+    return RN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+rn_status rn_rms_norm(const rn_tensor* out, const rn_tensor* x, const rn_tensor* weight,
+                      float eps, int64_t variance_size, void* stream) {
+    return run(rn::kRmsNorm, out, nullptr, x, nullptr, weight, eps, variance_size, stream);
+}
+
+rn_status rn_fused_add_rms_norm(const rn_tensor* out, const rn_tensor* x,
+                                const rn_tensor* residual, const rn_tensor* weight, float eps,
+                                int64_t variance_size, void* stream) {
+    return run(rn::kFusedAdd, out, nullptr, x, residual, weight, eps, variance_size, stream);
+}
+
+rn_status rn_fused_add_rms_norm_fp8(const rn_tensor* q, const rn_tensor* scale,
+                                    const rn_tensor* x, const rn_tensor* residual,
+                                    const rn_tensor* weight, float eps, int64_t variance_size,
+                                    void* stream) {
+    return run(rn::kFusedAddFp8, q, scale, x, residual, weight, eps, variance_size, stream);
+}
+
+rn_status rn_validate(int32_t op, const rn_tensor* out_or_q, const rn_tensor* scale,
+                      const rn_tensor* x, const rn_tensor* residual, const rn_tensor* weight,
+                      float eps, int64_t variance_size, rn_plan* plan) {
+    if (op < 0 || op > 2) return RN_ERR_CONFIG;
+    Common c;
+    rn_plan local;
+    bool launch_needed;
+    rn_status st = prepare(op, out_or_q, scale, x, residual, weight, eps, variance_size, &c,
+                           plan ? plan : &local, &launch_needed);
+    return st;
+}
+
+const char* rn_status_string(rn_status s) {
+    switch (s) {
+        case RN_OK: return "ok";
+        case RN_ERR_NULL: return "a required pointer is NULL";
+        case RN_ERR_DTYPE: return "unsupported or mismatched dtype";
+        case RN_ERR_WEIGHT_DTYPE: return "weight dtype differs from the activation dtype";
+        case RN_ERR_SHAPE: return "bad shape (ndim, H == 0, mismatched [T x H], weight or scale size)";
+        case RN_ERR_LAYOUT: return "not a dense unit-stride 2-D view, or misaligned pointer";
+        case RN_ERR_ALIAS: return "forbidden overlap between operands";
+        case RN_ERR_VARIANCE_SIZE: return "variance_size override is not supported";
+        case RN_ERR_EPS: return "eps must be finite and >= 0";
+        case RN_ERR_CUDA: return "CUDA error (see rn_last_cuda_error)";
+        case RN_ERR_CONFIG: return "unsupported launch configuration";
+    }
+    return "unknown status";
+}
+
+const char* rn_last_cuda_error(void) { return g_cuda_error; }
+
+rn_status rn_plan_launch(int32_t op, int32_t dtype, int64_t T, int64_t H, int32_t vector_ok,
+                         rn_plan* plan) {
+    if (!plan) return RN_ERR_NULL;
+    if (op < 0 || op > 2) return RN_ERR_CONFIG;
+    if (!is16(dtype)) return RN_ERR_DTYPE;
+    return plan_impl(T, H, vector_ok != 0, plan);
+}
+
+rn_status rn_force_plan(int32_t threads_per_row, int32_t vectors_per_thread) {
+    if (threads_per_row == 0 && vectors_per_thread == 0) {
+        g_force_tpr.store(0);
+        g_force_vpt.store(0);
+        return RN_OK;
+    }
+    if (!tpr_valid(threads_per_row) || !vpt_compiled(vectors_per_thread)) return RN_ERR_CONFIG;
+    g_force_vpt.store(vectors_per_thread);
+    g_force_tpr.store(threads_per_row);
+    return RN_OK;
+}
+
+int32_t rn_supported_vectors_per_thread(int32_t* out, int32_t cap) {
+    for (int i = 0; i < rn::kNumVpt && i < cap; ++i) out[i] = rn::kVptList[i];
+    return rn::kNumVpt;
+}
+
+const char* rn_version(void) { return "0.1.0"; }
+
+}  // extern "C"

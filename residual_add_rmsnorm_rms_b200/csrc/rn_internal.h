@@ -1,0 +1,48 @@
+// rn_internal.h -- interface between the C-ABI layer (rmsnorm_api.cpp) and
+// the sm_100a kernels (rmsnorm_kernels.cu). Not installed, not part of the ABI.
+#pragma once
+
+#include <cstdint>
+
+#include <cuda_runtime_api.h>
+
+namespace rn {
+
+// Flattened operands of one call. residual is read and written in place.
+struct Args {
+    const void* x;
+    void* residual;      // fused ops only
+    const void* weight;  // nullptr = all ones
+    void* out;           // 16-bit output (rms_norm, fused_add_rms_norm)
+    uint8_t* q;          // e4m3 codes (fp8 op)
+    float* scale;        // per-row scale (fp8 op)
+    int64_t T;
+    int64_t H;
+    float eps;
+};
+
+struct Launch {
+    int kernel;  // 0 = vector, 1 = scalar
+    int tpr;     // threads per row
+    int vpt;     // 16-byte vectors per thread
+    int rpc;     // rows per CTA
+    int block;   // threads per CTA
+    int smem;    // dynamic shared memory bytes
+    int64_t grid;
+};
+
+enum Op { kRmsNorm = 0, kFusedAdd = 1, kFusedAddFp8 = 2 };
+enum Dt { kF16 = 0, kBF16 = 1 };
+
+// Compiled vectors-per-thread widths of the vector kernel, ascending.
+constexpr int kVptList[] = {1, 2, 3, 4, 5, 6, 7, 8, 10, 12, 14, 15, 16};
+constexpr int kNumVpt = sizeof(kVptList) / sizeof(kVptList[0]);
+
+// Largest block the vector kernel of a given width is compiled for (its
+// __launch_bounds__), which bounds the registers it may use per thread.
+constexpr int max_block_for_vpt(int vpt) { return vpt <= 4 ? 1024 : (vpt <= 8 ? 512 : 256); }
+
+// Enqueues one launch; returns the CUDA error of the launch itself.
+cudaError_t launch(int op, int dtype, const Args& a, const Launch& l, cudaStream_t s);
+
+}  // namespace rn

@@ -1,0 +1,269 @@
+"""Host-side tests of the C ABI (CPU only: nothing here launches a kernel).
+
+* the shared library loads and exports every function include/rmsnorm_b200.h
+  declares;
+* argument validation (rn_validate, the dry run that performs exactly the
+  checks of the real entry points) accepts and rejects the layouts of
+  flatten_to_2d_is_free ("vllm.kernels.aiter_ops") and the dtype /
+  variance-size rules of rms_no_var_16bit_only and rms_add_no_var_16bit_only;
+* the launch planner's invariants.
+The real entry points are also called, but only with arguments that fail
+validation (so they return before any CUDA call).
+"""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+import torch
+
+import residual_add_rmsnorm_rms_b200 as rn
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "rmsnorm_b200.h")
+BF, F16 = torch.bfloat16, torch.float16
+
+
+def header_functions():
+    src = open(HEADER).read()
+    return sorted(set(re.findall(r"^RN_API\s+[\w\s\*]+?\b(rn_\w+)\s*\(", src, flags=re.M)))
+
+
+def test_header_declares_the_three_operators():
+    names = header_functions()
+    for op in ("rn_rms_norm", "rn_fused_add_rms_norm", "rn_fused_add_rms_norm_fp8"):
+        assert op in names
+
+
+def test_library_exports_every_declared_symbol():
+    names = header_functions()
+    assert len(names) >= 10
+    for n in names:
+        assert hasattr(rn.lib, n), n
+    out = subprocess.run(["nm", "-D", "--defined-only", rn.LIB_PATH], capture_output=True,
+                         text=True, check=True).stdout
+    exported = set(re.findall(r"\sT\s+(\w+)$", out, flags=re.M))
+    assert set(names) <= exported
+    # nothing else leaks out of the library under the rn_ prefix
+    assert {e for e in exported if e.startswith("rn_")} == set(names)
+
+
+def test_library_targets_sm100a_only():
+    out = subprocess.run(["cuobjdump", "--list-elf", rn.LIB_PATH], capture_output=True, text=True)
+    if out.returncode != 0:
+        pytest.skip("cuobjdump unavailable")
+    archs = set(re.findall(r"sm_(\d+a?)", out.stdout))
+    assert archs == {"100a"}, archs
+
+
+def V(op, *args, **kw):
+    return rn.validate(op, *args, **kw)[0]
+
+
+def VR(out, x, weight=None, **kw):
+    """rms_norm dry run (it takes no residual)."""
+    return rn.validate("rms_norm", out, x, None, weight, **kw)[0]
+
+
+def t(shape, dtype=BF, **kw):
+    return torch.empty(shape, dtype=dtype, **kw)
+
+
+H = 256
+
+
+@pytest.mark.parametrize("op", ["rms_norm", "fused_add_rms_norm"])
+def test_flatten_to_2d_is_free_cases(op):
+    def call(x):
+        out = torch.empty_like(x, memory_format=torch.contiguous_format) if x.is_contiguous() \
+            else torch.empty(x.shape, dtype=x.dtype)
+        res = torch.empty(x.shape, dtype=x.dtype) if op != "rms_norm" else None
+        return V(op, out, x, res)
+
+    # contiguous N-D: accepted
+    assert call(t((2, 3, H))) == "RN_OK"
+    assert call(t((H,))) == "RN_OK"  # 1-D: a single row
+    # transposed leading dims: reshape would copy -> rejected
+    assert call(t((3, 2, H)).transpose(0, 1)) == "RN_ERR_LAYOUT"
+    # size-1 dims may carry any stride
+    x = t((4 * H,)).as_strided((4, 1, H), (H, 7, 1))
+    assert call(x) == "RN_OK"
+    # strided last dim: flattens without a copy but not densely -> rejected
+    assert call(t((4, 2 * H))[:, ::2]) == "RN_ERR_LAYOUT"
+    # padded rows: rejected for > 2-D and (this library's reading) for 2-D
+    assert call(t((2, 4, H + 8))[:, :, :H]) == "RN_ERR_LAYOUT"
+    assert call(t((4, H + 8))[:, :H]) == "RN_ERR_LAYOUT"
+    # degenerate shapes
+    assert call(t((0, H))) == "RN_OK"  # T == 0: a no-op
+    assert call(t((4, 0))) == "RN_ERR_SHAPE"  # H == 0
+    assert call(torch.tensor(1.0, dtype=BF)) == "RN_ERR_SHAPE"  # 0-d
+
+
+def test_dtype_and_weight_rules():
+    x = t((4, H))
+    assert VR(t((4, H)), x, None) == "RN_OK"
+    assert VR(t((4, H), F16), t((4, H), F16), t((H,), F16)) == "RN_OK"
+    assert VR(t((4, H), torch.float32), t((4, H), torch.float32), None) == "RN_ERR_DTYPE"
+    assert VR(t((4, H), F16), x, None) == "RN_ERR_DTYPE"  # out dtype != x
+    assert VR(t((4, H)), x, t((H,), F16)) == "RN_ERR_WEIGHT_DTYPE"
+    assert VR(t((4, H)), x, t((H,), torch.float32)) == "RN_ERR_WEIGHT_DTYPE"
+    assert VR(t((4, H)), x, t((H + 1,))) == "RN_ERR_SHAPE"
+    assert VR(t((4, H)), x, t((1, H))) == "RN_ERR_SHAPE"
+    assert VR(t((4, H)), x, t((2 * H,))[::2]) == "RN_ERR_LAYOUT"
+    assert V("fused_add_rms_norm", t((4, H)), x, t((4, H), F16), None) == "RN_ERR_DTYPE"
+    assert V("fused_add_rms_norm", t((4, H)), x, t((4, H + 8)), None) == "RN_ERR_SHAPE"
+    assert V("fused_add_rms_norm", t((4, H)), x, t((5, H)), None) == "RN_ERR_SHAPE"
+    # N-D views of matching [T x H] flatten alike
+    assert V("fused_add_rms_norm", t((2, 2, H)), x, t((4, 1, H)), None) == "RN_OK"
+
+
+def test_variance_size_and_eps():
+    x = t((4, H))
+    for op, res in (("rms_norm", None), ("fused_add_rms_norm", t((4, H)))):
+        assert V(op, t((4, H)), x, res, variance_size=H) == "RN_ERR_VARIANCE_SIZE"
+        assert V(op, t((4, H)), x, res, variance_size=0) == "RN_ERR_VARIANCE_SIZE"
+        assert V(op, t((4, H)), x, res, variance_size=None) == "RN_OK"
+        for eps in (-1e-6, float("nan"), float("inf")):
+            assert V(op, t((4, H)), x, res, eps=eps) == "RN_ERR_EPS"
+        assert V(op, t((4, H)), x, res, eps=0.0) == "RN_OK"
+
+
+def test_fp8_operands():
+    x, r = t((4, H)), t((4, H))
+    q, s = t((4, H), torch.float8_e4m3fn), t((4,), torch.float32)
+    assert V("fused_add_rms_norm_fp8", q, x, r, None, scale=s) == "RN_OK"
+    assert V("fused_add_rms_norm_fp8", t((4, H), torch.uint8), x, r, None, scale=s) == "RN_OK"
+    assert V("fused_add_rms_norm_fp8", q, x, r, None, scale=t((4, 1), torch.float32)) == "RN_OK"
+    assert V("fused_add_rms_norm_fp8", t((4, H)), x, r, None, scale=s) == "RN_ERR_DTYPE"
+    assert V("fused_add_rms_norm_fp8", q, x, r, None, scale=t((4,), BF)) == "RN_ERR_DTYPE"
+    assert V("fused_add_rms_norm_fp8", q, x, r, None, scale=t((5,), torch.float32)) == "RN_ERR_SHAPE"
+    assert V("fused_add_rms_norm_fp8", q, x, r, None, scale=t((8,), torch.float32)[::2]) == "RN_ERR_LAYOUT"
+    assert V("fused_add_rms_norm_fp8", q, x, r, None, scale=None) == "RN_ERR_NULL"
+    assert V("fused_add_rms_norm_fp8", t((4, H + 8), torch.float8_e4m3fn)[:, :H], x, r, None,
+             scale=s) == "RN_ERR_LAYOUT"
+
+
+def test_aliasing_rules():
+    buf = t((8, H))
+    x = buf[:4]
+    # out == x exactly: in place, allowed
+    assert VR(x, x, None) == "RN_OK"
+    assert V("fused_add_rms_norm", x, x, t((4, H)), None) == "RN_OK"
+    # out overlapping x partially
+    assert VR(buf[2:6], x, None) == "RN_ERR_ALIAS"
+    # residual aliasing x, or out aliasing residual
+    r = t((4, H))
+    assert V("fused_add_rms_norm", t((4, H)), x, x, None) == "RN_ERR_ALIAS"
+    assert V("fused_add_rms_norm", r, x, r, None) == "RN_ERR_ALIAS"
+    # weight inside a written buffer
+    out = t((4, H))
+    assert VR(out, x, out[0]) == "RN_ERR_ALIAS"
+    # weight inside x is read-only data: allowed when x is not written
+    assert VR(t((4, H)), x, x[0]) == "RN_OK"
+    # fp8: q/scale overlapping inputs or each other
+    big = t((16, H))
+    q8 = big.view(torch.uint8)[:2].reshape(4, H)  # the bytes of bf16 rows 0-1
+    assert V("fused_add_rms_norm_fp8", q8, big[8:12], big[12:16], None,
+             scale=t((4,), torch.float32)) == "RN_OK"
+    qx = big.view(torch.uint8)[4:6].reshape(4, H)  # inside x = rows 4-7
+    assert V("fused_add_rms_norm_fp8", qx, big[4:8], big[12:16], None,
+             scale=t((4,), torch.float32)) == "RN_ERR_ALIAS"
+    sc = big[12].view(torch.float32)[:4]
+    assert V("fused_add_rms_norm_fp8", q8, big[8:12], big[12:16], None, scale=sc) == "RN_ERR_ALIAS"
+
+
+def _raw_desc(ptr, shape, strides, dtype=1):
+    n = len(shape)
+    sizes = (ctypes.c_int64 * n)(*shape)
+    strd = (ctypes.c_int64 * n)(*strides)
+    return rn.RnTensor(ptr, dtype, n, sizes, strd), (sizes, strd)
+
+
+def test_null_and_misaligned_pointers_never_launch():
+    # data NULL with T > 0
+    d0, k0 = _raw_desc(0, (4, H), (H, 1))
+    d1, k1 = _raw_desc(0x10000, (4, H), (H, 1))
+    plan = rn.RnPlan()
+    assert rn.lib.rn_validate(0, ctypes.byref(d1), None, ctypes.byref(d0), None, None, 1e-6, -1,
+                              ctypes.byref(plan)) == 1
+    # misaligned (odd byte address) 16-bit data
+    dm, km = _raw_desc(0x10001, (4, H), (H, 1))
+    assert rn.lib.rn_validate(0, ctypes.byref(d1), None, ctypes.byref(dm), None, None, 1e-6, -1,
+                              None) == 5
+    # NULL descriptors on the real entry points return before any CUDA call
+    assert rn.lib.rn_rms_norm(None, ctypes.byref(d1), None, 1e-6, -1, None) == 1
+    assert rn.lib.rn_fused_add_rms_norm(ctypes.byref(d1), ctypes.byref(d1), None, None, 1e-6, -1,
+                                        None) == 1
+    assert rn.lib.rn_fused_add_rms_norm_fp8(None, None, ctypes.byref(d1), ctypes.byref(d1), None,
+                                            1e-6, -1, None) == 1
+    # and so do the other validation failures
+    assert rn.lib.rn_rms_norm(ctypes.byref(d1), ctypes.byref(d1), None, 1e-6, 3, None) == 7
+    assert rn.lib.rn_rms_norm(ctypes.byref(d1), ctypes.byref(d1), None, -1.0, -1, None) == 8
+
+
+def test_binding_rejects_cpu_tensors():
+    x = t((4, H))
+    with pytest.raises(ValueError):
+        rn.rms_norm(torch.empty_like(x), x, None, 1e-6)
+
+
+def test_alignment_selects_kernel():
+    x = t((4, 4096 + 16))
+    xs = x[:, 1:4097]  # not a dense view -> layout error
+    assert VR(t((4, 4096)), xs, None) == "RN_ERR_LAYOUT"
+    flat = t((4 * 4096 + 1,))
+    xo = flat[1:].view(4, 4096)  # dense but 2-byte (not 16-byte) aligned
+    st, plan = rn.validate("rms_norm", t((4, 4096)), xo)
+    assert st == "RN_OK" and plan["kernel"] == 1  # scalar kernel
+    st, plan = rn.validate("rms_norm", t((4, 4096)), t((4, 4096)))
+    assert st == "RN_OK" and plan["kernel"] == 0
+    st, plan = rn.validate("rms_norm", t((4, 1004)), t((4, 1004)))  # H % 8 != 0
+    assert st == "RN_OK" and plan["kernel"] == 1
+
+
+SWEEP_T = (1, 8, 16, 64, 256, 4096, 8192, 32768, 65536)
+SWEEP_H = (512, 2048, 3840, 4096, 5120, 7168, 8192, 16384)
+
+
+@pytest.mark.parametrize("op", list(rn.OPS))
+def test_planner_invariants(op):
+    for T in SWEEP_T:
+        for Hh in SWEEP_H:
+            p = rn.plan_launch(op, BF, T, Hh)
+            assert p["kernel"] == 0, (T, Hh)
+            tpr, vpt, rpc = p["threads_per_row"], p["vectors_per_thread"], p["rows_per_cta"]
+            assert tpr * vpt * 8 >= Hh
+            assert tpr * vpt * 8 - Hh < Hh  # at most one idle slot per used slot
+            assert p["block_threads"] == tpr * rpc
+            assert p["block_threads"] % 32 == 0 and p["block_threads"] <= 1024
+            if tpr > 32:
+                assert tpr % 32 == 0 and rpc <= 15
+            else:
+                assert 32 % tpr == 0
+            assert p["grid"] * rpc >= T
+            assert vpt in rn.supported_vectors_per_thread()
+    # the scalar kernel beyond the vector kernel's reach
+    assert rn.plan_launch(op, BF, 4, 1 << 17)["kernel"] == 1
+
+
+def test_force_plan_hook():
+    with pytest.raises(rn.RmsNormError):
+        rn.force_plan(48, 4)  # not a power of two <= 32 nor a multiple of 32
+    with pytest.raises(rn.RmsNormError):
+        rn.force_plan(64, 9)  # width not compiled
+    try:
+        rn.force_plan(32, 16)
+        p = rn.plan_launch("fused_add_rms_norm", BF, 100, 4096)
+        assert (p["threads_per_row"], p["vectors_per_thread"]) == (32, 16)
+        # a forced shape too small for the row falls back to the scalar kernel
+        assert rn.plan_launch("fused_add_rms_norm", BF, 100, 8192)["kernel"] == 1
+    finally:
+        rn.force_plan(0, 0)
+    assert rn.plan_launch("fused_add_rms_norm", BF, 100, 4096)["kernel"] == 0
+
+
+def test_status_strings():
+    for code, name in rn.STATUS.items():
+        assert rn.status_string(code)
+    assert rn.status_string(999) == "unknown status"

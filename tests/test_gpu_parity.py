@@ -1,0 +1,91 @@
+"""GPU parity: every operator through the C ABI against the fp64 CPU oracle,
+on the seeded workloads of ``synth`` (bit-exact residual, <= 1 ulp 16-bit
+outputs, <= 1 e4m3 code on <= 0.1 % of elements, scales within 1e-6).
+
+Full comparisons where the oracle finishes in seconds; for the large sweep
+cells, the inputs are drawn on the GPU and a row sample (first, last, evenly
+spaced and random rows) is compared, in the same launch configuration the
+benchmark uses (the automatic plan).
+"""
+import numpy as np
+import pytest
+import torch
+
+import synth
+import residual_add_rmsnorm_rms_b200 as rn
+from tests.gpu_util import DT, compare, gpu_run, oracle_run, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.fail("GPU tests need a CUDA device")
+    rn.force_plan(0, 0)
+
+
+def _full(op, wl, with_weight=True):
+    dev = "cuda"
+    x = wl.x.to(dev)
+    r = None if wl.residual is None else wl.residual.to(dev).clone()
+    w = wl.weight.to(dev) if with_weight else None
+    got = gpu_run(op, x, r, w, wl.eps)
+    torch.cuda.synchronize()
+    want = oracle_run(op, wl.x, wl.residual, wl.weight if with_weight else None, wl.eps,
+                      DT[wl.dtype])
+    return compare(op, got, want, DT[wl.dtype])
+
+
+@pytest.mark.parametrize("with_weight", [True, False])
+def test_small_rms_norm(with_weight):
+    """rms_norm, bf16, x [8 x 512] ~ N(0,1), eps 1e-6, seed 0."""
+    wl = synth.make_inputs("small", "rms_norm", "bf16", 8, 512)
+    assert wl.seed == 0
+    _full("rms_norm", wl, with_weight)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
+@pytest.mark.parametrize("T", synth.DECODE_T)
+def test_decode_fused(T, dtype):
+    """fused_add_rms_norm, [T x 4096], x ~ N(0,1), residual ~ N(0,4), eps 1e-5."""
+    wl = synth.make_inputs("decode", "fused_add_rms_norm", dtype, T, 4096)
+    _full("fused_add_rms_norm", wl)
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
+def test_outlier_fp8(dtype):
+    """fused_add_rms_norm_fp8, [64 x 16384], 1 % outlier channels x50 (bf16 is
+    the named workload; fp16 is an extra)."""
+    wl = synth.make_inputs("outlier", "fused_add_rms_norm_fp8", dtype, 64, 16384)
+    stats = _full("fused_add_rms_norm_fp8", wl)
+    print(dtype, stats)
+
+
+@pytest.mark.parametrize("op", ["fused_add_rms_norm", "fused_add_rms_norm_fp8"])
+def test_prefill(op):
+    """[8192 x 3840] bf16, x ~ Student-t(3) clipped to +-1e3, residual ~
+    N(0,16): both outputs (bf16 and fp8), each from a fresh residual copy.
+    This is the benchmark's workload, in its launch configuration."""
+    wl = synth.make_inputs("prefill", op, "bf16", 8192, 3840)
+    stats = _full(op, wl)
+    print(op, stats)
+
+
+@pytest.mark.parametrize("H", synth.SWEEP_H)
+@pytest.mark.parametrize("T", synth.SWEEP_T)
+@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
+@pytest.mark.parametrize("op", ["rms_norm", "fused_add_rms_norm", "fused_add_rms_norm_fp8"])
+def test_sweep(op, dtype, T, H):
+    """Bandwidth-sweep cells: inputs drawn on the GPU, a row sample checked."""
+    wl = synth.make_inputs("sweep", op, dtype, T, H, device="cuda")
+    rows = sample_rows(T)
+    ridx = torch.from_numpy(rows).cuda()
+    x_s = wl.x.index_select(0, ridx).cpu()
+    r_s = None if wl.residual is None else wl.residual.index_select(0, ridx).cpu()
+    got = gpu_run(op, wl.x, wl.residual, wl.weight, wl.eps)
+    got = {k: (v.index_select(0, ridx) if v.dim() and v.shape[0] == T else v) for k, v in got.items()}
+    torch.cuda.synchronize()
+    want = oracle_run(op, x_s, r_s, wl.weight.cpu(), wl.eps, dtype)
+    compare(op, got, want, dtype)
+    del wl, got

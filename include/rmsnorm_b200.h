@@ -145,15 +145,21 @@ RN_API const char* rn_last_cuda_error(void);
 /* ---- launch planning (introspection; no memory is touched) ------------- */
 
 typedef enum { RN_OP_RMS_NORM = 0, RN_OP_FUSED_ADD = 1, RN_OP_FUSED_ADD_FP8 = 2 } rn_op;
-typedef enum { RN_KERNEL_VECTOR = 0, RN_KERNEL_SCALAR = 1 } rn_kernel;
+/* Kernels: VECTOR keeps each row in registers (a group of threads per row);
+ * STAGED is persistent and streams whole rows into a shared-memory ring with
+ * bulk asynchronous copies (one block per row at a time); SCALAR handles
+ * unaligned or ragged rows. */
+typedef enum { RN_KERNEL_VECTOR = 0, RN_KERNEL_SCALAR = 1, RN_KERNEL_STAGED = 2 } rn_kernel;
 
 typedef struct {
     int32_t kernel;             /* rn_kernel */
     int32_t threads_per_row;    /* threads cooperating on one row */
-    int32_t vectors_per_thread; /* 16-byte vectors each thread holds per row */
-    int32_t rows_per_cta;       /* rows in flight per thread block */
+    int32_t vectors_per_thread; /* VECTOR: 16-byte vectors each thread holds per row; else 0 */
+    int32_t rows_per_cta;       /* rows a block works on at once */
     int32_t block_threads;      /* threads per block */
     int32_t smem_bytes;         /* dynamic shared memory per block */
+    int32_t stages;             /* STAGED: depth of the shared-memory row ring; else 0 */
+    int32_t ctas_per_sm;        /* STAGED: resident blocks per SM the grid is sized for; else 0 */
     int64_t grid;               /* blocks launched */
 } rn_plan;
 
@@ -184,6 +190,20 @@ RN_API rn_status rn_validate(int32_t op, const rn_tensor* out_or_q, const rn_ten
  * exceeds the kernel's block limit falls back to the scalar kernel. Not
  * thread-safe with concurrent launches; meant for tests and tuning. */
 RN_API rn_status rn_force_plan(int32_t threads_per_row, int32_t vectors_per_thread);
+
+/* Test hook: force the STAGED kernel with `ctas_per_sm` resident blocks per SM
+ * (1, 2 or 4), `stages` ring slots (>= 2) and `threads` per block (a multiple
+ * of 32, 32..1024) for every later call with 16-byte-aligned operands; a
+ * shape whose shared memory exceeds the per-block limit falls back to the
+ * automatic choice. (0, 0, 0) restores automatic choice; a forced STAGED shape
+ * takes precedence over rn_force_plan. Not thread-safe with concurrent
+ * launches; meant for tests and tuning. */
+RN_API rn_status rn_force_staged(int32_t ctas_per_sm, int32_t stages, int32_t threads);
+
+/* Reads and clears the device-side error flags of the current device:
+ * bit 0 = a bounded wait inside the STAGED kernel timed out (some rows of
+ * that call were not written). Synchronises with the device. */
+RN_API rn_status rn_device_errors(uint32_t* flags);
 
 /* Writes up to `cap` compiled vectors_per_thread values into `out` and
  * returns how many exist. */

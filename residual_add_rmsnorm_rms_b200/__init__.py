@@ -23,7 +23,7 @@ import torch
 
 __all__ = [
     "RmsNormError", "rms_norm", "fused_add_rms_norm", "fused_add_rms_norm_fp8",
-    "plan_launch", "validate", "force_plan", "supported_vectors_per_thread", "status_string",
+    "plan_launch", "validate", "force_plan", "force_staged", "device_errors", "supported_vectors_per_thread", "status_string",
     "LIB_PATH", "lib", "RnTensor", "RnPlan", "STATUS", "OPS",
 ]
 
@@ -57,6 +57,8 @@ class RnPlan(ctypes.Structure):
         ("rows_per_cta", ctypes.c_int32),
         ("block_threads", ctypes.c_int32),
         ("smem_bytes", ctypes.c_int32),
+        ("stages", ctypes.c_int32),
+        ("ctas_per_sm", ctypes.c_int32),
         ("grid", ctypes.c_int64),
     ]
 
@@ -95,6 +97,10 @@ def _load():
     L.rn_validate.restype = ctypes.c_int
     L.rn_force_plan.argtypes = [ctypes.c_int32, ctypes.c_int32]
     L.rn_force_plan.restype = ctypes.c_int
+    L.rn_force_staged.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32]
+    L.rn_force_staged.restype = ctypes.c_int
+    L.rn_device_errors.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
+    L.rn_device_errors.restype = ctypes.c_int
     L.rn_supported_vectors_per_thread.argtypes = [ctypes.POINTER(ctypes.c_int32), ctypes.c_int32]
     L.rn_supported_vectors_per_thread.restype = ctypes.c_int32
     L.rn_version.argtypes = []
@@ -224,6 +230,18 @@ def validate(op: str, out_or_q, x, residual=None, weight=None, eps: float = 1e-6
 def force_plan(threads_per_row: int, vectors_per_thread: int) -> None:
     """Test/tuning hook: force the vector kernel's shape; (0, 0) restores auto."""
     _check(lib.rn_force_plan(threads_per_row, vectors_per_thread), "rn_force_plan")
+
+
+def force_staged(ctas_per_sm: int, stages: int, threads: int) -> None:
+    """Test/tuning hook: force the staged kernel's shape; (0, 0, 0) restores auto."""
+    _check(lib.rn_force_staged(ctas_per_sm, stages, threads), "rn_force_staged")
+
+
+def device_errors() -> int:
+    """Reads and clears the current device's kernel error flags (0 = none)."""
+    v = ctypes.c_uint32(0)
+    _check(lib.rn_device_errors(ctypes.byref(v)), "rn_device_errors")
+    return int(v.value)
 
 
 def supported_vectors_per_thread() -> list[int]:

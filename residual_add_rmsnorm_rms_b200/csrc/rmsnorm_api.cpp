@@ -4,11 +4,13 @@
 // None, no variance-size override, free flattening to dense 2-D), aliasing
 // rules, launch planning and the launch itself. Pure host code.
 #include <cmath>
+#include <cstdlib>
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
 
 #include <atomic>
+#include <initializer_list>
 
 #include <cuda_runtime_api.h>
 
@@ -20,6 +22,10 @@ namespace {
 thread_local char g_cuda_error[256] = "";
 std::atomic<int> g_force_tpr{0};
 std::atomic<int> g_force_vpt{0};
+std::atomic<int> g_force_staged_c{0};
+std::atomic<int> g_force_staged_s{0};
+std::atomic<int> g_force_staged_t{0};
+constexpr int kDefaultSms = 148;  // B200; dry runs (no device) plan for it
 
 int elem_size(int32_t dt) {
     switch (dt) {
@@ -127,6 +133,59 @@ void fill_vector_plan(int tpr, int vpt, int64_t T, rn_plan* p) {
     p->grid = T > 0 ? (T + rpc - 1) / rpc : 0;
 }
 
+int64_t round_up(int64_t v, int64_t m) { return (v + m - 1) / m * m; }
+
+int64_t staged_smem(int op, int64_t H, int stages) {
+    const int nin = op == rn::kRmsNorm ? 1 : 2;
+    return stages * nin * round_up(2 * H, 128) + stages * 8 + 32 * 8;
+}
+
+// Fills a STAGED plan for (c CTAs per SM, S stages, threads); false if it
+// does not fit the per-block shared memory.
+bool fill_staged_plan(int op, int64_t T, int64_t H, int c, int S, int threads, int num_sms,
+                      rn_plan* p) {
+    const int64_t smem = staged_smem(op, H, S);
+    if (S < 2 || smem > rn::kStagedMaxSmem || threads < 32 || threads > 1024 || threads % 32)
+        return false;
+    p->kernel = RN_KERNEL_STAGED;
+    p->threads_per_row = threads;
+    p->vectors_per_thread = 0;
+    p->rows_per_cta = 1;
+    p->block_threads = threads;
+    p->smem_bytes = static_cast<int32_t>(smem);
+    p->stages = S;
+    p->ctas_per_sm = c;
+    const int64_t g = static_cast<int64_t>(c) * num_sms;
+    p->grid = T < g ? T : g;
+    return true;
+}
+
+// Automatic STAGED shape: as many resident CTAs per SM (4, 2, 1) as leave
+// each at least 3 ring stages (2 for the widest rows) inside the per-SM
+// shared-memory budget, up to 8 stages; about two 16-byte vectors per thread
+// per pass.
+bool auto_staged_plan(int op, int64_t T, int64_t H, int num_sms, rn_plan* p) {
+    const int nin = op == rn::kRmsNorm ? 1 : 2;
+    const int64_t stage = nin * round_up(2 * H, 128);
+    const int64_t nvec = H / 8;
+    for (int c : {4, 2, 1}) {
+        const int64_t per_cta = rn::kStagedSmemPerSm / c - 1024;
+        int64_t S = per_cta / stage;
+        if (S > 8) S = 8;
+        if (S >= 3 || (c == 1 && S >= 2)) {
+            int64_t threads = round_up((nvec + 1) / 2, 32);
+            // <= 1024 resident threads per SM: at ~48 registers per thread
+            // that is what the 64K-register file holds for c blocks.
+            const int64_t cap = 1024 / c;
+            if (threads > cap) threads = cap;
+            if (threads < 64) threads = 64;
+            return fill_staged_plan(op, T, H, c, static_cast<int>(S), static_cast<int>(threads),
+                                    num_sms, p);
+        }
+    }
+    return false;
+}
+
 void fill_scalar_plan(int64_t T, rn_plan* p) {
     p->kernel = RN_KERNEL_SCALAR;
     p->threads_per_row = 256;
@@ -153,13 +212,17 @@ bool auto_vector_plan(int64_t T, int64_t H, rn_plan* p) {
         if (tpr > rn::max_block_for_vpt(vpt)) continue;
         const int64_t slots = static_cast<int64_t>(tpr) * vpt;
         const double idle = static_cast<double>(slots - nvec) / static_cast<double>(slots);
-        if (idle > 1.0 / 16) continue;
         const double threads = static_cast<double>(T) * tpr;
         double score;
         if (threads >= 4.0 * kFillThreads) {
-            // Plenty of rows: prefer 4..8 vectors per thread.
-            score = -(vpt < 4 ? (4 - vpt) : (vpt > 8 ? (vpt - 8) : 0)) * 1.0 - idle * 8;
+            // Plenty of rows: 4 vectors per thread keeps the kernel at <= 64
+            // registers (32 resident warps per SM) with 64 bytes of loads in
+            // flight per thread per tensor; measured best on B200 for H in
+            // 3840..16384 even with up to 1/8 idle slots.
+            if (idle > 1.0 / 8) continue;
+            score = -std::abs(vpt - 4) * 1.0 - idle * 4;
         } else {
+            if (idle > 1.0 / 16) continue;
             // Few rows: prefer the most threads per row (latency-bound).
             score = static_cast<double>(tpr) / 1024.0 - idle * 8 - (vpt > 8 ? 1 : 0);
         }
@@ -174,13 +237,17 @@ bool auto_vector_plan(int64_t T, int64_t H, rn_plan* p) {
     return true;
 }
 
-rn_status plan_impl(int64_t T, int64_t H, bool vector_ok, rn_plan* p) {
+rn_status plan_impl(int op, int64_t T, int64_t H, bool vector_ok, int num_sms, rn_plan* p) {
     if (H < 1 || T < 0) return RN_ERR_SHAPE;
     std::memset(p, 0, sizeof *p);
     if (!vector_ok || H % 8 != 0) {
         fill_scalar_plan(T, p);
         return RN_OK;
     }
+    const int fc = g_force_staged_c.load(), fs = g_force_staged_s.load(),
+              ft = g_force_staged_t.load();
+    if (fc && fs && ft && fill_staged_plan(op, T, H, fc, fs, ft, num_sms, p)) return RN_OK;
+    std::memset(p, 0, sizeof *p);
     const int ftpr = g_force_tpr.load(), fvpt = g_force_vpt.load();
     if (ftpr && fvpt) {
         const int64_t nvec = H / 8;
@@ -191,8 +258,19 @@ rn_status plan_impl(int64_t T, int64_t H, bool vector_ok, rn_plan* p) {
         }
         return RN_OK;
     }
+    // Enough rows for every resident CTA to stream several: the staged kernel.
+    if (T >= 4LL * num_sms && auto_staged_plan(op, T, H, num_sms, p)) return RN_OK;
+    std::memset(p, 0, sizeof *p);
     if (!auto_vector_plan(T, H, p)) fill_scalar_plan(T, p);
     return RN_OK;
+}
+
+int device_sms() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return kDefaultSms;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess || n < 1)
+        return kDefaultSms;
+    return n;
 }
 
 struct Common {
@@ -263,7 +341,7 @@ rn_status check_descriptors(int op, const rn_tensor* o, const rn_tensor* sc, con
 
 // Pointer-level checks (NULL data, element alignment, aliasing) and the plan.
 // Only called for T > 0.
-rn_status check_pointers_and_plan(int op, const Common& c, rn_plan* plan) {
+rn_status check_pointers_and_plan(int op, const Common& c, int num_sms, rn_plan* plan) {
     const int64_t T = c.x.T, H = c.x.H;
     if (!c.x.ptr || (op != rn::kFusedAddFp8 && !c.out.ptr)) return RN_ERR_NULL;
     if (op != rn::kRmsNorm && !c.res.ptr) return RN_ERR_NULL;
@@ -299,7 +377,7 @@ rn_status check_pointers_and_plan(int op, const Common& c, rn_plan* plan) {
     if (op != rn::kFusedAddFp8) vector_ok = vector_ok && aligned(c.out.ptr, 16);
     if (op != rn::kRmsNorm) vector_ok = vector_ok && aligned(c.res.ptr, 16);
     if (op == rn::kFusedAddFp8) vector_ok = vector_ok && aligned(c.q.ptr, 8);
-    rn_status st = plan_impl(T, H, vector_ok, plan);
+    rn_status st = plan_impl(op, T, H, vector_ok, num_sms, plan);
     if (st != RN_OK) return st;
     if (plan->grid > 0x7fffffffLL) plan->grid = 0x7fffffffLL;  // grid-stride loops cover the rest
     return RN_OK;
@@ -308,13 +386,13 @@ rn_status check_pointers_and_plan(int op, const Common& c, rn_plan* plan) {
 // All checks of one call; *launch_needed is false for the T == 0 no-op.
 rn_status prepare(int op, const rn_tensor* o, const rn_tensor* sc, const rn_tensor* x,
                   const rn_tensor* r, const rn_tensor* w, float eps, int64_t variance_size,
-                  Common* c, rn_plan* plan, bool* launch_needed) {
+                  int num_sms, Common* c, rn_plan* plan, bool* launch_needed) {
     *launch_needed = false;
     std::memset(plan, 0, sizeof *plan);
     rn_status st = check_descriptors(op, o, sc, x, r, w, eps, variance_size, c);
     if (st != RN_OK) return st;
     if (c->x.T == 0) return RN_OK;
-    st = check_pointers_and_plan(op, *c, plan);
+    st = check_pointers_and_plan(op, *c, num_sms, plan);
     if (st != RN_OK) return st;
     *launch_needed = true;
     return RN_OK;
@@ -326,7 +404,10 @@ rn_status run(int op, const rn_tensor* o, const rn_tensor* sc, const rn_tensor* 
     Common c;
     rn_plan plan;
     bool launch_needed;
-    rn_status st = prepare(op, o, sc, x, r, w, eps, variance_size, &c, &plan, &launch_needed);
+    rn_status st = check_descriptors(op, o, sc, x, r, w, eps, variance_size, &c);
+    if (st != RN_OK || c.x.T == 0) return st;
+    st = prepare(op, o, sc, x, r, w, eps, variance_size, device_sms(), &c, &plan,
+                 &launch_needed);
     if (st != RN_OK || !launch_needed) return st;
     rn::Args a;
     a.x = c.x.ptr;
@@ -338,8 +419,13 @@ rn_status run(int op, const rn_tensor* o, const rn_tensor* sc, const rn_tensor* 
     a.T = c.x.T;
     a.H = c.x.H;
     a.eps = eps;
-    const rn::Launch l{plan.kernel, plan.threads_per_row, plan.vectors_per_thread,
-                       plan.rows_per_cta, plan.block_threads, plan.smem_bytes, plan.grid};
+    const rn::Launch l{plan.kernel,
+                       plan.threads_per_row,
+                       plan.kernel == RN_KERNEL_STAGED ? plan.stages : plan.vectors_per_thread,
+                       plan.rows_per_cta,
+                       plan.block_threads,
+                       plan.smem_bytes,
+                       plan.grid};
     const cudaError_t e = rn::launch(op, c.dt, a, l, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) {
         std::snprintf(g_cuda_error, sizeof g_cuda_error, "%s: %s", cudaGetErrorName(e),
@@ -378,8 +464,8 @@ rn_status rn_validate(int32_t op, const rn_tensor* out_or_q, const rn_tensor* sc
     Common c;
     rn_plan local;
     bool launch_needed;
-    rn_status st = prepare(op, out_or_q, scale, x, residual, weight, eps, variance_size, &c,
-                           plan ? plan : &local, &launch_needed);
+    rn_status st = prepare(op, out_or_q, scale, x, residual, weight, eps, variance_size,
+                           kDefaultSms, &c, plan ? plan : &local, &launch_needed);
     return st;
 }
 
@@ -407,7 +493,36 @@ rn_status rn_plan_launch(int32_t op, int32_t dtype, int64_t T, int64_t H, int32_
     if (!plan) return RN_ERR_NULL;
     if (op < 0 || op > 2) return RN_ERR_CONFIG;
     if (!is16(dtype)) return RN_ERR_DTYPE;
-    return plan_impl(T, H, vector_ok != 0, plan);
+    return plan_impl(op, T, H, vector_ok != 0, kDefaultSms, plan);
+}
+
+rn_status rn_force_staged(int32_t ctas_per_sm, int32_t stages, int32_t threads) {
+    if (ctas_per_sm == 0 && stages == 0 && threads == 0) {
+        g_force_staged_c.store(0);
+        g_force_staged_s.store(0);
+        g_force_staged_t.store(0);
+        return RN_OK;
+    }
+    if (!(ctas_per_sm == 1 || ctas_per_sm == 2 || ctas_per_sm == 4) || stages < 2 ||
+        stages > 64 || threads < 32 || threads > 1024 || threads % 32)
+        return RN_ERR_CONFIG;
+    g_force_staged_s.store(stages);
+    g_force_staged_t.store(threads);
+    g_force_staged_c.store(ctas_per_sm);
+    return RN_OK;
+}
+
+rn_status rn_device_errors(uint32_t* flags) {
+    if (!flags) return RN_ERR_NULL;
+    unsigned v = 0;
+    const cudaError_t e = rn::read_and_clear_device_errors(&v);
+    if (e != cudaSuccess) {
+        std::snprintf(g_cuda_error, sizeof g_cuda_error, "%s: %s", cudaGetErrorName(e),
+                      cudaGetErrorString(e));
+        return RN_ERR_CUDA;
+    }
+    *flags = v;
+    return RN_OK;
 }
 
 rn_status rn_force_plan(int32_t threads_per_row, int32_t vectors_per_thread) {
@@ -427,6 +542,6 @@ int32_t rn_supported_vectors_per_thread(int32_t* out, int32_t cap) {
     return rn::kNumVpt;
 }
 
-const char* rn_version(void) { return "0.1.0"; }
+const char* rn_version(void) { return "0.2.0"; }
 
 }  // extern "C"

@@ -276,6 +276,242 @@ __global__ void __launch_bounds__(max_block_for_vpt(VPT))
     }
 }
 
+// ---------------------------------------------------------------- staged kernel
+//
+// Persistent, row -> CTA. Thread 0 streams whole rows of x (and the residual)
+// into a ring of `stages` shared-memory slots with one bulk asynchronous copy
+// per row and tensor (cp.async.bulk, completion counted on an mbarrier), up
+// to `stages` rows ahead, so the bytes in flight per SM are set by shared
+// memory rather than by registers. All threads then make two passes over the
+// staged row: (1) residual add, write-back (global, and over the x slot in
+// shared memory), sum of squares [and max |v * w|]; (2) the output. CTA b owns
+// rows b, b + gridDim.x, ... Every mbarrier wait is bounded; on a timeout the
+// CTA records kErrWaitTimeout in g_rn_device_error, waits (bounded) for the
+// copies it issued, and returns.
+
+__device__ unsigned int g_rn_device_error = 0;
+
+constexpr unsigned kErrWaitTimeout = 1u;
+constexpr long long kWaitLimitCycles = 4000000000LL;  // ~2 s at 1.9 GHz
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+    return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint32_t bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count) : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint32_t bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(bar), "r"(bytes)
+                 : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint32_t bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait for phase `parity` of an mbarrier; false on timeout.
+__device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    while (!mbar_try_wait(bar, parity)) {
+        if (clock64() - t0 > kWaitLimitCycles) return false;
+    }
+    return true;
+}
+
+// Global -> shared bulk copy of `bytes` (multiple of 16, both ends 16-byte
+// aligned), completing on mbarrier `bar`; L2 evict-first (read once).
+__device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes,
+                                          uint32_t bar, uint64_t policy) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint"
+        " [%0], [%1], %2, [%3], %4;" ::"r"(dst),
+        "l"(src), "r"(bytes), "r"(bar), "l"(policy)
+        : "memory");
+}
+
+__device__ __forceinline__ uint64_t policy_evict_first() {
+    uint64_t p;
+    asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
+    return p;
+}
+
+template <typename T, int OP>
+__global__ void __launch_bounds__(1024)
+    rn_staged_kernel(const Args a, const int stages, const uint32_t slot_bytes) {
+    using F = Fmt<T>;
+    constexpr bool kFused = OP != kRmsNorm;
+    constexpr bool kFp8 = OP == kFusedAddFp8;
+    constexpr int kSlots = kFused ? 2 : 1;  // x [, residual] per stage
+    extern __shared__ __align__(128) unsigned char smem[];
+
+    const int tid = threadIdx.x;
+    const int nthr = blockDim.x;
+    const int nwarps = nthr >> 5;
+    const int64_t nvec = a.H >> 3;
+    const uint32_t row_bytes = static_cast<uint32_t>(a.H) * 2u;
+    const uint32_t stage_bytes = kSlots * slot_bytes;
+    const int64_t G = gridDim.x;
+    const int64_t first = blockIdx.x;
+    const int64_t nrows = first < a.T ? (a.T - 1 - first) / G + 1 : 0;
+    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + static_cast<size_t>(stages) * stage_bytes);
+    float2* red = reinterpret_cast<float2*>(bars + stages);
+    const uint4* __restrict__ wv = static_cast<const uint4*>(a.weight);
+    const bool has_w = wv != nullptr;
+    const float hf = static_cast<float>(a.H);
+    const char* xg = static_cast<const char*>(a.x);
+    char* rg = static_cast<char*>(a.residual);
+
+    uint64_t policy = 0;
+    if (tid == 0) {
+        policy = policy_evict_first();
+        for (int s = 0; s < stages; ++s) mbar_init(smem_u32(bars + s), 1);
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    }
+    __syncthreads();
+
+    auto issue = [&](int s, int64_t row) {
+        const uint32_t bar = smem_u32(bars + s);
+        const uint32_t dst = smem_u32(smem + static_cast<size_t>(s) * stage_bytes);
+        mbar_arrive_expect_tx(bar, kSlots * row_bytes);
+        bulk_load(dst, xg + row * row_bytes, row_bytes, bar, policy);
+        if constexpr (kFused) bulk_load(dst + slot_bytes, rg + row * row_bytes, row_bytes, bar, policy);
+    };
+    if (tid == 0) {
+        for (int s = 0; s < stages && s < nrows; ++s) issue(s, first + s * G);
+    }
+
+    int64_t k = 0;
+    for (; k < nrows; ++k) {
+        const int s = static_cast<int>(k % stages);
+        const uint32_t parity = static_cast<uint32_t>((k / stages) & 1);
+        const int64_t row = first + k * G;
+        const bool ok = mbar_wait(smem_u32(bars + s), parity);
+        uint4* sx = reinterpret_cast<uint4*>(smem + static_cast<size_t>(s) * stage_bytes);
+        const uint4* sr = reinterpret_cast<const uint4*>(smem + static_cast<size_t>(s) * stage_bytes + slot_bytes);
+
+        // pass 1: [residual add + write-back], sum of squares [, max |v * w|]
+        float ss = 0.f, pm = 0.f;
+        if (ok) {
+            for (int64_t j = tid; j < nvec; j += nthr) {
+                uint4 v = sx[j];
+                uint32_t* vs = &v.x;
+                if constexpr (kFused) {
+                    const uint4 r = sr[j];
+                    const uint32_t* rs = &r.x;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const float2 fx = F::unpack(vs[c]);
+                        const float2 fr = F::unpack(rs[c]);
+                        vs[c] = F::pack(fx.x + fr.x, fx.y + fr.y);
+                    }
+                    st_v4(reinterpret_cast<uint4*>(rg + row * row_bytes) + j, v);
+                    sx[j] = v;
+                }
+                uint4 w4 = make_uint4(0, 0, 0, 0);
+                if constexpr (kFp8) {
+                    if (has_w) w4 = __ldg(wv + j);
+                }
+                const uint32_t* ws = &w4.x;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const float2 f = F::unpack(vs[c]);
+                    ss = fmaf(f.x, f.x, ss);
+                    ss = fmaf(f.y, f.y, ss);
+                    if constexpr (kFp8) {
+                        const float2 wf = has_w ? F::unpack(ws[c]) : make_float2(1.f, 1.f);
+                        pm = fmaxf(pm, fabsf(f.x * wf.x));
+                        pm = fmaxf(pm, fabsf(f.y * wf.y));
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            ss += __shfl_xor_sync(0xffffffffu, ss, o);
+            if constexpr (kFp8) pm = fmaxf(pm, __shfl_xor_sync(0xffffffffu, pm, o));
+        }
+        if ((tid & 31) == 0) red[tid >> 5] = make_float2(ss, pm);
+        // Barrier A: publishes `red` and makes a timeout uniform across the CTA.
+        if (__syncthreads_or(!ok)) {
+            if (tid == 0) atomicOr(&g_rn_device_error, kErrWaitTimeout);
+            break;
+        }
+        ss = 0.f;
+        pm = 0.f;
+        for (int i = 0; i < nwarps; ++i) {
+            const float2 t = red[i];
+            ss += t.x;
+            pm = fmaxf(pm, t.y);
+        }
+        const float inv = 1.0f / sqrtf(ss / hf + a.eps);
+
+        // pass 2: outputs from the staged (written-back) row
+        if constexpr (!kFp8) {
+            uint4* og = reinterpret_cast<uint4*>(static_cast<char*>(a.out) + row * row_bytes);
+            for (int64_t j = tid; j < nvec; j += nthr) {
+                const uint4 v = sx[j];
+                const uint4 w4 = has_w ? __ldg(wv + j) : make_uint4(0, 0, 0, 0);
+                const uint32_t* vs = &v.x;
+                const uint32_t* ws = &w4.x;
+                uint4 o;
+                uint32_t* os = &o.x;
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const float2 f = F::unpack(vs[c]);
+                    const float2 wf = has_w ? F::unpack(ws[c]) : make_float2(1.f, 1.f);
+                    os[c] = F::pack((f.x * wf.x) * inv, (f.y * wf.y) * inv);
+                }
+                st_v4(og + j, o);
+            }
+        } else {
+            const float qmul = pm > 0.f ? 448.0f / pm : 0.f;
+            if (tid == 0) a.scale[row] = pm > 0.f ? (pm * inv) / 448.0f : 0.f;
+            uint2* qg = reinterpret_cast<uint2*>(a.q + row * a.H);
+            for (int64_t j = tid; j < nvec; j += nthr) {
+                const uint4 v = sx[j];
+                const uint4 w4 = has_w ? __ldg(wv + j) : make_uint4(0, 0, 0, 0);
+                const uint32_t* vs = &v.x;
+                const uint32_t* ws = &w4.x;
+                uint32_t e[4];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const float2 f = F::unpack(vs[c]);
+                    const float2 wf = has_w ? F::unpack(ws[c]) : make_float2(1.f, 1.f);
+                    e[c] = e4m3x2((f.x * wf.x) * qmul, (f.y * wf.y) * qmul);
+                }
+                uint2 o = make_uint2(e[0] | (e[1] << 16), e[2] | (e[3] << 16));
+                if (!(pm > 0.f)) o = make_uint2(0, 0);
+                st_v2(qg + j, o);
+            }
+        }
+        // Barrier B: every thread is done with stage s (and with `red`).
+        __syncthreads();
+        if (tid == 0 && k + stages < nrows) {
+            asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+            issue(s, first + (k + stages) * G);
+        }
+    }
+    if (k < nrows && tid == 0) {
+        // Timed out: wait (bounded) for the copies still in flight, then leave.
+        const int64_t last = (k + stages < nrows ? k + stages : nrows);
+        for (int64_t kk = k; kk < last; ++kk) {
+            mbar_wait(smem_u32(bars + (kk % stages)), static_cast<uint32_t>((kk / stages) & 1));
+        }
+    }
+}
+
 // ---------------------------------------------------------------- scalar kernel
 
 constexpr int kScalarBlock = 256;
@@ -354,9 +590,34 @@ cudaError_t dispatch_vpt(const Args& a, const Launch& l, cudaStream_t s) {
     }
 }
 
+// Opt each staged-kernel instantiation into large dynamic shared memory once
+// per device (the attribute is per function and per device context).
+template <typename T, int OP>
+cudaError_t prepare_staged(int smem) {
+    static unsigned long long done_mask = 0;  // bit d: device d configured
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return e;
+    const unsigned long long bit = dev < 64 ? (1ull << dev) : 0;
+    if (bit && (__atomic_load_n(&done_mask, __ATOMIC_ACQUIRE) & bit)) return cudaSuccess;
+    (void)smem;
+    e = cudaFuncSetAttribute(rn_staged_kernel<T, OP>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             kStagedMaxSmem);
+    if (e == cudaSuccess && bit) __atomic_fetch_or(&done_mask, bit, __ATOMIC_ACQ_REL);
+    return e;
+}
+
 template <typename T, int OP>
 cudaError_t launch_typed(const Args& a, const Launch& l, cudaStream_t s) {
     if (l.kernel == 0) return dispatch_vpt<T, OP>(a, l, s);
+    if (l.kernel == 2) {
+        cudaError_t e = prepare_staged<T, OP>(l.smem);
+        if (e != cudaSuccess) return e;
+        const uint32_t slot = static_cast<uint32_t>(((a.H * 2 + 127) / 128) * 128);
+        rn_staged_kernel<T, OP><<<static_cast<unsigned>(l.grid), l.block, l.smem, s>>>(a, l.vpt,
+                                                                                       slot);
+        return cudaGetLastError();
+    }
     rn_scalar_kernel<T, OP><<<static_cast<unsigned>(l.grid), kScalarBlock, 0, s>>>(a);
     return cudaGetLastError();
 }
@@ -372,6 +633,18 @@ cudaError_t launch_op(int op, const Args& a, const Launch& l, cudaStream_t s) {
 }
 
 }  // namespace
+
+cudaError_t read_and_clear_device_errors(unsigned* flags) {
+    unsigned v = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&v, g_rn_device_error, sizeof v);
+    if (e != cudaSuccess) return e;
+    *flags = v;
+    if (v) {
+        const unsigned zero = 0;
+        e = cudaMemcpyToSymbol(g_rn_device_error, &zero, sizeof zero);
+    }
+    return e;
+}
 
 cudaError_t launch(int op, int dtype, const Args& a, const Launch& l, cudaStream_t s) {
     if (dtype == kBF16) return launch_op<__nv_bfloat16>(op, a, l, s);

@@ -22,9 +22,9 @@ struct Args {
 };
 
 struct Launch {
-    int kernel;  // 0 = vector, 1 = scalar
+    int kernel;  // 0 = vector, 1 = scalar, 2 = staged
     int tpr;     // threads per row
-    int vpt;     // 16-byte vectors per thread
+    int vpt;     // vector kernel: 16-byte vectors per thread; staged kernel: stages
     int rpc;     // rows per CTA
     int block;   // threads per CTA
     int smem;    // dynamic shared memory bytes
@@ -42,7 +42,16 @@ constexpr int kNumVpt = sizeof(kVptList) / sizeof(kVptList[0]);
 // __launch_bounds__), which bounds the registers it may use per thread.
 constexpr int max_block_for_vpt(int vpt) { return vpt <= 4 ? 1024 : (vpt <= 8 ? 512 : 256); }
 
+// Dynamic shared memory the staged kernel may be configured for (B200: 227 KB
+// per block) and the per-SM budget the planner spreads over resident CTAs.
+constexpr int kStagedMaxSmem = 227 * 1024;
+constexpr int kStagedSmemPerSm = 220 * 1024;
+
 // Enqueues one launch; returns the CUDA error of the launch itself.
 cudaError_t launch(int op, int dtype, const Args& a, const Launch& l, cudaStream_t s);
+
+// Reads, and clears when set, the device-side error flags of the current
+// device (bit 0: an mbarrier wait timed out). Synchronous.
+cudaError_t read_and_clear_device_errors(unsigned* flags);
 
 }  // namespace rn

@@ -231,7 +231,20 @@ def test_planner_invariants(op):
     for T in SWEEP_T:
         for Hh in SWEEP_H:
             p = rn.plan_launch(op, BF, T, Hh)
-            assert p["kernel"] == 0, (T, Hh)
+            assert p["kernel"] in (0, 2), (T, Hh)
+            if p["kernel"] == 2:
+                # staged: persistent grid, ring of >= 2 stages within 227 KB
+                nin = 1 if op == "rms_norm" else 2
+                slot = -(-2 * Hh // 128) * 128
+                assert p["stages"] >= 2
+                assert p["smem_bytes"] == p["stages"] * (nin * slot + 8) + 256
+                assert p["smem_bytes"] <= 227 * 1024
+                assert p["ctas_per_sm"] * (p["smem_bytes"] + 1024) <= 228 * 1024
+                assert p["ctas_per_sm"] * p["block_threads"] <= 1024
+                assert p["block_threads"] % 32 == 0
+                assert p["grid"] == min(T, p["ctas_per_sm"] * 148)
+                assert T >= 4 * 148
+                continue
             tpr, vpt, rpc = p["threads_per_row"], p["vectors_per_thread"], p["rows_per_cta"]
             assert tpr * vpt * 8 >= Hh
             assert tpr * vpt * 8 - Hh < Hh  # at most one idle slot per used slot
@@ -261,6 +274,26 @@ def test_force_plan_hook():
     finally:
         rn.force_plan(0, 0)
     assert rn.plan_launch("fused_add_rms_norm", BF, 100, 4096)["kernel"] == 0
+
+
+def test_force_staged_hook():
+    with pytest.raises(rn.RmsNormError):
+        rn.force_staged(3, 4, 256)
+    with pytest.raises(rn.RmsNormError):
+        rn.force_staged(2, 1, 256)
+    with pytest.raises(rn.RmsNormError):
+        rn.force_staged(2, 4, 100)
+    try:
+        rn.force_staged(1, 5, 384)
+        p = rn.plan_launch("fused_add_rms_norm", BF, 50, 3840)
+        assert (p["kernel"], p["ctas_per_sm"], p["stages"], p["block_threads"]) == (2, 1, 5, 384)
+        assert p["grid"] == 50
+        # a forced ring that does not fit in shared memory is not used
+        p = rn.plan_launch("fused_add_rms_norm", BF, 50, 16384 * 4)
+        assert p["kernel"] != 2
+    finally:
+        rn.force_staged(0, 0, 0)
+    assert rn.plan_launch("fused_add_rms_norm", BF, 50, 3840)["kernel"] == 0
 
 
 def test_status_strings():

@@ -24,8 +24,11 @@ def _cuda():
     if not torch.cuda.is_available():
         pytest.fail("GPU tests need a CUDA device")
     rn.force_plan(0, 0)
+    rn.force_staged(0, 0, 0)
     yield
     rn.force_plan(0, 0)
+    rn.force_staged(0, 0, 0)
+    assert rn.device_errors() == 0, "a kernel recorded a device-side error"
 
 
 def _inputs(T, H, dtype, seed, var_r=4.0):
@@ -97,7 +100,7 @@ def test_every_compiled_width_forced(op, dtype):
 def test_sub_warp_and_idle_slot_shapes(op):
     """Rows narrower than a warp (several rows per warp), and shapes that
     leave idle vector slots (H = 3840 on 64 x 8 = 512 slots for 480 vectors)."""
-    cases = [(512, 2, 4), (512, 4, 16), (512, 8, 8), (512, 16, 4), (512, 32, 2), (512, 64, 1),
+    cases = [(512, 4, 16), (512, 8, 8), (512, 16, 4), (512, 32, 2), (512, 64, 1),
              (3840, 64, 8), (3840, 32, 15), (3840, 96, 5), (3840, 160, 3), (3840, 480, 1),
              (2048 + 8, 32, 10), (8, 1, 1)]
     for H, tpr, vpt in cases:
@@ -106,6 +109,43 @@ def test_sub_warp_and_idle_slot_shapes(op):
             x, r, w = _inputs(T, H, "bf16", seed=H + tpr + T)
             _check(op, x, r, w, 1e-6, "bf16", expect_kernel=0)
     rn.force_plan(0, 0)
+
+
+STAGED_SHAPES = [  # (H, ctas per SM, stages, threads, T)
+    (3840, 4, 3, 256, 1000), (3840, 1, 2, 96, 7), (4096, 2, 6, 256, 333), (512, 4, 8, 64, 777),
+    (16384, 1, 3, 1024, 150), (2048, 4, 5, 32, 1), (7168, 2, 3, 448, 300), (8, 4, 4, 32, 50),
+    (5120, 2, 5, 320, 597),
+]
+
+
+@pytest.mark.parametrize("dtype", ["bf16", "fp16"])
+@pytest.mark.parametrize("op", OPS)
+def test_staged_kernel_forced_shapes(op, dtype):
+    """The shared-memory-ring kernel on rings of 2..8 stages, 1..4 CTAs per SM,
+    threads from 1 to 5 vectors per pass, and row counts that leave CTAs with
+    unequal numbers of rows."""
+    for H, c, S, thr, T in STAGED_SHAPES:
+        rn.force_staged(c, S, thr)
+        x, r, w = _inputs(T, H, dtype, seed=H + S + T)
+        _check(op, x, r, w, 1e-6, dtype, expect_kernel=2)
+        _check(op, x, r, None, 1e-6, dtype, expect_kernel=2)
+    rn.force_staged(0, 0, 0)
+
+
+@pytest.mark.parametrize("op", ["rms_norm", "fused_add_rms_norm"])
+def test_staged_in_place_out_is_x(op):
+    rn.force_staged(2, 4, 128)
+    T, H = 500, 2048
+    x, r, w = _inputs(T, H, "bf16", seed=21)
+    xd, rd = x.cuda().clone(), r.cuda().clone()
+    if op == "rms_norm":
+        rn.rms_norm(xd, xd, w.cuda(), 1e-6)
+        got = {"out": xd}
+    else:
+        rn.fused_add_rms_norm(xd, xd, rd, w.cuda(), 1e-6)
+        got = {"out": xd, "residual": rd}
+    torch.cuda.synchronize()
+    compare(op, got, oracle_run(op, x, r, w, 1e-6, "bf16"), "bf16")
 
 
 @pytest.mark.parametrize("op", OPS)
@@ -196,7 +236,8 @@ def test_deterministic(op):
     wl = synth.make_inputs("prefill", op, "bf16", 1024, 3840)
     outs = []
     for _ in range(2):
-        got = gpu_run(op, wl.x.cuda(), wl.residual.cuda().clone(), wl.weight.cuda(), wl.eps)
+        r = None if wl.residual is None else wl.residual.cuda().clone()
+        got = gpu_run(op, wl.x.cuda(), r, wl.weight.cuda(), wl.eps)
         torch.cuda.synchronize()
         outs.append({k: bits16(v) if v.dtype in (torch.bfloat16, torch.float16)
                      else v.view(torch.uint8).cpu().numpy() if v.dtype == torch.float8_e4m3fn

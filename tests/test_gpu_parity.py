@@ -23,6 +23,13 @@ def _cuda():
     if not torch.cuda.is_available():
         pytest.fail("GPU tests need a CUDA device")
     rn.force_plan(0, 0)
+    rn.force_staged(0, 0, 0)
+
+
+@pytest.fixture(autouse=True)
+def _no_device_errors():
+    yield
+    assert rn.device_errors() == 0, "a kernel recorded a device-side error"
 
 
 def _full(op, wl, with_weight=True):

@@ -200,6 +200,15 @@ RN_API rn_status rn_force_plan(int32_t threads_per_row, int32_t vectors_per_thre
  * launches; meant for tests and tuning. */
 RN_API rn_status rn_force_staged(int32_t ctas_per_sm, int32_t stages, int32_t threads);
 
+/* Launch options for every later call in the process (tuning hook):
+ * pdl = 1 launches with programmatic dependent launch (the kernel may begin
+ * launching while the previous kernel in the stream drains; it waits for that
+ * kernel to complete before touching memory), 0 launches plainly, -1 restores
+ * the library default; max_grid > 0 caps the blocks launched (the kernels
+ * stride over the remaining rows), 0 removes the cap. RN_ERR_CONFIG for other
+ * values. Not thread-safe with concurrent launches. */
+RN_API rn_status rn_set_launch_options(int32_t pdl, int64_t max_grid);
+
 /* Reads and clears the device-side error flags of the current device:
  * bit 0 = a bounded wait inside the STAGED kernel timed out (some rows of
  * that call were not written). Synchronises with the device. */

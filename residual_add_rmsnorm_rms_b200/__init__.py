@@ -18,12 +18,13 @@ from __future__ import annotations
 
 import ctypes
 import os
+import threading
 
 import torch
 
 __all__ = [
     "RmsNormError", "rms_norm", "fused_add_rms_norm", "fused_add_rms_norm_fp8",
-    "plan_launch", "validate", "force_plan", "force_staged", "device_errors", "supported_vectors_per_thread", "status_string",
+    "plan_launch", "validate", "force_plan", "force_staged", "set_launch_options", "device_errors", "supported_vectors_per_thread", "status_string",
     "LIB_PATH", "lib", "RnTensor", "RnPlan", "STATUS", "OPS",
 ]
 
@@ -99,6 +100,8 @@ def _load():
     L.rn_force_plan.restype = ctypes.c_int
     L.rn_force_staged.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32]
     L.rn_force_staged.restype = ctypes.c_int
+    L.rn_set_launch_options.argtypes = [ctypes.c_int32, ctypes.c_int64]
+    L.rn_set_launch_options.restype = ctypes.c_int
     L.rn_device_errors.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
     L.rn_device_errors.restype = ctypes.c_int
     L.rn_supported_vectors_per_thread.argtypes = [ctypes.POINTER(ctypes.c_int32), ctypes.c_int32]
@@ -116,7 +119,8 @@ def status_string(status: int) -> str:
 
 
 def describe(t: torch.Tensor | None):
-    """(RnTensor, keepalive) for a tensor; (None, None) for None."""
+    """(RnTensor, keepalive) for a tensor; (None, None) for None. Builds fresh
+    ctypes arrays (used by validate(); the operator calls use _desc)."""
     if t is None:
         return None, None
     n = t.dim()
@@ -127,6 +131,28 @@ def describe(t: torch.Tensor | None):
     return d, (sizes, strides)
 
 
+_tls = threading.local()
+_CACHE_MAX = 256
+
+
+def _desc(t: torch.Tensor, slot: int):
+    """A by-reference rn_tensor for `t`. Descriptors are cached per thread,
+    argument slot and (dtype, shape, strides), and only the data pointer is
+    rewritten per call: marshalling stays cheap next to a kernel launch."""
+    cache = getattr(_tls, "cache", None)
+    if cache is None:
+        cache = _tls.cache = {}
+    key = (slot, t.dtype, t.shape, t.stride())
+    ent = cache.get(key)
+    if ent is None:
+        if len(cache) >= _CACHE_MAX:
+            cache.clear()
+        d, keep = describe(t)
+        ent = cache[key] = (d, keep, ctypes.byref(d))
+    ent[0].data = t.data_ptr() if t.numel() else 0
+    return ent[2]
+
+
 def _ref(d):
     return None if d is None else ctypes.byref(d)
 
@@ -135,20 +161,29 @@ def _vs(variance_size) -> int:
     return -1 if variance_size is None else int(variance_size)
 
 
-def _device_and_stream(tensors, stream):
-    dev = None
+def _stream_for(tensors, stream):
+    """The device index shared by all tensors and the raw stream handle."""
+    dev = -2
     for t in tensors:
         if t is None:
             continue
-        if not t.is_cuda:
+        d = t.get_device()
+        if d < 0:
             raise ValueError("all operands must be CUDA tensors (the library takes device pointers)")
-        if dev is None:
-            dev = t.device
-        elif t.device != dev:
+        if dev == -2:
+            dev = d
+        elif d != dev:
             raise ValueError("operands are on different devices")
     if stream is None:
         stream = torch.cuda.current_stream(dev)
     return dev, (stream.cuda_stream if hasattr(stream, "cuda_stream") else stream)
+
+
+def _call(fn, dev: int, *args):
+    if torch.cuda.current_device() == dev:
+        return fn(*args)
+    with torch.cuda.device(dev):
+        return fn(*args)
 
 
 def _check(status: int, what: str):
@@ -162,12 +197,9 @@ def _check(status: int, what: str):
 def rms_norm(out: torch.Tensor, x: torch.Tensor, weight: torch.Tensor | None, eps: float,
              variance_size=None, stream=None) -> None:
     """out = x / sqrt(mean(x^2) + eps) * weight over the last dim (C ABI rn_rms_norm)."""
-    dev, s = _device_and_stream((out, x, weight), stream)
-    do, ko = describe(out)
-    dx, kx = describe(x)
-    dw, kw = describe(weight)
-    with torch.cuda.device(dev):
-        st = lib.rn_rms_norm(_ref(do), _ref(dx), _ref(dw), eps, _vs(variance_size), s)
+    dev, s = _stream_for((out, x, weight), stream)
+    st = _call(lib.rn_rms_norm, dev, _desc(out, 0), _desc(x, 1),
+               None if weight is None else _desc(weight, 2), eps, _vs(variance_size), s)
     _check(st, "rn_rms_norm")
 
 
@@ -175,14 +207,9 @@ def fused_add_rms_norm(out: torch.Tensor, x: torch.Tensor, residual: torch.Tenso
                        weight: torch.Tensor | None, eps: float, variance_size=None,
                        stream=None) -> None:
     """residual += x (rounded, in place); out = rms_norm(residual) (C ABI rn_fused_add_rms_norm)."""
-    dev, s = _device_and_stream((out, x, residual, weight), stream)
-    do, ko = describe(out)
-    dx, kx = describe(x)
-    dr, kr = describe(residual)
-    dw, kw = describe(weight)
-    with torch.cuda.device(dev):
-        st = lib.rn_fused_add_rms_norm(_ref(do), _ref(dx), _ref(dr), _ref(dw), eps,
-                                       _vs(variance_size), s)
+    dev, s = _stream_for((out, x, residual, weight), stream)
+    st = _call(lib.rn_fused_add_rms_norm, dev, _desc(out, 0), _desc(x, 1), _desc(residual, 2),
+               None if weight is None else _desc(weight, 3), eps, _vs(variance_size), s)
     _check(st, "rn_fused_add_rms_norm")
 
 
@@ -191,15 +218,10 @@ def fused_add_rms_norm_fp8(q: torch.Tensor, scale: torch.Tensor, x: torch.Tensor
                            variance_size=None, stream=None) -> None:
     """residual += x (in place); q, scale = per-token e4m3 cast of rms_norm(residual)
     (C ABI rn_fused_add_rms_norm_fp8). q: float8_e4m3fn (or uint8) [T, H]; scale: float32 [T]."""
-    dev, s = _device_and_stream((q, scale, x, residual, weight), stream)
-    dq, kq = describe(q)
-    dsc, ks = describe(scale)
-    dx, kx = describe(x)
-    dr, kr = describe(residual)
-    dw, kw = describe(weight)
-    with torch.cuda.device(dev):
-        st = lib.rn_fused_add_rms_norm_fp8(_ref(dq), _ref(dsc), _ref(dx), _ref(dr), _ref(dw), eps,
-                                           _vs(variance_size), s)
+    dev, s = _stream_for((q, scale, x, residual, weight), stream)
+    st = _call(lib.rn_fused_add_rms_norm_fp8, dev, _desc(q, 0), _desc(scale, 1), _desc(x, 2),
+               _desc(residual, 3), None if weight is None else _desc(weight, 4), eps,
+               _vs(variance_size), s)
     _check(st, "rn_fused_add_rms_norm_fp8")
 
 
@@ -235,6 +257,11 @@ def force_plan(threads_per_row: int, vectors_per_thread: int) -> None:
 def force_staged(ctas_per_sm: int, stages: int, threads: int) -> None:
     """Test/tuning hook: force the staged kernel's shape; (0, 0, 0) restores auto."""
     _check(lib.rn_force_staged(ctas_per_sm, stages, threads), "rn_force_staged")
+
+
+def set_launch_options(pdl: int = -1, max_grid: int = 0) -> None:
+    """Tuning hook: pdl 1/0/-1 (on/off/default) and a cap on blocks launched (0 = none)."""
+    _check(lib.rn_set_launch_options(pdl, max_grid), "rn_set_launch_options")
 
 
 def device_errors() -> int:

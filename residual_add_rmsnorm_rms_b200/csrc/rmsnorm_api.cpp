@@ -25,6 +25,14 @@ std::atomic<int> g_force_vpt{0};
 std::atomic<int> g_force_staged_c{0};
 std::atomic<int> g_force_staged_s{0};
 std::atomic<int> g_force_staged_t{0};
+std::atomic<int> g_pdl{-1};              // -1 default, 0 off, 1 on
+std::atomic<long long> g_max_grid{0};    // 0: no cap
+// Launch defaults, measured on B200 (prefill [8192 x 3840], two ops
+// alternating in one stream): programmatic dependent launch lets the next
+// kernel's blocks start as this one drains (+4-5 %), and capping the vector
+// kernel's grid at 16 blocks per SM (blocks then stride over rows) adds ~1 %.
+constexpr bool kPdlDefault = true;
+constexpr int kVectorBlocksPerSmCap = 16;
 constexpr int kDefaultSms = 148;  // B200; dry runs (no device) plan for it
 
 int elem_size(int32_t dt) {
@@ -137,7 +145,8 @@ int64_t round_up(int64_t v, int64_t m) { return (v + m - 1) / m * m; }
 
 int64_t staged_smem(int op, int64_t H, int stages) {
     const int nin = op == rn::kRmsNorm ? 1 : 2;
-    return stages * nin * round_up(2 * H, 128) + stages * 8 + 32 * 8;
+    // ring + fp32 copy of the weight + one mbarrier per stage + reduction slots
+    return stages * nin * round_up(2 * H, 128) + 4 * H + stages * 8 + 32 * 8;
 }
 
 // Fills a STAGED plan for (c CTAs per SM, S stages, threads); false if it
@@ -158,32 +167,6 @@ bool fill_staged_plan(int op, int64_t T, int64_t H, int c, int S, int threads, i
     const int64_t g = static_cast<int64_t>(c) * num_sms;
     p->grid = T < g ? T : g;
     return true;
-}
-
-// Automatic STAGED shape: as many resident CTAs per SM (4, 2, 1) as leave
-// each at least 3 ring stages (2 for the widest rows) inside the per-SM
-// shared-memory budget, up to 8 stages; about two 16-byte vectors per thread
-// per pass.
-bool auto_staged_plan(int op, int64_t T, int64_t H, int num_sms, rn_plan* p) {
-    const int nin = op == rn::kRmsNorm ? 1 : 2;
-    const int64_t stage = nin * round_up(2 * H, 128);
-    const int64_t nvec = H / 8;
-    for (int c : {4, 2, 1}) {
-        const int64_t per_cta = rn::kStagedSmemPerSm / c - 1024;
-        int64_t S = per_cta / stage;
-        if (S > 8) S = 8;
-        if (S >= 3 || (c == 1 && S >= 2)) {
-            int64_t threads = round_up((nvec + 1) / 2, 32);
-            // <= 1024 resident threads per SM: at ~48 registers per thread
-            // that is what the 64K-register file holds for c blocks.
-            const int64_t cap = 1024 / c;
-            if (threads > cap) threads = cap;
-            if (threads < 64) threads = 64;
-            return fill_staged_plan(op, T, H, c, static_cast<int>(S), static_cast<int>(threads),
-                                    num_sms, p);
-        }
-    }
-    return false;
 }
 
 void fill_scalar_plan(int64_t T, rn_plan* p) {
@@ -237,7 +220,22 @@ bool auto_vector_plan(int64_t T, int64_t H, rn_plan* p) {
     return true;
 }
 
+rn_status plan_shape(int op, int64_t T, int64_t H, bool vector_ok, int num_sms, rn_plan* p);
+
+// The launch plan: the kernel and its shape, then the grid cap (the kernels
+// stride over the rows a capped grid does not cover).
 rn_status plan_impl(int op, int64_t T, int64_t H, bool vector_ok, int num_sms, rn_plan* p) {
+    const rn_status st = plan_shape(op, T, H, vector_ok, num_sms, p);
+    if (st != RN_OK) return st;
+    long long cap = g_max_grid.load();
+    if (cap == 0 && p->kernel == RN_KERNEL_VECTOR)
+        cap = static_cast<long long>(kVectorBlocksPerSmCap) * num_sms;
+    if (cap > 0 && p->grid > cap) p->grid = cap;
+    if (p->grid > 0x7fffffffLL) p->grid = 0x7fffffffLL;
+    return RN_OK;
+}
+
+rn_status plan_shape(int op, int64_t T, int64_t H, bool vector_ok, int num_sms, rn_plan* p) {
     if (H < 1 || T < 0) return RN_ERR_SHAPE;
     std::memset(p, 0, sizeof *p);
     if (!vector_ok || H % 8 != 0) {
@@ -258,9 +256,9 @@ rn_status plan_impl(int op, int64_t T, int64_t H, bool vector_ok, int num_sms, r
         }
         return RN_OK;
     }
-    // Enough rows for every resident CTA to stream several: the staged kernel.
-    if (T >= 4LL * num_sms && auto_staged_plan(op, T, H, num_sms, p)) return RN_OK;
-    std::memset(p, 0, sizeof *p);
+    // The STAGED kernel is chosen only when forced: measured on B200 it trails
+    // the VECTOR kernel at every shape tried (T up to 65536, H 2048..16384).
+    (void)num_sms;
     if (!auto_vector_plan(T, H, p)) fill_scalar_plan(T, p);
     return RN_OK;
 }
@@ -379,7 +377,7 @@ rn_status check_pointers_and_plan(int op, const Common& c, int num_sms, rn_plan*
     if (op == rn::kFusedAddFp8) vector_ok = vector_ok && aligned(c.q.ptr, 8);
     rn_status st = plan_impl(op, T, H, vector_ok, num_sms, plan);
     if (st != RN_OK) return st;
-    if (plan->grid > 0x7fffffffLL) plan->grid = 0x7fffffffLL;  // grid-stride loops cover the rest
+
     return RN_OK;
 }
 
@@ -425,7 +423,8 @@ rn_status run(int op, const rn_tensor* o, const rn_tensor* sc, const rn_tensor* 
                        plan.rows_per_cta,
                        plan.block_threads,
                        plan.smem_bytes,
-                       plan.grid};
+                       plan.grid,
+                       g_pdl.load() < 0 ? kPdlDefault : g_pdl.load() == 1};
     const cudaError_t e = rn::launch(op, c.dt, a, l, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) {
         std::snprintf(g_cuda_error, sizeof g_cuda_error, "%s: %s", cudaGetErrorName(e),
@@ -509,6 +508,13 @@ rn_status rn_force_staged(int32_t ctas_per_sm, int32_t stages, int32_t threads) 
     g_force_staged_s.store(stages);
     g_force_staged_t.store(threads);
     g_force_staged_c.store(ctas_per_sm);
+    return RN_OK;
+}
+
+rn_status rn_set_launch_options(int32_t pdl, int64_t max_grid) {
+    if (pdl < -1 || pdl > 1 || max_grid < 0) return RN_ERR_CONFIG;
+    g_pdl.store(pdl);
+    g_max_grid.store(max_grid);
     return RN_OK;
 }
 

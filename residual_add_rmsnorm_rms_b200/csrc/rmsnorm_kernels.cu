@@ -18,21 +18,25 @@
 //    total), then, for rows wider than a warp, one named barrier per row
 //    group and a fixed-order sum over the group's warps from shared memory.
 //    The order is fixed, so results are bit-reproducible run to run.
+//  * staged kernel: persistent; whole rows streamed into a shared-memory ring
+//    by bulk asynchronous copies (see its section).
 //  * scalar kernel: one CTA per row, two passes (the second re-reads the row,
 //    mostly from L2); any H and any element-aligned pointers. It exists for
 //    correctness on inputs the vector kernel cannot take.
 //
-// Numerics (identical in both kernels): residual sums in fp32 then one
-// round-to-nearest-even to 16 bits (fp32 holds >= 2p+2 bits of either 16-bit
-// format, so this equals the correctly rounded sum); squares accumulated in
-// fp32; inv = 1 / sqrt(ss / H + eps) with IEEE sqrt and division; y = (v * w)
-// * inv, where v * w is exact in fp32; fp8: P = max |v * w| (exact),
-// q = e4m3(RNE, satfinite)((v * w) * (448 / P)), scale = (P * inv) / 448,
-// which equals max |y| / 448 because rounding is monotonic.
+// Numerics (all kernels): the residual sum is the correctly rounded 16-bit
+// sum (packed add.rn in the fast kernels; fp32 add then one rounding in the
+// scalar kernel, which is the same value because fp32 holds >= 2p+2 bits of
+// either 16-bit format); squares accumulated in fp32; inv = 1 / sqrt(ss / H +
+// eps) with IEEE sqrt and division; y = (v * w) * inv, where v * w is exact in
+// fp32; fp8: P = max |v * w| (exact), q = e4m3(RNE, satfinite)((v * w) *
+// (448 / P)), scale = (P * inv) / 448, which equals max |y| / 448 because
+// rounding is monotonic.
 #include <cuda_bf16.h>
 #include <cuda_fp16.h>
 
 #include <cstdint>
+#include <utility>
 
 #include "rn_internal.h"
 
@@ -40,19 +44,28 @@ namespace rn {
 namespace {
 
 // ---------------------------------------------------------------- formats
+//
+// Per 16-bit format: packed residual add (one round-to-nearest-even of the
+// exact sum of each pair: the correctly rounded sum, identical to adding in
+// fp32 and rounding once), exact widening of a packed pair to fp32, and
+// narrowing of an fp32 pair with one round-to-nearest-even.
 
 template <typename T>
 struct Fmt;
 
 template <>
 struct Fmt<__nv_bfloat16> {
-    static __device__ __forceinline__ float2 unpack(uint32_t u) {
-        __nv_bfloat162 h;
-        memcpy(&h, &u, 4);
-        return __bfloat1622float2(h);
+    static __device__ __forceinline__ uint32_t add2(uint32_t a, uint32_t b) {
+        uint32_t d;
+        asm("add.rn.bf16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+        return d;
     }
-    static __device__ __forceinline__ uint32_t pack(float lo, float hi) {
-        __nv_bfloat162 h = __floats2bfloat162_rn(lo, hi);
+    static __device__ __forceinline__ float2 unpack(uint32_t u) {
+        // bf16 is the upper half of an fp32 word
+        return make_float2(__uint_as_float(u << 16), __uint_as_float(u & 0xffff0000u));
+    }
+    static __device__ __forceinline__ uint32_t pack(float2 f) {
+        __nv_bfloat162 h = __floats2bfloat162_rn(f.x, f.y);
         uint32_t u;
         memcpy(&u, &h, 4);
         return u;
@@ -70,13 +83,18 @@ struct Fmt<__nv_bfloat16> {
 
 template <>
 struct Fmt<__half> {
+    static __device__ __forceinline__ uint32_t add2(uint32_t a, uint32_t b) {
+        uint32_t d;
+        asm("add.rn.f16x2 %0, %1, %2;" : "=r"(d) : "r"(a), "r"(b));
+        return d;
+    }
     static __device__ __forceinline__ float2 unpack(uint32_t u) {
         __half2 h;
         memcpy(&h, &u, 4);
         return __half22float2(h);
     }
-    static __device__ __forceinline__ uint32_t pack(float lo, float hi) {
-        __half2 h = __floats2half2_rn(lo, hi);
+    static __device__ __forceinline__ uint32_t pack(float2 f) {
+        __half2 h = __floats2half2_rn(f.x, f.y);
         uint32_t u;
         memcpy(&u, &h, 4);
         return u;
@@ -129,25 +147,135 @@ __device__ __forceinline__ uint32_t e4m3x2(float lo, float hi) {
     return r;
 }
 
+// Programmatic dependent launch. Every kernel lets the next kernel in the
+// stream begin launching at once (its blocks then wait, below, for this grid
+// to finish), and waits for the previous kernel in the stream to complete and
+// flush its memory before touching global memory. Without the launch
+// attribute both are no-ops, so the kernels are correct either way.
+__device__ __forceinline__ void pdl_allow_dependents() {
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait_for_prior_grid() {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+// ---------------------------------------------------------------- 8-element vector ops
+//
+// A uint4 holds 8 16-bit elements (4 packed pairs). Weights arrive as 4 fp32
+// pairs. The fp32 arithmetic uses Blackwell's paired instructions (two
+// lanes of fp32 per instruction, each rounded exactly like its scalar form).
+
+struct W8 {
+    float2 w[4];
+};
+
+template <typename T>
+__device__ __forceinline__ W8 w8_from_bits(const uint4& b) {
+    W8 r;
+    r.w[0] = Fmt<T>::unpack(b.x);
+    r.w[1] = Fmt<T>::unpack(b.y);
+    r.w[2] = Fmt<T>::unpack(b.z);
+    r.w[3] = Fmt<T>::unpack(b.w);
+    return r;
+}
+
+__device__ __forceinline__ W8 w8_from_f32(const float4* p) {
+    const float4 a = p[0], b = p[1];
+    W8 r;
+    r.w[0] = make_float2(a.x, a.y);
+    r.w[1] = make_float2(a.z, a.w);
+    r.w[2] = make_float2(b.x, b.y);
+    r.w[3] = make_float2(b.z, b.w);
+    return r;
+}
+
+template <typename T>
+__device__ __forceinline__ uint4 add8(const uint4& x, const uint4& r) {
+    return make_uint4(Fmt<T>::add2(x.x, r.x), Fmt<T>::add2(x.y, r.y), Fmt<T>::add2(x.z, r.z),
+                      Fmt<T>::add2(x.w, r.w));
+}
+
+// acc += v * v, pairwise (acc.x collects even elements, acc.y odd ones).
+template <typename T>
+__device__ __forceinline__ float2 ssq8(const uint4& v, float2 acc) {
+    const uint32_t* u = &v.x;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        const float2 f = Fmt<T>::unpack(u[c]);
+        acc = __ffma2_rn(f, f, acc);
+    }
+    return acc;
+}
+
+// Pair c (0..3) of 8 weights, as fp32: from widened fp32 weights (W8) or
+// straight from the packed 16-bit weights (uint4), widened pair by pair so
+// only 4 registers stay live.
+template <typename T>
+__device__ __forceinline__ float2 wpair(const W8& w, int c) {
+    return w.w[c];
+}
+template <typename T>
+__device__ __forceinline__ float2 wpair(const uint4& w, int c) {
+    return Fmt<T>::unpack((&w.x)[c]);
+}
+
+// max(pm, max |v * w|): v * w is exact in fp32 (a product of two 16-bit values).
+template <typename T, bool kHasW, typename WT>
+__device__ __forceinline__ float amax8(const uint4& v, const WT& w, float pm) {
+    const uint32_t* u = &v.x;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        float2 p = Fmt<T>::unpack(u[c]);
+        if constexpr (kHasW) p = __fmul2_rn(p, wpair<T>(w, c));
+        pm = fmaxf(pm, fmaxf(fabsf(p.x), fabsf(p.y)));
+    }
+    return pm;
+}
+
+// RNE16((v * w) * inv) for 8 elements.
+template <typename T, bool kHasW, typename WT>
+__device__ __forceinline__ uint4 scale8(const uint4& v, const WT& w, float2 inv2) {
+    const uint32_t* u = &v.x;
+    uint4 o;
+    uint32_t* os = &o.x;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        float2 p = Fmt<T>::unpack(u[c]);
+        if constexpr (kHasW) p = __fmul2_rn(p, wpair<T>(w, c));
+        os[c] = Fmt<T>::pack(__fmul2_rn(p, inv2));
+    }
+    return o;
+}
+
+// e4m3(RNE, satfinite)((v * w) * qmul) for 8 elements, 8 bytes.
+template <typename T, bool kHasW, typename WT>
+__device__ __forceinline__ uint2 quant8(const uint4& v, const WT& w, float2 qmul2) {
+    const uint32_t* u = &v.x;
+    uint32_t e[4];
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        float2 p = Fmt<T>::unpack(u[c]);
+        if constexpr (kHasW) p = __fmul2_rn(p, wpair<T>(w, c));
+        p = __fmul2_rn(p, qmul2);
+        e[c] = e4m3x2(p.x, p.y);
+    }
+    return make_uint2(e[0] | (e[1] << 16), e[2] | (e[3] << 16));
+}
+
 // ---------------------------------------------------------------- vector kernel
 
-template <typename T, int VPT, int OP>
-__global__ void __launch_bounds__(max_block_for_vpt(VPT))
-    rn_vector_kernel(const Args a, const int tpr, const int rpc) {
-    using F = Fmt<T>;
+template <typename T, int VPT, int OP, bool kHasW>
+__device__ __forceinline__ void vector_rows(const Args& a, const int tpr, const int rpc,
+                                            float2* red) {
     constexpr bool kFused = OP != kRmsNorm;
     constexpr bool kFp8 = OP == kFusedAddFp8;
-    extern __shared__ float2 red[];  // [2][rpc][warps per row]
 
     const int row_in_cta = threadIdx.x / tpr;
     const int lr = threadIdx.x - row_in_cta * tpr;
     const int wpr = tpr >> 5;
-    const int64_t nvec = a.H >> 3;
+    const int nvec = static_cast<int>(a.H >> 3);
     const float hf = static_cast<float>(a.H);
-    const uint4* __restrict__ xv = static_cast<const uint4*>(a.x);
-    uint4* rv = static_cast<uint4*>(a.residual);
     const uint4* __restrict__ wv = static_cast<const uint4*>(a.weight);
-    const bool has_w = wv != nullptr;
     int parity = 0;
 
     // The loop bound depends only on the block, so every thread of a warp
@@ -156,58 +284,46 @@ __global__ void __launch_bounds__(max_block_for_vpt(VPT))
          base += static_cast<int64_t>(gridDim.x) * rpc) {
         const int64_t row = base + row_in_cta;
         const bool active = row < a.T;
-        const int64_t roff = row * nvec;
+        const int64_t roff = (active ? row : 0) * nvec;
+        const uint4* xrow = static_cast<const uint4*>(a.x) + roff;
+        uint4* rrow = static_cast<uint4*>(a.residual) + roff;
 
         uint4 v[VPT];
 #pragma unroll
         for (int k = 0; k < VPT; ++k) {
-            const int64_t j = lr + static_cast<int64_t>(k) * tpr;
-            v[k] = (active && j < nvec) ? ld_stream(xv + roff + j) : make_uint4(0, 0, 0, 0);
+            const int j = lr + k * tpr;
+            v[k] = (active && j < nvec) ? ld_stream(xrow + j) : make_uint4(0, 0, 0, 0);
         }
         if constexpr (kFused) {
             uint4 r[VPT];
 #pragma unroll
             for (int k = 0; k < VPT; ++k) {
-                const int64_t j = lr + static_cast<int64_t>(k) * tpr;
-                r[k] = (active && j < nvec) ? ld_stream(rv + roff + j) : make_uint4(0, 0, 0, 0);
+                const int j = lr + k * tpr;
+                r[k] = (active && j < nvec) ? ld_stream(rrow + j) : make_uint4(0, 0, 0, 0);
             }
 #pragma unroll
             for (int k = 0; k < VPT; ++k) {
-                const int64_t j = lr + static_cast<int64_t>(k) * tpr;
-                uint32_t* xs = &v[k].x;
-                const uint32_t* rs = &r[k].x;
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const float2 fx = F::unpack(xs[c]);
-                    const float2 fr = F::unpack(rs[c]);
-                    xs[c] = F::pack(fx.x + fr.x, fx.y + fr.y);
-                }
-                if (active && j < nvec) st_v4(rv + roff + j, v[k]);
+                const int j = lr + k * tpr;
+                v[k] = add8<T>(v[k], r[k]);
+                if (active && j < nvec) st_v4(rrow + j, v[k]);
             }
         }
 
-        float ss = 0.f, pm = 0.f;
+        float2 acc = make_float2(0.f, 0.f);
+        float pm = 0.f;
 #pragma unroll
         for (int k = 0; k < VPT; ++k) {
-            const uint32_t* xs = &v[k].x;
-            uint4 wk = make_uint4(0, 0, 0, 0);
+            acc = ssq8<T>(v[k], acc);
             if constexpr (kFp8) {
-                const int64_t j = lr + static_cast<int64_t>(k) * tpr;
-                if (has_w && j < nvec) wk = __ldg(wv + j);
-            }
-            const uint32_t* ws = &wk.x;
-#pragma unroll
-            for (int c = 0; c < 4; ++c) {
-                const float2 f = F::unpack(xs[c]);
-                ss = fmaf(f.x, f.x, ss);
-                ss = fmaf(f.y, f.y, ss);
-                if constexpr (kFp8) {
-                    const float2 wf = has_w ? F::unpack(ws[c]) : make_float2(1.f, 1.f);
-                    pm = fmaxf(pm, fabsf(f.x * wf.x));
-                    pm = fmaxf(pm, fabsf(f.y * wf.y));
+                const int j = lr + k * tpr;
+                uint4 w = make_uint4(0, 0, 0, 0);
+                if constexpr (kHasW) {
+                    if (j < nvec) w = __ldg(wv + j);
                 }
+                pm = amax8<T, kHasW>(v[k], w, pm);
             }
         }
+        float ss = acc.x + acc.y;
 
         const int width = tpr < 32 ? tpr : 32;
         for (int o = width >> 1; o > 0; o >>= 1) {
@@ -215,7 +331,7 @@ __global__ void __launch_bounds__(max_block_for_vpt(VPT))
             if constexpr (kFp8) pm = fmaxf(pm, __shfl_xor_sync(0xffffffffu, pm, o));
         }
         if (wpr > 1) {
-            float2* slot = red + (static_cast<int64_t>(parity) * rpc + row_in_cta) * wpr;
+            float2* slot = red + (parity * rpc + row_in_cta) * wpr;
             if ((lr & 31) == 0) slot[lr >> 5] = make_float2(ss, pm);
             group_barrier(1 + row_in_cta, tpr);
             float s = 0.f, m = 0.f;
@@ -232,48 +348,45 @@ __global__ void __launch_bounds__(max_block_for_vpt(VPT))
         const float inv = 1.0f / sqrtf(ss / hf + a.eps);
 
         if constexpr (!kFp8) {
-            uint4* ov = static_cast<uint4*>(a.out);
+            uint4* orow = static_cast<uint4*>(a.out) + roff;
+            const float2 inv2 = make_float2(inv, inv);
 #pragma unroll
             for (int k = 0; k < VPT; ++k) {
-                const int64_t j = lr + static_cast<int64_t>(k) * tpr;
+                const int j = lr + k * tpr;
                 if (!(active && j < nvec)) continue;
-                const uint4 wk = has_w ? __ldg(wv + j) : make_uint4(0, 0, 0, 0);
-                const uint32_t* xs = &v[k].x;
-                const uint32_t* ws = &wk.x;
-                uint4 o;
-                uint32_t* os = &o.x;
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const float2 f = F::unpack(xs[c]);
-                    const float2 wf = has_w ? F::unpack(ws[c]) : make_float2(1.f, 1.f);
-                    os[c] = F::pack((f.x * wf.x) * inv, (f.y * wf.y) * inv);
-                }
-                st_v4(ov + roff + j, o);
+                uint4 w = make_uint4(0, 0, 0, 0);
+                if constexpr (kHasW) w = __ldg(wv + j);
+                st_v4(orow + j, scale8<T, kHasW>(v[k], w, inv2));
             }
         } else {
             const float qmul = pm > 0.f ? 448.0f / pm : 0.f;
+            const float2 q2 = make_float2(qmul, qmul);
             if (active && lr == 0) a.scale[row] = pm > 0.f ? (pm * inv) / 448.0f : 0.f;
-            uint2* qv = reinterpret_cast<uint2*>(a.q);
+            uint2* qrow = reinterpret_cast<uint2*>(a.q) + roff;
 #pragma unroll
             for (int k = 0; k < VPT; ++k) {
-                const int64_t j = lr + static_cast<int64_t>(k) * tpr;
+                const int j = lr + k * tpr;
                 if (!(active && j < nvec)) continue;
-                const uint4 wk = has_w ? __ldg(wv + j) : make_uint4(0, 0, 0, 0);
-                const uint32_t* xs = &v[k].x;
-                const uint32_t* ws = &wk.x;
-                uint32_t e[4];
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const float2 f = F::unpack(xs[c]);
-                    const float2 wf = has_w ? F::unpack(ws[c]) : make_float2(1.f, 1.f);
-                    e[c] = e4m3x2((f.x * wf.x) * qmul, (f.y * wf.y) * qmul);
-                }
-                uint2 o = make_uint2(e[0] | (e[1] << 16), e[2] | (e[3] << 16));
+                uint4 w = make_uint4(0, 0, 0, 0);
+                if constexpr (kHasW) w = __ldg(wv + j);
+                uint2 o = quant8<T, kHasW>(v[k], w, q2);
                 if (!(pm > 0.f)) o = make_uint2(0, 0);
-                st_v2(qv + roff + j, o);
+                st_v2(qrow + j, o);
             }
         }
     }
+}
+
+template <typename T, int VPT, int OP>
+__global__ void __launch_bounds__(max_block_for_vpt(VPT))
+    rn_vector_kernel(const Args a, const int tpr, const int rpc) {
+    extern __shared__ float2 red[];  // [2][rpc][warps per row]
+    pdl_allow_dependents();
+    pdl_wait_for_prior_grid();
+    if (a.weight)
+        vector_rows<T, VPT, OP, true>(a, tpr, rpc, red);
+    else
+        vector_rows<T, VPT, OP, false>(a, tpr, rpc, red);
 }
 
 // ---------------------------------------------------------------- staged kernel
@@ -282,12 +395,13 @@ __global__ void __launch_bounds__(max_block_for_vpt(VPT))
 // into a ring of `stages` shared-memory slots with one bulk asynchronous copy
 // per row and tensor (cp.async.bulk, completion counted on an mbarrier), up
 // to `stages` rows ahead, so the bytes in flight per SM are set by shared
-// memory rather than by registers. All threads then make two passes over the
-// staged row: (1) residual add, write-back (global, and over the x slot in
-// shared memory), sum of squares [and max |v * w|]; (2) the output. CTA b owns
-// rows b, b + gridDim.x, ... Every mbarrier wait is bounded; on a timeout the
-// CTA records kErrWaitTimeout in g_rn_device_error, waits (bounded) for the
-// copies it issued, and returns.
+// memory rather than by registers. The weight is widened to fp32 into shared
+// memory once per CTA. All threads then make two passes over the staged row:
+// (1) residual add, write-back (global, and over the x slot in shared memory),
+// sum of squares [and max |v * w|]; (2) the output. CTA b owns rows
+// b, b + gridDim.x, ... Every mbarrier wait is bounded; on a timeout the CTA
+// records kErrWaitTimeout in g_rn_device_error, waits (bounded) for the copies
+// it issued, and returns.
 
 __device__ unsigned int g_rn_device_error = 0;
 
@@ -346,28 +460,27 @@ __device__ __forceinline__ uint64_t policy_evict_first() {
     return p;
 }
 
-template <typename T, int OP>
-__global__ void __launch_bounds__(1024)
-    rn_staged_kernel(const Args a, const int stages, const uint32_t slot_bytes) {
-    using F = Fmt<T>;
+template <typename T, int OP, bool kHasW>
+__device__ __forceinline__ void staged_rows(const Args& a, const int stages,
+                                            const uint32_t slot_bytes, unsigned char* smem) {
     constexpr bool kFused = OP != kRmsNorm;
     constexpr bool kFp8 = OP == kFusedAddFp8;
     constexpr int kSlots = kFused ? 2 : 1;  // x [, residual] per stage
-    extern __shared__ __align__(128) unsigned char smem[];
 
     const int tid = threadIdx.x;
     const int nthr = blockDim.x;
     const int nwarps = nthr >> 5;
-    const int64_t nvec = a.H >> 3;
+    const int nvec = static_cast<int>(a.H >> 3);
     const uint32_t row_bytes = static_cast<uint32_t>(a.H) * 2u;
     const uint32_t stage_bytes = kSlots * slot_bytes;
     const int64_t G = gridDim.x;
     const int64_t first = blockIdx.x;
     const int64_t nrows = first < a.T ? (a.T - 1 - first) / G + 1 : 0;
-    uint64_t* bars = reinterpret_cast<uint64_t*>(smem + static_cast<size_t>(stages) * stage_bytes);
+    // layout: [stages x stage][fp32 weight, 4H bytes][mbarriers][reduction]
+    float4* wf = reinterpret_cast<float4*>(smem + static_cast<size_t>(stages) * stage_bytes);
+    uint64_t* bars = reinterpret_cast<uint64_t*>(reinterpret_cast<unsigned char*>(wf) +
+                                                 static_cast<size_t>(a.H) * 4);
     float2* red = reinterpret_cast<float2*>(bars + stages);
-    const uint4* __restrict__ wv = static_cast<const uint4*>(a.weight);
-    const bool has_w = wv != nullptr;
     const float hf = static_cast<float>(a.H);
     const char* xg = static_cast<const char*>(a.x);
     char* rg = static_cast<char*>(a.residual);
@@ -379,8 +492,6 @@ __global__ void __launch_bounds__(1024)
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
         asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
     }
-    __syncthreads();
-
     auto issue = [&](int s, int64_t row) {
         const uint32_t bar = smem_u32(bars + s);
         const uint32_t dst = smem_u32(smem + static_cast<size_t>(s) * stage_bytes);
@@ -388,6 +499,15 @@ __global__ void __launch_bounds__(1024)
         bulk_load(dst, xg + row * row_bytes, row_bytes, bar, policy);
         if constexpr (kFused) bulk_load(dst + slot_bytes, rg + row * row_bytes, row_bytes, bar, policy);
     };
+    if constexpr (kHasW) {
+        const uint4* wv = static_cast<const uint4*>(a.weight);
+        for (int j = tid; j < nvec; j += nthr) {
+            const W8 w = w8_from_bits<T>(__ldg(wv + j));
+            wf[2 * j] = make_float4(w.w[0].x, w.w[0].y, w.w[1].x, w.w[1].y);
+            wf[2 * j + 1] = make_float4(w.w[2].x, w.w[2].y, w.w[3].x, w.w[3].y);
+        }
+    }
+    __syncthreads();
     if (tid == 0) {
         for (int s = 0; s < stages && s < nrows; ++s) issue(s, first + s * G);
     }
@@ -399,44 +519,29 @@ __global__ void __launch_bounds__(1024)
         const int64_t row = first + k * G;
         const bool ok = mbar_wait(smem_u32(bars + s), parity);
         uint4* sx = reinterpret_cast<uint4*>(smem + static_cast<size_t>(s) * stage_bytes);
-        const uint4* sr = reinterpret_cast<const uint4*>(smem + static_cast<size_t>(s) * stage_bytes + slot_bytes);
+        const uint4* sr = reinterpret_cast<const uint4*>(reinterpret_cast<unsigned char*>(sx) + slot_bytes);
 
         // pass 1: [residual add + write-back], sum of squares [, max |v * w|]
-        float ss = 0.f, pm = 0.f;
+        float2 acc = make_float2(0.f, 0.f);
+        float pm = 0.f;
         if (ok) {
-            for (int64_t j = tid; j < nvec; j += nthr) {
+            uint4* rrow = reinterpret_cast<uint4*>(rg + row * row_bytes);
+            for (int j = tid; j < nvec; j += nthr) {
                 uint4 v = sx[j];
-                uint32_t* vs = &v.x;
                 if constexpr (kFused) {
-                    const uint4 r = sr[j];
-                    const uint32_t* rs = &r.x;
-#pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const float2 fx = F::unpack(vs[c]);
-                        const float2 fr = F::unpack(rs[c]);
-                        vs[c] = F::pack(fx.x + fr.x, fx.y + fr.y);
-                    }
-                    st_v4(reinterpret_cast<uint4*>(rg + row * row_bytes) + j, v);
+                    v = add8<T>(v, sr[j]);
+                    st_v4(rrow + j, v);
                     sx[j] = v;
                 }
-                uint4 w4 = make_uint4(0, 0, 0, 0);
+                acc = ssq8<T>(v, acc);
                 if constexpr (kFp8) {
-                    if (has_w) w4 = __ldg(wv + j);
-                }
-                const uint32_t* ws = &w4.x;
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const float2 f = F::unpack(vs[c]);
-                    ss = fmaf(f.x, f.x, ss);
-                    ss = fmaf(f.y, f.y, ss);
-                    if constexpr (kFp8) {
-                        const float2 wf = has_w ? F::unpack(ws[c]) : make_float2(1.f, 1.f);
-                        pm = fmaxf(pm, fabsf(f.x * wf.x));
-                        pm = fmaxf(pm, fabsf(f.y * wf.y));
-                    }
+                    W8 w{};
+                    if constexpr (kHasW) w = w8_from_f32(wf + 2 * j);
+                    pm = amax8<T, kHasW>(v, w, pm);
                 }
             }
         }
+        float ss = acc.x + acc.y;
 #pragma unroll
         for (int o = 16; o > 0; o >>= 1) {
             ss += __shfl_xor_sync(0xffffffffu, ss, o);
@@ -460,38 +565,21 @@ __global__ void __launch_bounds__(1024)
         // pass 2: outputs from the staged (written-back) row
         if constexpr (!kFp8) {
             uint4* og = reinterpret_cast<uint4*>(static_cast<char*>(a.out) + row * row_bytes);
-            for (int64_t j = tid; j < nvec; j += nthr) {
-                const uint4 v = sx[j];
-                const uint4 w4 = has_w ? __ldg(wv + j) : make_uint4(0, 0, 0, 0);
-                const uint32_t* vs = &v.x;
-                const uint32_t* ws = &w4.x;
-                uint4 o;
-                uint32_t* os = &o.x;
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const float2 f = F::unpack(vs[c]);
-                    const float2 wf = has_w ? F::unpack(ws[c]) : make_float2(1.f, 1.f);
-                    os[c] = F::pack((f.x * wf.x) * inv, (f.y * wf.y) * inv);
-                }
-                st_v4(og + j, o);
+            const float2 inv2 = make_float2(inv, inv);
+            for (int j = tid; j < nvec; j += nthr) {
+                W8 w{};
+                if constexpr (kHasW) w = w8_from_f32(wf + 2 * j);
+                st_v4(og + j, scale8<T, kHasW>(sx[j], w, inv2));
             }
         } else {
             const float qmul = pm > 0.f ? 448.0f / pm : 0.f;
+            const float2 q2 = make_float2(qmul, qmul);
             if (tid == 0) a.scale[row] = pm > 0.f ? (pm * inv) / 448.0f : 0.f;
             uint2* qg = reinterpret_cast<uint2*>(a.q + row * a.H);
-            for (int64_t j = tid; j < nvec; j += nthr) {
-                const uint4 v = sx[j];
-                const uint4 w4 = has_w ? __ldg(wv + j) : make_uint4(0, 0, 0, 0);
-                const uint32_t* vs = &v.x;
-                const uint32_t* ws = &w4.x;
-                uint32_t e[4];
-#pragma unroll
-                for (int c = 0; c < 4; ++c) {
-                    const float2 f = F::unpack(vs[c]);
-                    const float2 wf = has_w ? F::unpack(ws[c]) : make_float2(1.f, 1.f);
-                    e[c] = e4m3x2((f.x * wf.x) * qmul, (f.y * wf.y) * qmul);
-                }
-                uint2 o = make_uint2(e[0] | (e[1] << 16), e[2] | (e[3] << 16));
+            for (int j = tid; j < nvec; j += nthr) {
+                W8 w{};
+                if constexpr (kHasW) w = w8_from_f32(wf + 2 * j);
+                uint2 o = quant8<T, kHasW>(sx[j], w, q2);
                 if (!(pm > 0.f)) o = make_uint2(0, 0);
                 st_v2(qg + j, o);
             }
@@ -512,6 +600,18 @@ __global__ void __launch_bounds__(1024)
     }
 }
 
+template <typename T, int OP>
+__global__ void __launch_bounds__(1024)
+    rn_staged_kernel(const Args a, const int stages, const uint32_t slot_bytes) {
+    extern __shared__ __align__(128) unsigned char smem[];
+    pdl_allow_dependents();
+    pdl_wait_for_prior_grid();
+    if (a.weight)
+        staged_rows<T, OP, true>(a, stages, slot_bytes, smem);
+    else
+        staged_rows<T, OP, false>(a, stages, slot_bytes, smem);
+}
+
 // ---------------------------------------------------------------- scalar kernel
 
 constexpr int kScalarBlock = 256;
@@ -522,6 +622,8 @@ __global__ void __launch_bounds__(kScalarBlock) rn_scalar_kernel(const Args a) {
     constexpr bool kFused = OP != kRmsNorm;
     constexpr bool kFp8 = OP == kFusedAddFp8;
     __shared__ float2 red[kScalarBlock / 32];
+    pdl_allow_dependents();
+    pdl_wait_for_prior_grid();
     const int lane = threadIdx.x & 31;
     const int warp = threadIdx.x >> 5;
     const float hf = static_cast<float>(a.H);
@@ -573,11 +675,30 @@ __global__ void __launch_bounds__(kScalarBlock) rn_scalar_kernel(const Args a) {
 
 // ---------------------------------------------------------------- dispatch
 
+// Launches `kernel` with the plan's shape, with the PDL attribute when asked.
+template <typename... KArgs, typename... Args2>
+cudaError_t launch_kernel(void (*kernel)(KArgs...), const Launch& l, cudaStream_t s,
+                          Args2&&... args) {
+    if (l.pdl) {
+        cudaLaunchConfig_t cfg = {};
+        cfg.gridDim = dim3(static_cast<unsigned>(l.grid));
+        cfg.blockDim = dim3(static_cast<unsigned>(l.block));
+        cfg.dynamicSmemBytes = static_cast<size_t>(l.smem);
+        cfg.stream = s;
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        return cudaLaunchKernelEx(&cfg, kernel, std::forward<Args2>(args)...);
+    }
+    kernel<<<static_cast<unsigned>(l.grid), l.block, l.smem, s>>>(std::forward<Args2>(args)...);
+    return cudaGetLastError();
+}
+
 template <typename T, int OP, int VPT>
 cudaError_t launch_vector(const Args& a, const Launch& l, cudaStream_t s) {
-    rn_vector_kernel<T, VPT, OP><<<static_cast<unsigned>(l.grid), l.block, l.smem, s>>>(a, l.tpr,
-                                                                                        l.rpc);
-    return cudaGetLastError();
+    return launch_kernel(rn_vector_kernel<T, VPT, OP>, l, s, a, l.tpr, l.rpc);
 }
 
 template <typename T, int OP, int I = 0>
@@ -614,12 +735,12 @@ cudaError_t launch_typed(const Args& a, const Launch& l, cudaStream_t s) {
         cudaError_t e = prepare_staged<T, OP>(l.smem);
         if (e != cudaSuccess) return e;
         const uint32_t slot = static_cast<uint32_t>(((a.H * 2 + 127) / 128) * 128);
-        rn_staged_kernel<T, OP><<<static_cast<unsigned>(l.grid), l.block, l.smem, s>>>(a, l.vpt,
-                                                                                       slot);
-        return cudaGetLastError();
+        return launch_kernel(rn_staged_kernel<T, OP>, l, s, a, l.vpt, slot);
     }
-    rn_scalar_kernel<T, OP><<<static_cast<unsigned>(l.grid), kScalarBlock, 0, s>>>(a);
-    return cudaGetLastError();
+    Launch ls = l;
+    ls.block = kScalarBlock;
+    ls.smem = 0;
+    return launch_kernel(rn_scalar_kernel<T, OP>, ls, s, a);
 }
 
 template <typename T>

@@ -29,6 +29,7 @@ struct Launch {
     int block;   // threads per CTA
     int smem;    // dynamic shared memory bytes
     int64_t grid;
+    bool pdl;    // launch with programmatic stream serialization (PDL)
 };
 
 enum Op { kRmsNorm = 0, kFusedAdd = 1, kFusedAddFp8 = 2 };

@@ -113,7 +113,7 @@ def test_sub_warp_and_idle_slot_shapes(op):
 
 STAGED_SHAPES = [  # (H, ctas per SM, stages, threads, T)
     (3840, 4, 3, 256, 1000), (3840, 1, 2, 96, 7), (4096, 2, 6, 256, 333), (512, 4, 8, 64, 777),
-    (16384, 1, 3, 1024, 150), (2048, 4, 5, 32, 1), (7168, 2, 3, 448, 300), (8, 4, 4, 32, 50),
+    (16384, 1, 2, 1024, 150), (2048, 4, 5, 32, 1), (7168, 2, 3, 448, 300), (8, 4, 4, 32, 50),
     (5120, 2, 5, 320, 597),
 ]
 

@@ -456,6 +456,118 @@ def run_e2e(args, rn, wl, S, device, stream):
                    "launches, both launches through the C ABI, D2H of residual, out, q, scale"}
 
 
+# ----------------------------------------------------------------------------- sweep
+
+def sweep_cells():
+    """Every (workload, op, dtype, T, H) cell of the named workloads."""
+    cells = [("small", "rms_norm", "bf16", 8, 512)]
+    for dt in ("bf16", "fp16"):
+        for T in synth.DECODE_T:
+            cells.append(("decode", "fused_add_rms_norm", dt, T, 4096))
+    cells.append(("outlier", "fused_add_rms_norm_fp8", "bf16", 64, 16384))
+    cells.append(("prefill", "fused_add_rms_norm", "bf16", T_PREFILL, H_PREFILL))
+    cells.append(("prefill", "fused_add_rms_norm_fp8", "bf16", T_PREFILL, H_PREFILL))
+    for op in ("rms_norm", "fused_add_rms_norm", "fused_add_rms_norm_fp8"):
+        for dt in ("bf16", "fp16"):
+            for T in synth.SWEEP_T:
+                for H in synth.SWEEP_H:
+                    cells.append(("sweep", op, dt, T, H))
+    return cells
+
+
+def time_cell(rn, name, op, dtype, T, H, iters, device, mem_cap_bytes=24 << 30):
+    """Median-free mean time per launch over `iters` launches that rotate
+    over buffer sets totalling >= 4x L2 (capped by memory), eager stream
+    launches; plus CUDA-graph replay time for launches under 30 us."""
+    wl = synth.make_inputs(name, op, dtype, T, H, device=device)
+    dt = wl.dtype
+    l2 = torch.cuda.get_device_properties(device).L2_cache_size
+    per = 2 * T * H * (1 if op == "rms_norm" else 3) + (T * H + 4 * T if op.endswith("fp8") else 0)
+    n = max(2, math.ceil(4 * l2 / max(per, 1)) + 1)
+    n = max(1, min(n, mem_cap_bytes // max(per, 1)))
+    sets = []
+    for _ in range(n):
+        s = {"x": wl.x.clone(), "r": None if wl.residual is None else wl.residual.clone()}
+        if op.endswith("fp8"):
+            s["q"] = torch.empty(T, H, dtype=torch.float8_e4m3fn, device=device)
+            s["scale"] = torch.empty(T, dtype=torch.float32, device=device)
+        else:
+            s["out"] = torch.empty(T, H, dtype=dt, device=device)
+        sets.append(s)
+    w, eps = wl.weight, wl.eps
+    del wl
+
+    def launch(i):
+        s = sets[i % n]
+        if op == "rms_norm":
+            rn.rms_norm(s["out"], s["x"], w, eps)
+        elif op == "fused_add_rms_norm":
+            rn.fused_add_rms_norm(s["out"], s["x"], s["r"], w, eps)
+        else:
+            rn.fused_add_rms_norm_fp8(s["q"], s["scale"], s["x"], s["r"], w, eps)
+
+    for i in range(5):
+        launch(i)
+    torch.cuda.synchronize(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(iters):
+        launch(i)
+    e1.record()
+    torch.cuda.synchronize(device)
+    us = e0.elapsed_time(e1) / iters * 1e3
+    graph_us = None
+    if us < 30:
+        g = torch.cuda.CUDAGraph()
+        st = torch.cuda.Stream(device)
+        with torch.cuda.stream(st):
+            launch(0)
+            torch.cuda.synchronize(device)
+            with torch.cuda.graph(g, stream=st):
+                for i in range(100):
+                    launch(i)
+        torch.cuda.synchronize(device)
+        g.replay()
+        torch.cuda.synchronize(device)
+        e0.record()
+        for _ in range(5):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize(device)
+        graph_us = e0.elapsed_time(e1) / 500 * 1e3
+        del g
+    plan = rn.plan_launch(op, dt, T, H)
+    del sets
+    torch.cuda.empty_cache()
+    return us, graph_us, plan, n
+
+
+def run_sweep(args, world, rank, local):
+    import residual_add_rmsnorm_rms_b200 as rn
+    device = torch.device("cuda", local)
+    torch.cuda.set_device(device)
+    peak, _ = measured_peak()
+    out = open(args.sweep_out, "w")
+    for name, op, dtype, T, H in sweep_cells():
+        us, gus, plan, nsets = time_cell(rn, name, op, dtype, T, H, args.sweep_iters, device)
+        nbytes = op_bytes(op, T, H)
+        best = gus if gus is not None else us
+        rec = {"workload": name, "op": op, "dtype": dtype, "T": T, "H": H,
+               "us": round(us, 3), "graph_us": None if gus is None else round(gus, 3),
+               "gbs": round(nbytes / us / 1e3, 1), "graph_gbs": None if gus is None else
+               round(nbytes / gus / 1e3, 1), "rows_per_s": round(T / (best / 1e6), 1),
+               "frac_of_8tbs": round(nbytes / best / 1e3 / NOMINAL_HBM_GBS, 4),
+               "frac_of_measured": round(nbytes / best / 1e3 / peak, 4),
+               "bytes": nbytes, "buffer_sets": nsets,
+               "kernel": {0: "vector", 1: "scalar", 2: "staged"}[plan["kernel"]],
+               "tpr": plan["threads_per_row"], "vpt": plan["vectors_per_thread"]}
+        out.write(json.dumps(rec) + "\n")
+        out.flush()
+    out.close()
+    assert rn.device_errors() == 0
+    print(json.dumps({"sweep": args.sweep_out, "cells": len(sweep_cells())}))
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__.splitlines()[0])
     ap.add_argument("--gpus", type=int, default=1)
@@ -466,6 +578,10 @@ def main():
                     help="skip the oracle timing (for profiler runs)")
     ap.add_argument("--reference-rows", type=int, default=1024,
                     help="rows of the prefill batch per reference (oracle) step")
+    ap.add_argument("--sweep-out", default=None,
+                    help="instead of the step benchmark, time every workload cell and write "
+                         "one JSON line per cell to this file")
+    ap.add_argument("--sweep-iters", type=int, default=50)
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours" and not args.no_cpu_baseline:
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)
@@ -473,7 +589,9 @@ def main():
     if world != args.gpus:
         args.gpus = world if world > 1 else args.gpus
     try:
-        if args.impl == "reference":
+        if args.sweep_out:
+            run_sweep(args, world, rank, local)
+        elif args.impl == "reference":
             run_reference(args, world, rank)
         else:
             run_ours(args, world, rank, local)

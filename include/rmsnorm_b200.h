@@ -181,15 +181,18 @@ RN_API rn_status rn_validate(int32_t op, const rn_tensor* out_or_q, const rn_ten
                       const rn_tensor* x, const rn_tensor* residual, const rn_tensor* weight,
                       float eps, int64_t variance_size, rn_plan* plan);
 
-/* Test hook: force the vector kernel's (threads_per_row, vectors_per_thread)
- * for every later call in the process; (0, 0) restores automatic choice.
+/* Test hook: force the vector kernel's (threads_per_row, vectors_per_thread,
+ * rows_per_cta; rows_per_cta 0 = automatic) for every later call in the
+ * process; (0, 0, 0) restores automatic choice. rows_per_cta is clamped to
+ * what the block limit and the named barriers allow.
  * threads_per_row must be a power of two <= 32 or a multiple of 32 <= 1024,
  * and vectors_per_thread one of the compiled widths (see
  * rn_supported_vectors_per_thread); otherwise RN_ERR_CONFIG. A forced shape
  * that cannot cover a row (threads_per_row * vectors_per_thread * 8 < H) or
  * exceeds the kernel's block limit falls back to the scalar kernel. Not
  * thread-safe with concurrent launches; meant for tests and tuning. */
-RN_API rn_status rn_force_plan(int32_t threads_per_row, int32_t vectors_per_thread);
+RN_API rn_status rn_force_plan(int32_t threads_per_row, int32_t vectors_per_thread,
+                                int32_t rows_per_cta);
 
 /* Test hook: force the STAGED kernel with `ctas_per_sm` resident blocks per SM
  * (1, 2 or 4), `stages` ring slots (>= 2) and `threads` per block (a multiple

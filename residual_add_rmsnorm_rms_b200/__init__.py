@@ -96,7 +96,7 @@ def _load():
     L.rn_plan_launch.restype = ctypes.c_int
     L.rn_validate.argtypes = [ctypes.c_int32, P, P, P, P, P, F, I64, ctypes.POINTER(RnPlan)]
     L.rn_validate.restype = ctypes.c_int
-    L.rn_force_plan.argtypes = [ctypes.c_int32, ctypes.c_int32]
+    L.rn_force_plan.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32]
     L.rn_force_plan.restype = ctypes.c_int
     L.rn_force_staged.argtypes = [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32]
     L.rn_force_staged.restype = ctypes.c_int
@@ -249,9 +249,9 @@ def validate(op: str, out_or_q, x, residual=None, weight=None, eps: float = 1e-6
     return STATUS.get(st, str(st)), p.as_dict()
 
 
-def force_plan(threads_per_row: int, vectors_per_thread: int) -> None:
+def force_plan(threads_per_row: int, vectors_per_thread: int, rows_per_cta: int = 0) -> None:
     """Test/tuning hook: force the vector kernel's shape; (0, 0) restores auto."""
-    _check(lib.rn_force_plan(threads_per_row, vectors_per_thread), "rn_force_plan")
+    _check(lib.rn_force_plan(threads_per_row, vectors_per_thread, rows_per_cta), "rn_force_plan")
 
 
 def force_staged(ctas_per_sm: int, stages: int, threads: int) -> None:

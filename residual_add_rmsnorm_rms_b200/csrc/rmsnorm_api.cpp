@@ -22,6 +22,7 @@ namespace {
 thread_local char g_cuda_error[256] = "";
 std::atomic<int> g_force_tpr{0};
 std::atomic<int> g_force_vpt{0};
+std::atomic<int> g_force_rpc{0};
 std::atomic<int> g_force_staged_c{0};
 std::atomic<int> g_force_staged_s{0};
 std::atomic<int> g_force_staged_t{0};
@@ -127,9 +128,11 @@ int tpr_for(int64_t nvec, int vpt) {
     return static_cast<int>(((need + 31) / 32) * 32);
 }
 
-void fill_vector_plan(int tpr, int vpt, int64_t T, rn_plan* p) {
+void fill_vector_plan(int tpr, int vpt, int64_t T, rn_plan* p, int want_rpc = 0) {
     // Aim for ~256-thread blocks: several rows per block for narrow rows.
-    int rpc = tpr >= 256 ? 1 : 256 / tpr;
+    int rpc = want_rpc > 0 ? want_rpc : (tpr >= 256 ? 1 : 256 / tpr);
+    while (rpc > 1 && tpr * rpc > rn::max_block_for_vpt(vpt)) --rpc;
+    if (tpr < 32) rpc = ((rpc + 32 / tpr - 1) / (32 / tpr)) * (32 / tpr);  // whole warps
     rpc = clamp_rpc(rpc, tpr, T);
     p->kernel = RN_KERNEL_VECTOR;
     p->threads_per_row = tpr;
@@ -179,45 +182,65 @@ void fill_scalar_plan(int64_t T, rn_plan* p) {
     p->grid = T;
 }
 
-// Automatic choice of (threads per row, vectors per thread) for the vector
-// kernel. Candidates cover the row with at most 1/16 idle slots and respect
-// the per-width block limit; among them, many rows favour wide per-thread
-// work (fewer threads per row: fewer cross-warp steps), few rows favour more
-// threads per row (more parallelism and bytes in flight per row).
-bool auto_vector_plan(int64_t T, int64_t H, rn_plan* p) {
+// Automatic choice of (threads per row, vectors per thread, rows per block)
+// for the vector kernel, from a sweep of forced shapes on B200 (H 2048..16384,
+// T 1..32768, all three ops):
+//  * many rows (T x threads-per-row at 4 vectors/thread >= two full waves of
+//    1024 threads per SM): 4 vectors per thread (<= 64 registers, so 32 warps
+//    per SM stay resident with 64 bytes of loads in flight per thread and
+//    tensor), tolerating up to 1/8 idle vector slots; rows per block such
+//    that a block holds ~256 threads (~512 when T >= 16384, where coarser
+//    blocks cost less at the tail), two rows for 129..256 threads per row,
+//    one above;
+//  * few rows (decode): about 256 threads per row (512 for H > 4096) with
+//    the fewest vectors per thread that cover the row (more threads per row
+//    buy latency, not bandwidth, past that point); rows per block as above
+//    but never fewer blocks than SMs.
+int rows_per_block(int tpr, int64_t T) {
+    if (tpr <= 128) return (T >= 16384 ? 512 : 256) / tpr;
+    if (tpr <= 256) return 2;
+    return 1;
+}
+
+bool auto_vector_plan(int64_t T, int64_t H, int num_sms, rn_plan* p) {
     const int64_t nvec = H / 8;
-    const int64_t kFillThreads = 148LL * 1024;  // one full wave of resident threads
-    int best_tpr = 0, best_vpt = 0;
-    double best_score = -1e300;
+    auto idle_of = [&](int tpr, int vpt) {
+        const int64_t slots = static_cast<int64_t>(tpr) * vpt;
+        return static_cast<double>(slots - nvec) / static_cast<double>(slots);
+    };
+    const int tpr4 = tpr_for(nvec, 4);
+    const bool many_rows = tpr4 <= rn::max_block_for_vpt(4) &&
+                           static_cast<double>(T) * tpr4 >= 2.0 * num_sms * 1024;
+    if (many_rows) {
+        for (int vpt : {4, 5, 3, 6, 8, 2}) {
+            const int tpr = tpr_for(nvec, vpt);
+            if (tpr > rn::max_block_for_vpt(vpt) || idle_of(tpr, vpt) > 1.0 / 8) continue;
+            fill_vector_plan(tpr, vpt, T, p, rows_per_block(tpr, T));
+            return true;
+        }
+    }
+    const int target = nvec <= 512 ? 256 : 512;
+    for (int i = 0; i < rn::kNumVpt; ++i) {
+        const int vpt = rn::kVptList[i];
+        const int tpr = tpr_for(nvec, vpt);
+        if (tpr > target || tpr > rn::max_block_for_vpt(vpt) || idle_of(tpr, vpt) > 1.0 / 8)
+            continue;
+        // narrow rows share a block, but keep at least one block per SM
+        int rpc = rows_per_block(tpr, T);
+        const int64_t per_sm = T / num_sms > 0 ? T / num_sms : 1;
+        if (rpc > per_sm) rpc = static_cast<int>(per_sm);
+        fill_vector_plan(tpr, vpt, T, p, rpc);
+        return true;
+    }
+    // Rows too wide for the preferred targets: any width that fits.
     for (int i = 0; i < rn::kNumVpt; ++i) {
         const int vpt = rn::kVptList[i];
         const int tpr = tpr_for(nvec, vpt);
         if (tpr > rn::max_block_for_vpt(vpt)) continue;
-        const int64_t slots = static_cast<int64_t>(tpr) * vpt;
-        const double idle = static_cast<double>(slots - nvec) / static_cast<double>(slots);
-        const double threads = static_cast<double>(T) * tpr;
-        double score;
-        if (threads >= 4.0 * kFillThreads) {
-            // Plenty of rows: 4 vectors per thread keeps the kernel at <= 64
-            // registers (32 resident warps per SM) with 64 bytes of loads in
-            // flight per thread per tensor; measured best on B200 for H in
-            // 3840..16384 even with up to 1/8 idle slots.
-            if (idle > 1.0 / 8) continue;
-            score = -std::abs(vpt - 4) * 1.0 - idle * 4;
-        } else {
-            if (idle > 1.0 / 16) continue;
-            // Few rows: prefer the most threads per row (latency-bound).
-            score = static_cast<double>(tpr) / 1024.0 - idle * 8 - (vpt > 8 ? 1 : 0);
-        }
-        if (score > best_score) {
-            best_score = score;
-            best_tpr = tpr;
-            best_vpt = vpt;
-        }
+        fill_vector_plan(tpr, vpt, T, p, 1);
+        return true;
     }
-    if (!best_tpr) return false;
-    fill_vector_plan(best_tpr, best_vpt, T, p);
-    return true;
+    return false;
 }
 
 rn_status plan_shape(int op, int64_t T, int64_t H, bool vector_ok, int num_sms, rn_plan* p);
@@ -250,7 +273,7 @@ rn_status plan_shape(int op, int64_t T, int64_t H, bool vector_ok, int num_sms, 
     if (ftpr && fvpt) {
         const int64_t nvec = H / 8;
         if (static_cast<int64_t>(ftpr) * fvpt >= nvec && ftpr <= rn::max_block_for_vpt(fvpt)) {
-            fill_vector_plan(ftpr, fvpt, T, p);
+            fill_vector_plan(ftpr, fvpt, T, p, g_force_rpc.load());
         } else {
             fill_scalar_plan(T, p);
         }
@@ -258,8 +281,7 @@ rn_status plan_shape(int op, int64_t T, int64_t H, bool vector_ok, int num_sms, 
     }
     // The STAGED kernel is chosen only when forced: measured on B200 it trails
     // the VECTOR kernel at every shape tried (T up to 65536, H 2048..16384).
-    (void)num_sms;
-    if (!auto_vector_plan(T, H, p)) fill_scalar_plan(T, p);
+    if (!auto_vector_plan(T, H, num_sms, p)) fill_scalar_plan(T, p);
     return RN_OK;
 }
 
@@ -531,13 +553,18 @@ rn_status rn_device_errors(uint32_t* flags) {
     return RN_OK;
 }
 
-rn_status rn_force_plan(int32_t threads_per_row, int32_t vectors_per_thread) {
+rn_status rn_force_plan(int32_t threads_per_row, int32_t vectors_per_thread,
+                        int32_t rows_per_cta) {
     if (threads_per_row == 0 && vectors_per_thread == 0) {
         g_force_tpr.store(0);
         g_force_vpt.store(0);
+        g_force_rpc.store(0);
         return RN_OK;
     }
-    if (!tpr_valid(threads_per_row) || !vpt_compiled(vectors_per_thread)) return RN_ERR_CONFIG;
+    if (!tpr_valid(threads_per_row) || !vpt_compiled(vectors_per_thread) || rows_per_cta < 0 ||
+        rows_per_cta > 1024)
+        return RN_ERR_CONFIG;
+    g_force_rpc.store(rows_per_cta);
     g_force_vpt.store(vectors_per_thread);
     g_force_tpr.store(threads_per_row);
     return RN_OK;

@@ -185,14 +185,15 @@ void fill_scalar_plan(int64_t T, rn_plan* p) {
 // Automatic choice of (threads per row, vectors per thread, rows per block)
 // for the vector kernel, from a sweep of forced shapes on B200 (H 2048..16384,
 // T 1..32768, all three ops):
-//  * many rows (T x threads-per-row at 4 vectors/thread >= two full waves of
+//  * many rows (T x threads-per-row at 4 vectors/thread >= one full wave of
 //    1024 threads per SM): 4 vectors per thread (<= 64 registers, so 32 warps
 //    per SM stay resident with 64 bytes of loads in flight per thread and
 //    tensor), tolerating up to 1/8 idle vector slots; rows per block such
 //    that a block holds ~256 threads (~512 when T >= 16384, where coarser
 //    blocks cost less at the tail), two rows for 129..256 threads per row,
 //    one above;
-//  * few rows (decode): about 256 threads per row (512 for H > 4096) with
+//  * few rows (decode): about 256 threads per row (512 for H > 4096; 1024 for
+//    H >= 16384 with T <= 64) with
 //    the fewest vectors per thread that cover the row (more threads per row
 //    buy latency, not bandwidth, past that point); rows per block as above
 //    but never fewer blocks than SMs.
@@ -210,7 +211,7 @@ bool auto_vector_plan(int64_t T, int64_t H, int num_sms, rn_plan* p) {
     };
     const int tpr4 = tpr_for(nvec, 4);
     const bool many_rows = tpr4 <= rn::max_block_for_vpt(4) &&
-                           static_cast<double>(T) * tpr4 >= 2.0 * num_sms * 1024;
+                           static_cast<double>(T) * tpr4 >= 1.0 * num_sms * 1024;
     if (many_rows) {
         for (int vpt : {4, 5, 3, 6, 8, 2}) {
             const int tpr = tpr_for(nvec, vpt);
@@ -219,7 +220,8 @@ bool auto_vector_plan(int64_t T, int64_t H, int num_sms, rn_plan* p) {
             return true;
         }
     }
-    const int target = nvec <= 512 ? 256 : 512;
+    // very few very wide rows: every extra thread per row shortens the row
+    const int target = (nvec >= 2048 && T <= 64) ? 1024 : (nvec <= 512 ? 256 : 512);
     for (int i = 0; i < rn::kNumVpt; ++i) {
         const int vpt = rn::kVptList[i];
         const int tpr = tpr_for(nvec, vpt);

@@ -52,6 +52,8 @@ def op_bytes(op: str, T: int, H: int, esize: int = 2) -> int:
         return 2 * esize * H * T + esize * H          # read x, write out; weight
     if op == "fused_add_rms_norm":
         return 4 * esize * H * T + esize * H          # read x, r; write r, out; weight
+    if op == "silu_and_mul_fp8":                      # H = I: read gate, up; write q, scale
+        return (2 * esize + 1) * H * T + 4 * T
     return (3 * esize + 1) * H * T + 4 * T + esize * H  # read x, r; write r, q, scale; weight
 
 
@@ -67,7 +69,7 @@ def kernel_digest(plan: dict) -> str:
     the launch shape the planner gives it on the bench's workload."""
     h = hashlib.sha256()
     d = os.path.join(ROOT, "residual_add_rmsnorm_rms_b200", "csrc")
-    for name in ("rmsnorm_kernels.cu", "rn_internal.h"):
+    for name in ("rmsnorm_kernels.cu", "rn_device.cuh", "rn_internal.h"):
         with open(os.path.join(d, name), "rb") as f:
             h.update(name.encode() + f.read())
     shape = {k: plan[k] for k in ("kernel", "threads_per_row", "vectors_per_thread",
@@ -477,6 +479,9 @@ def sweep_cells():
     cells.append(("outlier", "fused_add_rms_norm_fp8", "bf16", 64, 16384))
     cells.append(("prefill", "fused_add_rms_norm", "bf16", T_PREFILL, H_PREFILL))
     cells.append(("prefill", "fused_add_rms_norm_fp8", "bf16", T_PREFILL, H_PREFILL))
+    for dt in ("bf16", "fp16"):
+        for T in synth.SWIGLU_T:
+            cells.append(("swiglu", "silu_and_mul_fp8", dt, T, synth.SWIGLU_I))
     for op in ("rms_norm", "fused_add_rms_norm", "fused_add_rms_norm_fp8"):
         for dt in ("bf16", "fp16"):
             for T in synth.SWEEP_T:
@@ -492,13 +497,16 @@ def time_cell(rn, name, op, dtype, T, H, iters, device, mem_cap_bytes=24 << 30):
     wl = synth.make_inputs(name, op, dtype, T, H, device=device)
     dt = wl.dtype
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
-    per = 2 * T * H * (1 if op == "rms_norm" else 3) + (T * H + 4 * T if op.endswith("fp8") else 0)
+    per = op_bytes(op, T, H)
     n = max(2, math.ceil(4 * l2 / max(per, 1)) + 1)
     n = max(1, min(n, mem_cap_bytes // max(per, 1)))
     sets = []
     for _ in range(n):
         s = {"x": wl.x.clone(), "r": None if wl.residual is None else wl.residual.clone()}
-        if op.endswith("fp8"):
+        if op == "silu_and_mul_fp8":
+            s["q"] = torch.empty(T, H, dtype=torch.float8_e4m3fn, device=device)
+            s["scale"] = torch.empty(T, dtype=torch.float32, device=device)
+        elif op.endswith("fp8"):
             s["q"] = torch.empty(T, H, dtype=torch.float8_e4m3fn, device=device)
             s["scale"] = torch.empty(T, dtype=torch.float32, device=device)
         else:
@@ -513,6 +521,8 @@ def time_cell(rn, name, op, dtype, T, H, iters, device, mem_cap_bytes=24 << 30):
             rn.rms_norm(s["out"], s["x"], w, eps)
         elif op == "fused_add_rms_norm":
             rn.fused_add_rms_norm(s["out"], s["x"], s["r"], w, eps)
+        elif op == "silu_and_mul_fp8":
+            rn.silu_and_mul_fp8(s["q"], s["scale"], s["x"])
         else:
             rn.fused_add_rms_norm_fp8(s["q"], s["scale"], s["x"], s["r"], w, eps)
 

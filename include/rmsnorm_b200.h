@@ -136,6 +136,21 @@ RN_API rn_status rn_fused_add_rms_norm_fp8(const rn_tensor* q, const rn_tensor* 
                                     const rn_tensor* weight, float eps,
                                     int64_t variance_size, void* stream);
 
+/* silu_and_mul_fp8: the fused SwiGLU + per-token dynamic FP8 cast, the
+ * second kernel of "Custom CUDA kernels juice Llama 3.1 405B on AMD MI300X,
+ * skipping Nvidia lock-in" ("the SwiGLU activation function, again merging
+ * it with an FP8 cast"). Per row of x = [gate | up] ([T x 2I], fp16/bf16,
+ * gate in the first half): y_i = silu(gate_i) * up_i with silu(a) =
+ * a / (1 + e^-a) in fp32 (fast exponential; relative error of y below 2e-6
+ * for |gate| <= 6), scale[t] = max|y| / 448, q = e4m3fn(RNE, satfinite)
+ * (y / scale); a row with max|y| = 0 gets scale 0 and zero codes.
+ * q: [T x I] RN_E4M3 dense; scale: T RN_F32 dense; x: any view whose flattening
+ * to [T x 2I] is free (the rules of the norm ops). 2I must be even.
+ * Validation, streams, aliasing (q and scale overlap nothing) and T == 0 as
+ * for the norm ops. */
+RN_API rn_status rn_silu_and_mul_fp8(const rn_tensor* q, const rn_tensor* scale,
+                                     const rn_tensor* x, void* stream);
+
 /* Static text for a status code (never NULL). */
 RN_API const char* rn_status_string(rn_status status);
 

@@ -62,6 +62,8 @@ def _load():
         for f in (lib.oracle_rms_norm, lib.oracle_fused_add_rms_norm,
                   lib.oracle_fused_add_rms_norm_fp8):
             f.restype = I
+        lib.oracle_silu_and_mul_fp8.argtypes = [P, I, I64, I64, P, P, P, P]
+        lib.oracle_silu_and_mul_fp8.restype = I
         lib.oracle_decode16_array.argtypes = [P, I, I64, P]
         lib.oracle_encode16_array.argtypes = [P, I, I64, P]
         lib.oracle_decode_e4m3_array.argtypes = [P, I64, P]
@@ -213,6 +215,29 @@ def fused_add_rms_norm_fp8(x, residual, weight, dtype: str, eps: float,
 
     _run(blk, T, H, threads)
     return (r_out, q, scale, y) if want_y else (r_out, q, scale)
+
+
+def silu_and_mul_fp8(x, dtype: str, want_y: bool = False, threads: int = 1):
+    """x: [T x 2I] 16-bit bits, gate first. Returns (q [T x I], scale [T][, y])."""
+    lib = _load()
+    xb = _bits16(x)
+    T, H2 = _shape2d(xb)
+    if H2 % 2:
+        raise ValueError("x must have an even last dimension")
+    I = H2 // 2
+    q = np.empty((T, I), np.uint8)
+    scale = np.empty((T,), np.float32)
+    y = np.empty((T, I), np.float64) if want_y else None
+    dt = DTYPES[dtype]
+
+    def blk(t0, t1, row, yrow):
+        rc = lib.oracle_silu_and_mul_fp8(_ptr(xb[t0:t1]), dt, t1 - t0, I, _ptr(q[t0:t1]),
+                                         _ptr(scale[t0:t1]), None if y is None else _ptr(y[t0:t1]),
+                                         _ptr(yrow))
+        assert rc == 0
+
+    _run(blk, T, I, threads)
+    return (q, scale, y) if want_y else (q, scale)
 
 
 def usable_cores() -> int:

@@ -295,3 +295,33 @@ void oracle_decode_e4m3_array(const uint8_t* in, int64_t n, double* out) {
 void oracle_encode_e4m3_array(const double* in, int64_t n, uint8_t* out) {
     for (int64_t i = 0; i < n; ++i) out[i] = oracle_f64_to_e4m3_satfinite(in[i]);
 }
+
+/* ------------------------------------------------------------------------ */
+/* Fused SwiGLU + per-token FP8 cast, the second kernel of "Custom CUDA      */
+/* kernels juice Llama 3.1 405B on AMD MI300X, skipping Nvidia lock-in".    */
+/* Row t of x holds [gate | up] (2I values). y_i = silu(gate_i) * up_i with */
+/* silu(a) = a / (1 + e^-a) (libm exp, binary64); amax = max |y_i|;        */
+/* s = amax / 448; q_i = E4M3(y_i / s); the stored scale is (float)s; a row */
+/* with amax == 0 gets s = 0 and zero codes.                                */
+int oracle_silu_and_mul_fp8(const uint16_t* x, int dtype, int64_t T, int64_t I, uint8_t* q,
+                            float* scale, double* y_out, double* yrow) {
+    if ((dtype != OR_F16 && dtype != OR_BF16) || I <= 0 || T < 0) return -1;
+    for (int64_t t = 0; t < T; ++t) {
+        const uint16_t* xr = x + t * 2 * I;
+        double amax = 0.0;
+        for (int64_t i = 0; i < I; ++i) {
+            double a = load16(xr, i, dtype);
+            double b = load16(xr, I + i, dtype);
+            double y = a / (1.0 + exp(-a)) * b;
+            yrow[i] = y;
+            if (fabs(y) > amax) amax = fabs(y);
+        }
+        double s = amax / 448.0;
+        scale[t] = (float)s;
+        for (int64_t i = 0; i < I; ++i) {
+            q[t * I + i] = amax > 0.0 ? oracle_f64_to_e4m3_satfinite(yrow[i] / s) : 0;
+            if (y_out) y_out[t * I + i] = yrow[i];
+        }
+    }
+    return 0;
+}

@@ -24,6 +24,7 @@ import torch
 
 __all__ = [
     "RmsNormError", "rms_norm", "fused_add_rms_norm", "fused_add_rms_norm_fp8",
+    "silu_and_mul_fp8",
     "plan_launch", "validate", "force_plan", "force_staged", "set_launch_options", "device_errors", "supported_vectors_per_thread", "status_string",
     "LIB_PATH", "lib", "RnTensor", "RnPlan", "STATUS", "OPS",
 ]
@@ -87,6 +88,8 @@ def _load():
     L.rn_fused_add_rms_norm_fp8.argtypes = [P, P, P, P, P, F, I64, VP]
     for f in (L.rn_rms_norm, L.rn_fused_add_rms_norm, L.rn_fused_add_rms_norm_fp8):
         f.restype = ctypes.c_int
+    L.rn_silu_and_mul_fp8.argtypes = [P, P, P, VP]
+    L.rn_silu_and_mul_fp8.restype = ctypes.c_int
     L.rn_status_string.argtypes = [ctypes.c_int]
     L.rn_status_string.restype = ctypes.c_char_p
     L.rn_last_cuda_error.argtypes = []
@@ -223,6 +226,14 @@ def fused_add_rms_norm_fp8(q: torch.Tensor, scale: torch.Tensor, x: torch.Tensor
                _desc(residual, 3), None if weight is None else _desc(weight, 4), eps,
                _vs(variance_size), s)
     _check(st, "rn_fused_add_rms_norm_fp8")
+
+
+def silu_and_mul_fp8(q: torch.Tensor, scale: torch.Tensor, x: torch.Tensor, stream=None) -> None:
+    """Fused SwiGLU + per-token e4m3 cast (C ABI rn_silu_and_mul_fp8): x = [gate | up]
+    ([..., 2I]); q (float8_e4m3fn or uint8, [..., I]); scale (float32, T values)."""
+    dev, s = _stream_for((q, scale, x), stream)
+    st = _call(lib.rn_silu_and_mul_fp8, dev, _desc(q, 0), _desc(scale, 1), _desc(x, 2), s)
+    _check(st, "rn_silu_and_mul_fp8")
 
 
 def plan_launch(op: str, dtype: torch.dtype, T: int, H: int, vector_ok: bool = True) -> dict:

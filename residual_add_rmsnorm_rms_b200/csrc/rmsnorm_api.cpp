@@ -245,12 +245,15 @@ bool auto_vector_plan(int64_t T, int64_t H, int num_sms, rn_plan* p) {
     return false;
 }
 
-rn_status plan_shape(int op, int64_t T, int64_t H, bool vector_ok, int num_sms, rn_plan* p);
+rn_status plan_shape(int op, int64_t T, int64_t H, bool vector_ok, int num_sms, rn_plan* p,
+                     bool allow_staged);
 
 // The launch plan: the kernel and its shape, then the grid cap (the kernels
-// stride over the rows a capped grid does not cover).
-rn_status plan_impl(int op, int64_t T, int64_t H, bool vector_ok, int num_sms, rn_plan* p) {
-    const rn_status st = plan_shape(op, T, H, vector_ok, num_sms, p);
+// stride over the rows a capped grid does not cover). `allow_staged` is false
+// for kernels that have no staged form.
+rn_status plan_impl(int op, int64_t T, int64_t H, bool vector_ok, int num_sms, rn_plan* p,
+                    bool allow_staged = true) {
+    const rn_status st = plan_shape(op, T, H, vector_ok, num_sms, p, allow_staged);
     if (st != RN_OK) return st;
     long long cap = g_max_grid.load();
     if (cap == 0 && p->kernel == RN_KERNEL_VECTOR)
@@ -260,7 +263,8 @@ rn_status plan_impl(int op, int64_t T, int64_t H, bool vector_ok, int num_sms, r
     return RN_OK;
 }
 
-rn_status plan_shape(int op, int64_t T, int64_t H, bool vector_ok, int num_sms, rn_plan* p) {
+rn_status plan_shape(int op, int64_t T, int64_t H, bool vector_ok, int num_sms, rn_plan* p,
+                     bool allow_staged) {
     if (H < 1 || T < 0) return RN_ERR_SHAPE;
     std::memset(p, 0, sizeof *p);
     if (!vector_ok || H % 8 != 0) {
@@ -269,7 +273,8 @@ rn_status plan_shape(int op, int64_t T, int64_t H, bool vector_ok, int num_sms, 
     }
     const int fc = g_force_staged_c.load(), fs = g_force_staged_s.load(),
               ft = g_force_staged_t.load();
-    if (fc && fs && ft && fill_staged_plan(op, T, H, fc, fs, ft, num_sms, p)) return RN_OK;
+    if (allow_staged && fc && fs && ft && fill_staged_plan(op, T, H, fc, fs, ft, num_sms, p))
+        return RN_OK;
     std::memset(p, 0, sizeof *p);
     const int ftpr = g_force_tpr.load(), fvpt = g_force_vpt.load();
     if (ftpr && fvpt) {
@@ -478,6 +483,50 @@ rn_status rn_fused_add_rms_norm_fp8(const rn_tensor* q, const rn_tensor* scale,
                                     const rn_tensor* weight, float eps, int64_t variance_size,
                                     void* stream) {
     return run(rn::kFusedAddFp8, q, scale, x, residual, weight, eps, variance_size, stream);
+}
+
+rn_status rn_silu_and_mul_fp8(const rn_tensor* q, const rn_tensor* scale, const rn_tensor* x,
+                              void* stream) {
+    if (!q || !scale || !x) return RN_ERR_NULL;
+    if (!is16(x->dtype) || q->dtype != RN_E4M3 || scale->dtype != RN_F32) return RN_ERR_DTYPE;
+    Flat fx, fq, fs;
+    rn_status st = flatten(x, &fx);
+    if (st != RN_OK) return st;
+    if (fx.H % 2 != 0) return RN_ERR_SHAPE;
+    const int64_t I = fx.H / 2;
+    if ((st = flatten(q, &fq)) != RN_OK) return st;
+    if (fq.H != I || fq.T != fx.T) return RN_ERR_SHAPE;
+    if (fx.T == 0) return RN_OK;
+    if ((st = flatten(scale, &fs)) != RN_OK) return st;
+    if (fs.numel != fx.T) return RN_ERR_SHAPE;
+    fs.esize = 4;
+    if (!fx.ptr || !fq.ptr || !fs.ptr) return RN_ERR_NULL;
+    if (!aligned(fx.ptr, 2) || !aligned(fs.ptr, 4)) return RN_ERR_LAYOUT;
+    if (overlap(fq, fx) || overlap(fs, fx) || overlap(fq, fs)) return RN_ERR_ALIAS;
+    const bool vector_ok = I % 8 == 0 && aligned(fx.ptr, 16) && aligned(fq.ptr, 8);
+    rn_plan plan;
+    // The row mapping of the fused norm op on I-wide rows: per output element
+    // it moves 2 x 2 bytes in and 1 byte out, within a few bytes of that op.
+    if ((st = plan_impl(rn::kFusedAddFp8, fx.T, I, vector_ok, device_sms(), &plan, false)) != RN_OK)
+        return st;
+    rn::SwigluArgs a{fx.ptr, reinterpret_cast<uint8_t*>(fq.ptr), reinterpret_cast<float*>(fs.ptr),
+                     fx.T, I};
+    rn::Launch l{plan.kernel == RN_KERNEL_VECTOR ? 0 : 1,
+                 plan.threads_per_row,
+                 plan.vectors_per_thread,
+                 plan.rows_per_cta,
+                 plan.block_threads,
+                 plan.smem_bytes,
+                 plan.grid,
+                 g_pdl.load() < 0 ? kPdlDefault : g_pdl.load() == 1};
+    const cudaError_t e = rn::launch_swiglu_fp8(x->dtype == RN_BF16 ? rn::kBF16 : rn::kF16, a, l,
+                                                static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) {
+        std::snprintf(g_cuda_error, sizeof g_cuda_error, "%s: %s", cudaGetErrorName(e),
+                      cudaGetErrorString(e));
+        return RN_ERR_CUDA;
+    }
+    return RN_OK;
 }
 
 rn_status rn_validate(int32_t op, const rn_tensor* out_or_q, const rn_tensor* scale,

@@ -21,6 +21,15 @@ struct Args {
     float eps;
 };
 
+// Operands of the fused SwiGLU + FP8 cast: x = [gate | up] rows of 2I.
+struct SwigluArgs {
+    const void* x;
+    uint8_t* q;
+    float* scale;
+    int64_t T;
+    int64_t I;
+};
+
 struct Launch {
     int kernel;  // 0 = vector, 1 = scalar, 2 = staged
     int tpr;     // threads per row
@@ -50,6 +59,9 @@ constexpr int kStagedSmemPerSm = 220 * 1024;
 
 // Enqueues one launch; returns the CUDA error of the launch itself.
 cudaError_t launch(int op, int dtype, const Args& a, const Launch& l, cudaStream_t s);
+
+// Enqueues the fused SwiGLU + FP8 cast (vector plan: kernel 0; scalar: 1).
+cudaError_t launch_swiglu_fp8(int dtype, const SwigluArgs& a, const Launch& l, cudaStream_t s);
 
 // Reads, and clears when set, the device-side error flags of the current
 // device (bit 0: an mbarrier wait timed out). Synchronous.

@@ -12,6 +12,9 @@ Ops (namespace ``rmsnorm_b200``; CUDA only, N-D inputs flattened to
 * ``rms_norm(x, weight, epsilon) -> out``
 * ``fused_add_rms_norm(x!, residual!, weight, epsilon) -> ()``: in place, as
   vLLM's fused op is used: residual := x + residual, x := rms_norm(residual)
+* ``silu_and_mul_fp8(x) -> (q, scale)``: x = [gate | up] over the last dim;
+  q (float8_e4m3fn, last dim halved), scale (float32, last dim 1): the fused
+  SwiGLU + per-token FP8 cast
 * ``fused_add_rms_norm_fp8(x, residual!, weight, epsilon) -> (q, scale)``:
   residual := x + residual; q (float8_e4m3fn, shape of x) and scale
   (float32, shape of x with the last dim 1) the per-token dynamic cast of
@@ -36,6 +39,7 @@ import torch
 from . import fused_add_rms_norm as _fused
 from . import fused_add_rms_norm_fp8 as _fused_fp8
 from . import rms_norm as _rms
+from . import silu_and_mul_fp8 as _silu_fp8
 
 __all__ = [
     "flatten_to_2d_is_free", "rms_no_var_16bit_only", "rms_add_no_var_16bit_only",
@@ -142,6 +146,22 @@ def _fused_add_rms_norm_fp8_op(x: torch.Tensor, residual: torch.Tensor,
 @_fused_add_rms_norm_fp8_op.register_fake
 def _(x, residual, weight, epsilon):
     return (_dense_like(x, torch.float8_e4m3fn),
+            torch.empty(x.shape[:-1] + (1,), dtype=torch.float32, device=x.device))
+
+
+@torch.library.custom_op(f"{LIB}::silu_and_mul_fp8", mutates_args=(), device_types="cuda")
+def _silu_and_mul_fp8_op(x: torch.Tensor) -> tuple[torch.Tensor, torch.Tensor]:
+    shape = x.shape[:-1] + (x.shape[-1] // 2,)
+    q = torch.empty(shape, dtype=torch.float8_e4m3fn, device=x.device)
+    scale = torch.empty(x.shape[:-1] + (1,), dtype=torch.float32, device=x.device)
+    _silu_fp8(q, scale, x)
+    return q, scale
+
+
+@_silu_and_mul_fp8_op.register_fake
+def _(x):
+    shape = x.shape[:-1] + (x.shape[-1] // 2,)
+    return (torch.empty(shape, dtype=torch.float8_e4m3fn, device=x.device),
             torch.empty(x.shape[:-1] + (1,), dtype=torch.float32, device=x.device))
 
 

@@ -22,6 +22,11 @@ Multiplies Run Slower"):
                in both, eps 1e-6.
 * ``prefill``  fused_add_rms_norm and fused_add_rms_norm_fp8, bf16, [8192 x 3840],
                x ~ Student-t(3) clipped to +-1e3, residual ~ N(0,16), eps 1e-6.
+* ``swiglu``   silu_and_mul_fp8, bf16 and fp16, x = [gate | up] of [T x 2I]
+               with I = 15360 (the Gemma 4 12B intermediate size: the
+               30720 x 3840 gate-up and 3840 x 15360 down projections in the
+               weight-shape table of "VLLM_ROCM_USE_AITER=1 slows Gemma 4 on an
+               AMD MI300X"), T in {1, 8, 64, 256, 8192}, gate, up ~ N(0,1).
 * ``sweep``    all three ops, bf16 and fp16, T in {1,16,256,4096,32768,65536} x
                H in {2048,4096,5120,7168,8192,16384}, x ~ N(0,1),
                residual ~ N(0,4), eps 1e-6.
@@ -47,12 +52,16 @@ __all__ = [
     "DECODE_T",
     "SWEEP_T",
     "SWEEP_H",
+    "SWIGLU_I",
+    "SWIGLU_T",
     "to_dtype",
 ]
 
 DECODE_T = (1, 8, 64, 256)
 SWEEP_T = (1, 16, 256, 4096, 32768, 65536)
 SWEEP_H = (2048, 4096, 5120, 7168, 8192, 16384)
+SWIGLU_I = 15360
+SWIGLU_T = (1, 8, 64, 256, 8192)
 
 
 def to_dtype(name: str) -> torch.dtype:
@@ -133,7 +142,7 @@ def make_inputs(name: str, op: str, dtype: str, T: int, H: int, device="cpu",
         seed = 0 if name == "small" else cell_seed(name, op, dtype, T, H)
     g = _gen(seed, device)
     outl = None
-    needs_res = op != "rms_norm"
+    needs_res = op not in ("rms_norm", "silu_and_mul_fp8")
     if name == "small":
         eps = 1e-6
         x = normal((T, H), 1.0, g, device)
@@ -154,6 +163,12 @@ def make_inputs(name: str, op: str, dtype: str, T: int, H: int, device="cpu",
         eps = 1e-6
         x = student_t3((T, H), 1e3, g, device)
         r = normal((T, H), 16.0, g, device) if needs_res else None
+    elif name == "swiglu":
+        # x = [gate | up] rows of 2 * H (H is the intermediate size I);
+        # gate, up ~ N(0, 1); no residual or weight
+        eps = 0.0
+        x = normal((T, 2 * H), 1.0, g, device)
+        r = None
     elif name == "sweep":
         eps = 1e-6
         x = normal((T, H), 1.0, g, device)

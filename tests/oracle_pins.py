@@ -353,4 +353,58 @@ def pin_zero_rows(orc, golden=None):
     assert np.isnan(y).all()  # 0/0 with eps = 0
 
 
+# ---------------------------------------------------------------- SwiGLU + FP8
+
+def _swiglu_inputs(dtype, T=16, I=512, seed=21):
+    wl = synth.make_inputs("swiglu", "silu_and_mul_fp8", dtype, T, I, seed=seed)
+    return wl.x
+
+
+def pin_swiglu_matches_torch_silu_float64(orc, golden=None):
+    """y = silu(gate) * up with gate the first half (torch.nn.functional.silu
+    in float64 as the library routine)."""
+    for dtype in ("bf16", "fp16"):
+        x = _swiglu_inputs(dtype)
+        q, scale, y = orc.silu_and_mul_fp8(bits16(x), dtype, want_y=True)
+        xd = x.double()
+        I = x.shape[1] // 2
+        ref = (torch.nn.functional.silu(xd[:, :I]) * xd[:, I:]).numpy()
+        np.testing.assert_allclose(y, ref, rtol=1e-14, atol=1e-300)
+        amax = np.abs(ref).max(axis=1)
+        np.testing.assert_allclose(scale, amax / 448.0, rtol=2 ** -24)
+
+
+def pin_swiglu_silu_identity(orc, golden=None):
+    """silu(a) - silu(-a) = a exactly in real arithmetic (sigma(-a) = 1 - sigma(a));
+    with up = 1 the oracle's y must satisfy it to binary64 rounding."""
+    for dtype in ("bf16", "fp16"):
+        g = torch.Generator().manual_seed(5)
+        a = synth.normal((4, 256), 4.0, g, "cpu").to(synth.to_dtype(dtype))
+        one = torch.ones_like(a)
+        xp = torch.cat([a, one], dim=1)
+        xn = torch.cat([-a, one], dim=1)
+        _, _, yp = orc.silu_and_mul_fp8(bits16(xp), dtype, want_y=True)
+        _, _, yn = orc.silu_and_mul_fp8(bits16(xn), dtype, want_y=True)
+        av = a.double().numpy()
+        np.testing.assert_allclose(yp - yn, av, rtol=1e-14, atol=1e-15)
+        # silu(0) = 0 and silu is positive for positive gates
+        x0 = torch.cat([torch.zeros(1, 8), torch.ones(1, 8)], dim=1).to(synth.to_dtype(dtype))
+        q0, s0, y0 = orc.silu_and_mul_fp8(bits16(x0), dtype, want_y=True)
+        assert (y0 == 0).all() and (s0 == 0).all() and (q0 == 0).all()
+        assert (yp[av > 0] > 0).all()
+
+
+def pin_swiglu_fp8_row_properties(orc, golden=None):
+    for dtype in ("bf16", "fp16"):
+        x = _swiglu_inputs(dtype, T=32, I=1024, seed=9)
+        q, scale, y = orc.silu_and_mul_fp8(bits16(x), dtype, want_y=True)
+        assert ((q == 0x7E) | (q == 0xFE)).any(axis=1).all()
+        assert not ((q & 0x7F) == 0x7F).any()
+        deq = torch.from_numpy(q.copy()).view(torch.float8_e4m3fn).double().numpy() \
+            * scale.astype(np.float64)[:, None]
+        amax = np.abs(y).max(axis=1)
+        half_step = np.maximum(np.abs(y) * 2.0 ** -4, 2.0 ** -10 * (amax / 448.0)[:, None])
+        assert (np.abs(deq - y) <= half_step * (1 + 1e-6)).all()
+
+
 PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

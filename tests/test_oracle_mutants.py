@@ -38,6 +38,14 @@ MUTANTS = {
                          "    return v;\n}\n\ndouble oracle_e4m3_to_f64"),
     "e4m3_bias_off_by_one": ("v = ldexp((double)(8 + m), e - 10);", "v = ldexp((double)(8 + m), e - 11);"),
     "e4m3_no_saturation": ("if (r > 448.0) r = 448.0;", "if (r > 480.0) r = 480.0;"),
+    "swiglu_sign_of_exponent": ("double y = a / (1.0 + exp(-a)) * b;",
+                                "double y = a / (1.0 + exp(a)) * b;"),
+    "swiglu_halves_swapped": ("double y = a / (1.0 + exp(-a)) * b;",
+                              "double y = b / (1.0 + exp(-b)) * a;"),
+    "swiglu_no_gate_in_numerator": ("double y = a / (1.0 + exp(-a)) * b;",
+                                    "double y = 1.0 / (1.0 + exp(-a)) * b;"),
+    "swiglu_scale_240": ("double s = amax / 448.0;\n        scale[t] = (float)s;\n        for (int64_t i = 0; i < I; ++i) {",
+                         "double s = amax / 240.0;\n        scale[t] = (float)s;\n        for (int64_t i = 0; i < I; ++i) {"),
     "bf16_overflow_threshold": ("if (r > maxf) return sign | 0x7f80; /* overflow to infinity */",
                                 "if (r >= maxf) return sign | 0x7f80;"),
 }

@@ -568,7 +568,10 @@ def run_sweep(args, world, rank, local):
     torch.cuda.set_device(device)
     peak, _ = measured_peak()
     out = open(args.sweep_out, "w")
-    for name, op, dtype, T, H in sweep_cells():
+    want = [w for w in (args.sweep_filter or "").split(",") if w]
+    cells = [c for c in sweep_cells() if all(w in (c[0], c[1], c[2], str(c[3]), str(c[4]))
+                                              for w in want)]
+    for name, op, dtype, T, H in cells:
         us, gus, plan, nsets = time_cell(rn, name, op, dtype, T, H, args.sweep_iters, device)
         nbytes = op_bytes(op, T, H)
         best = gus if gus is not None else us
@@ -585,7 +588,7 @@ def run_sweep(args, world, rank, local):
         out.flush()
     out.close()
     assert rn.device_errors() == 0
-    print(json.dumps({"sweep": args.sweep_out, "cells": len(sweep_cells())}))
+    print(json.dumps({"sweep": args.sweep_out, "cells": len(cells)}))
 
 
 def main():
@@ -602,6 +605,9 @@ def main():
                     help="instead of the step benchmark, time every workload cell and write "
                          "one JSON line per cell to this file")
     ap.add_argument("--sweep-iters", type=int, default=50)
+    ap.add_argument("--sweep-filter", default=None,
+                    help="comma-separated values a cell must all match (workload, op, dtype, "
+                         "T or H), e.g. swiglu,bf16,8192")
     args = ap.parse_args()
     if args.warmup < 3 and args.impl == "ours" and not args.no_cpu_baseline:
         print("warning: fewer than 3 warm-up steps", file=sys.stderr)

@@ -159,7 +159,12 @@ RN_API const char* rn_last_cuda_error(void);
 
 /* ---- launch planning (introspection; no memory is touched) ------------- */
 
-typedef enum { RN_OP_RMS_NORM = 0, RN_OP_FUSED_ADD = 1, RN_OP_FUSED_ADD_FP8 = 2 } rn_op;
+typedef enum {
+    RN_OP_RMS_NORM = 0,
+    RN_OP_FUSED_ADD = 1,
+    RN_OP_FUSED_ADD_FP8 = 2,
+    RN_OP_SILU_AND_MUL_FP8 = 3 /* rn_plan_launch only: H is I, the output width */
+} rn_op;
 /* Kernels: VECTOR keeps each row in registers (a group of threads per row);
  * STAGED is persistent and streams whole rows into a shared-memory ring with
  * bulk asynchronous copies (one block per row at a time); SCALAR handles

@@ -37,6 +37,7 @@ STATUS = {
     9: "RN_ERR_CUDA", 10: "RN_ERR_CONFIG",
 }
 OPS = {"rms_norm": 0, "fused_add_rms_norm": 1, "fused_add_rms_norm_fp8": 2}
+PLAN_OPS = dict(OPS, silu_and_mul_fp8=3)
 _DTYPES = {torch.float16: 0, torch.bfloat16: 1, torch.float8_e4m3fn: 2, torch.float32: 3,
            torch.uint8: 2}
 
@@ -239,7 +240,7 @@ def silu_and_mul_fp8(q: torch.Tensor, scale: torch.Tensor, x: torch.Tensor, stre
 def plan_launch(op: str, dtype: torch.dtype, T: int, H: int, vector_ok: bool = True) -> dict:
     """The launch shape the library picks (pure host logic; no GPU needed)."""
     p = RnPlan()
-    st = lib.rn_plan_launch(OPS[op], _DTYPES[dtype], T, H, int(vector_ok), ctypes.byref(p))
+    st = lib.rn_plan_launch(PLAN_OPS[op], _DTYPES[dtype], T, H, int(vector_ok), ctypes.byref(p))
     _check(st, "rn_plan_launch")
     return p.as_dict()
 

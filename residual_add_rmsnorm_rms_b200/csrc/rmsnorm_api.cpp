@@ -563,8 +563,10 @@ const char* rn_last_cuda_error(void) { return g_cuda_error; }
 rn_status rn_plan_launch(int32_t op, int32_t dtype, int64_t T, int64_t H, int32_t vector_ok,
                          rn_plan* plan) {
     if (!plan) return RN_ERR_NULL;
-    if (op < 0 || op > 2) return RN_ERR_CONFIG;
+    if (op < 0 || op > 3) return RN_ERR_CONFIG;
     if (!is16(dtype)) return RN_ERR_DTYPE;
+    if (op == RN_OP_SILU_AND_MUL_FP8)
+        return plan_impl(rn::kFusedAddFp8, T, H, vector_ok != 0, kDefaultSms, plan, false);
     return plan_impl(op, T, H, vector_ok != 0, kDefaultSms, plan);
 }
 

@@ -141,8 +141,9 @@ RN_API rn_status rn_fused_add_rms_norm_fp8(const rn_tensor* q, const rn_tensor* 
  * skipping Nvidia lock-in" ("the SwiGLU activation function, again merging
  * it with an FP8 cast"). Per row of x = [gate | up] ([T x 2I], fp16/bf16,
  * gate in the first half): y_i = silu(gate_i) * up_i with silu(a) =
- * a / (1 + e^-a) in fp32 (fast exponential; relative error of y below 2e-6
- * for |gate| <= 6), scale[t] = max|y| / 448, q = e4m3fn(RNE, satfinite)
+ * a / (1 + e^-a) in fp32 (fast exponential and division; relative error of y
+ * below 1e-6 for |gate| <= 6; silu(a) = 0 for a < -87.3, where its true
+ * magnitude is below 1e-36), scale[t] = max|y| / 448, q = e4m3fn(RNE, satfinite)
  * (y / scale); a row with max|y| = 0 gets scale 0 and zero codes.
  * q: [T x I] RN_E4M3 dense; scale: T RN_F32 dense; x: any view whose flattening
  * to [T x 2I] is free (the rules of the norm ops). 2I must be even.

@@ -12,9 +12,9 @@
 // threads per row, VPT 16-byte vectors of gate and of up per thread, all
 // loads issued before use, one max-reduction per row (warp butterfly, then a
 // named barrier across the row's warps), one pass writing the codes. silu
-// uses the fast exponential intrinsic (__expf, documented error 2 + 1.173|a|
-// ulp) and an IEEE reciprocal: at ~1.3e12 elements/s an accurate exponential
-// would make the kernel issue-bound.
+// uses the fast exponential and division intrinsics (two multi-function-unit
+// operations per element): at ~1.3e12 elements/s the accurate forms would
+// make the kernel issue-bound.
 #include <cstdint>
 
 #include "rn_device.cuh"
@@ -23,10 +23,13 @@
 namespace rn {
 namespace {
 
-// silu(g) * u for a pair, in fp32.
+// silu(g) * u for a pair, in fp32: fast exponential and fast division
+// intrinsics (documented errors: 2 + 1.173|g| ulp and 2 ulp), one rounding for
+// the up product. For g < -87.3 the divisor exceeds 2^126 and the fast
+// division returns 0: silu(g) is then below 1e-36 in magnitude.
 __device__ __forceinline__ float2 swiglu2(float2 g, float2 u) {
-    const float sx = g.x * __frcp_rn(1.0f + __expf(-g.x));
-    const float sy = g.y * __frcp_rn(1.0f + __expf(-g.y));
+    const float sx = __fdividef(g.x, 1.0f + __expf(-g.x));
+    const float sy = __fdividef(g.y, 1.0f + __expf(-g.y));
     return __fmul2_rn(make_float2(sx, sy), u);
 }
 

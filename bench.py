@@ -562,6 +562,53 @@ def time_cell(rn, name, op, dtype, T, H, iters, device, mem_cap_bytes=24 << 30):
     return us, graph_us, plan, n
 
 
+# (N, K) of Gemma 4 12B's fp8 linear layers (weight-shape table of
+# "VLLM_ROCM_USE_AITER=1 slows Gemma 4 on an AMD MI300X")
+GEMMA_NK = ((8192, 3840), (9216, 3840), (30720, 3840), (3840, 4096), (3840, 8192), (3840, 15360))
+GEMM_M = (1, 64, 256, 8192)
+
+
+def measured_fp8_peak():
+    """Dense fp8 tensor peak: the measured bf16 figure x the nominal fp8/bf16
+    ratio (4.5 / 2.25 PFLOP/s)."""
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(p) as f:
+            j = json.load(f)
+        return 2.0 * float(j["bf16_tflops"]), "2 x measured bf16 burst (MEASURED_PEAKS.json)"
+    except (OSError, KeyError, ValueError):
+        return 2.0 * 1590.0, "2 x fallback bf16 1.59 PFLOP/s"
+
+
+def time_gemm_cell(rn, M, N, K, iters, device):
+    g = torch.Generator(device=device).manual_seed(M + N + K)
+    n_sets = max(2, math.ceil(4 * torch.cuda.get_device_properties(device).L2_cache_size
+                              / (N * K + M * K + 2 * M * N)) + 1)
+    n_sets = min(n_sets, 8)
+    sets = []
+    for _ in range(n_sets):
+        a = (torch.randn(M, K, generator=g, device=device) * 40).clamp_(-448, 448)
+        b = (torch.randn(N, K, generator=g, device=device) * 40).clamp_(-448, 448)
+        sets.append((torch.empty(M, N, dtype=torch.bfloat16, device=device),
+                     a.to(torch.float8_e4m3fn), b.to(torch.float8_e4m3fn),
+                     torch.rand(M, generator=g, device=device) * 0.01,
+                     torch.rand(N, generator=g, device=device) * 0.01))
+        del a, b
+    for i in range(3):
+        rn.fp8_rowwise_gemm(*sets[i % n_sets])
+    torch.cuda.synchronize(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(iters):
+        rn.fp8_rowwise_gemm(*sets[i % n_sets])
+    e1.record()
+    torch.cuda.synchronize(device)
+    us = e0.elapsed_time(e1) / iters * 1e3
+    del sets
+    torch.cuda.empty_cache()
+    return us
+
+
 def run_sweep(args, world, rank, local):
     import residual_add_rmsnorm_rms_b200 as rn
     device = torch.device("cuda", local)
@@ -586,9 +633,22 @@ def run_sweep(args, world, rank, local):
                "tpr": plan["threads_per_row"], "vpt": plan["vectors_per_thread"]}
         out.write(json.dumps(rec) + "\n")
         out.flush()
+    gemm_cells = [(M, N, K) for (N, K) in GEMMA_NK for M in GEMM_M
+                  if all(w in ("gemm", "fp8_rowwise_gemm", str(M), f"{N}x{K}") for w in want)]
+    fp8_peak, fp8_src = measured_fp8_peak()
+    for M, N, K in gemm_cells:
+        us = time_gemm_cell(rn, M, N, K, args.sweep_iters, device)
+        tflops = 2.0 * M * N * K / us / 1e6
+        rec = {"workload": "gemm", "op": "fp8_rowwise_gemm", "dtype": "e4m3", "M": M, "N": N,
+               "K": K, "us": round(us, 3), "tflops": round(tflops, 1),
+               "frac_of_fp8_peak": round(tflops / fp8_peak, 4), "fp8_peak_tflops": fp8_peak,
+               "peak_source": fp8_src,
+               "weight_gbs": round(N * K / us / 1e3, 1)}
+        out.write(json.dumps(rec) + "\n")
+        out.flush()
     out.close()
     assert rn.device_errors() == 0
-    print(json.dumps({"sweep": args.sweep_out, "cells": len(cells)}))
+    print(json.dumps({"sweep": args.sweep_out, "cells": len(cells) + len(gemm_cells)}))
 
 
 def main():

@@ -152,6 +152,23 @@ RN_API rn_status rn_fused_add_rms_norm_fp8(const rn_tensor* q, const rn_tensor* 
 RN_API rn_status rn_silu_and_mul_fp8(const rn_tensor* q, const rn_tensor* scale,
                                      const rn_tensor* x, void* stream);
 
+/* fp8_rowwise_gemm: D[m, n] = bf16(b_scale[n] * (a_scale[m] * sum_k A[m, k] *
+ * B[n, k])), with fp32 accumulation on the tensor cores (tcgen05) and one
+ * rounding to bf16. The consumer of fused_add_rms_norm_fp8's codes and
+ * per-token scales: A is [M x K] e4m3 (row-major, as q), a_scale has M fp32
+ * values (as scale), B is an [N x K] e4m3 weight (row-major: K contiguous)
+ * with one fp32 scale per output channel in b_scale, and D is [M x N] bf16
+ * row-major. Row-wise fp8 linear layers appear in the table of
+ * "VLLM_ROCM_USE_AITER=1 slows Gemma 4 on an AMD MI300X"
+ * (RowWiseTorchFP8ScaledMMLinearKernel).
+ * Requirements: dense views (flattening rule of the norm ops), K % 16 == 0,
+ * N % 8 == 0, 16-byte-aligned A, B and D, K, N and M below 2^31; D must not
+ * overlap any input. M == 0 is a no-op. Needs no workspace. Asynchronous on
+ * `stream`; validation errors return before any CUDA call. */
+RN_API rn_status rn_fp8_rowwise_gemm(const rn_tensor* d, const rn_tensor* a,
+                                     const rn_tensor* b, const rn_tensor* a_scale,
+                                     const rn_tensor* b_scale, void* stream);
+
 /* Static text for a status code (never NULL). */
 RN_API const char* rn_status_string(rn_status status);
 

@@ -64,6 +64,8 @@ def _load():
             f.restype = I
         lib.oracle_silu_and_mul_fp8.argtypes = [P, I, I64, I64, P, P, P, P]
         lib.oracle_silu_and_mul_fp8.restype = I
+        lib.oracle_fp8_rowwise_gemm.argtypes = [P, P, P, P, I64, I64, I64, I64, I64, P, P]
+        lib.oracle_fp8_rowwise_gemm.restype = I
         lib.oracle_decode16_array.argtypes = [P, I, I64, P]
         lib.oracle_encode16_array.argtypes = [P, I, I64, P]
         lib.oracle_decode_e4m3_array.argtypes = [P, I64, P]
@@ -238,6 +240,36 @@ def silu_and_mul_fp8(x, dtype: str, want_y: bool = False, threads: int = 1):
 
     _run(blk, T, I, threads)
     return (q, scale, y) if want_y else (q, scale)
+
+
+def fp8_rowwise_gemm(a_codes, b_codes, a_scale, b_scale, rows=None, want_y: bool = False,
+                     threads: int = 1):
+    """D = bf16((A @ B^T) * a_scale[:, None] * b_scale[None, :]) from e4m3 codes
+    (uint8, A [M x K], B [N x K]). `rows` (sorted indices) restricts the rows
+    computed; the result then holds those rows only. Returns D bits [, y]."""
+    lib = _load()
+    A = np.ascontiguousarray(a_codes, dtype=np.uint8)
+    B = np.ascontiguousarray(b_codes, dtype=np.uint8)
+    sa = np.ascontiguousarray(a_scale, dtype=np.float32).reshape(-1)
+    sb = np.ascontiguousarray(b_scale, dtype=np.float32).reshape(-1)
+    M, K = A.shape
+    N = B.shape[0]
+    if B.shape[1] != K or sa.size != M or sb.size != N:
+        raise ValueError("shape mismatch")
+    if rows is not None:
+        rows = np.asarray(rows, dtype=np.int64)
+        A, sa = np.ascontiguousarray(A[rows]), np.ascontiguousarray(sa[rows])
+        M = A.shape[0]
+    D = np.empty((M, N), np.uint16)
+    y = np.empty((M, N), np.float64) if want_y else None
+
+    def blk(t0, t1, row, yrow):
+        rc = lib.oracle_fp8_rowwise_gemm(_ptr(A), _ptr(B), _ptr(sa), _ptr(sb), M, N, K, t0, t1,
+                                         _ptr(D), None if y is None else _ptr(y))
+        assert rc == 0
+
+    _run(blk, M, 1, threads)
+    return (D, y) if want_y else D
 
 
 def usable_cores() -> int:

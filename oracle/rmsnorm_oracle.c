@@ -325,3 +325,32 @@ int oracle_silu_and_mul_fp8(const uint16_t* x, int dtype, int64_t T, int64_t I, 
     }
     return 0;
 }
+
+/* ------------------------------------------------------------------------ */
+/* Row-wise scaled fp8 GEMM, the consumer of the per-token codes (the fp8   */
+/* linear layers of "VLLM_ROCM_USE_AITER=1 slows Gemma 4 on an AMD MI300X"):*/
+/*   D[m, n] = RNE_bf16( (sum_k A[m, k] * B[n, k]) * a_scale[m] * b_scale[n] ) */
+/* A [M x K] and B [N x K] are e4m3fn codes. Every product of two e4m3      */
+/* values is an integer multiple of 2^-18 below 2^18, so the binary64 sum of */
+/* up to 2^17 products is exact: the only roundings are the two scale       */
+/* products and the final cast. Rows m in [m0, m1) only (the caller may     */
+/* sample rows); d_out (nullable) receives the unrounded values.            */
+int oracle_fp8_rowwise_gemm(const uint8_t* A, const uint8_t* B, const float* a_scale,
+                            const float* b_scale, int64_t M, int64_t N, int64_t K, int64_t m0,
+                            int64_t m1, uint16_t* D, double* d_out) {
+    if (M < 0 || N <= 0 || K <= 0 || K > (1 << 17) || m0 < 0 || m1 > M || m0 > m1) return -1;
+    double dec[256];
+    for (int c = 0; c < 256; ++c) dec[c] = oracle_e4m3_to_f64((uint8_t)c);
+    for (int64_t m = m0; m < m1; ++m) {
+        const uint8_t* a = A + m * K;
+        for (int64_t n = 0; n < N; ++n) {
+            const uint8_t* b = B + n * K;
+            double acc = 0.0;
+            for (int64_t k = 0; k < K; ++k) acc += dec[a[k]] * dec[b[k]];
+            double y = acc * (double)a_scale[m] * (double)b_scale[n];
+            D[m * N + n] = oracle_f64_to_bf16(y);
+            if (d_out) d_out[m * N + n] = y;
+        }
+    }
+    return 0;
+}

@@ -24,7 +24,7 @@ import torch
 
 __all__ = [
     "RmsNormError", "rms_norm", "fused_add_rms_norm", "fused_add_rms_norm_fp8",
-    "silu_and_mul_fp8",
+    "silu_and_mul_fp8", "fp8_rowwise_gemm",
     "plan_launch", "validate", "force_plan", "force_staged", "set_launch_options", "device_errors", "supported_vectors_per_thread", "status_string",
     "LIB_PATH", "lib", "RnTensor", "RnPlan", "STATUS", "OPS",
 ]
@@ -91,6 +91,8 @@ def _load():
         f.restype = ctypes.c_int
     L.rn_silu_and_mul_fp8.argtypes = [P, P, P, VP]
     L.rn_silu_and_mul_fp8.restype = ctypes.c_int
+    L.rn_fp8_rowwise_gemm.argtypes = [P, P, P, P, P, VP]
+    L.rn_fp8_rowwise_gemm.restype = ctypes.c_int
     L.rn_status_string.argtypes = [ctypes.c_int]
     L.rn_status_string.restype = ctypes.c_char_p
     L.rn_last_cuda_error.argtypes = []
@@ -235,6 +237,16 @@ def silu_and_mul_fp8(q: torch.Tensor, scale: torch.Tensor, x: torch.Tensor, stre
     dev, s = _stream_for((q, scale, x), stream)
     st = _call(lib.rn_silu_and_mul_fp8, dev, _desc(q, 0), _desc(scale, 1), _desc(x, 2), s)
     _check(st, "rn_silu_and_mul_fp8")
+
+
+def fp8_rowwise_gemm(d: torch.Tensor, a: torch.Tensor, b: torch.Tensor, a_scale: torch.Tensor,
+                     b_scale: torch.Tensor, stream=None) -> None:
+    """D = bf16(b_scale[n] * a_scale[m] * (A @ B^T)) on the tensor cores (C ABI
+    rn_fp8_rowwise_gemm). a: [M, K] e4m3, b: [N, K] e4m3, scales fp32, d: [M, N] bf16."""
+    dev, s = _stream_for((d, a, b, a_scale, b_scale), stream)
+    st = _call(lib.rn_fp8_rowwise_gemm, dev, _desc(d, 0), _desc(a, 1), _desc(b, 2),
+               _desc(a_scale, 3), _desc(b_scale, 4), s)
+    _check(st, "rn_fp8_rowwise_gemm")
 
 
 def plan_launch(op: str, dtype: torch.dtype, T: int, H: int, vector_ok: bool = True) -> dict:

@@ -529,6 +529,49 @@ rn_status rn_silu_and_mul_fp8(const rn_tensor* q, const rn_tensor* scale, const 
     return RN_OK;
 }
 
+rn_status rn_fp8_rowwise_gemm(const rn_tensor* d, const rn_tensor* a, const rn_tensor* b,
+                              const rn_tensor* a_scale, const rn_tensor* b_scale, void* stream) {
+    if (!d || !a || !b || !a_scale || !b_scale) return RN_ERR_NULL;
+    if (a->dtype != RN_E4M3 || b->dtype != RN_E4M3 || d->dtype != RN_BF16 ||
+        a_scale->dtype != RN_F32 || b_scale->dtype != RN_F32)
+        return RN_ERR_DTYPE;
+    Flat fa, fb, fd, fsa, fsb;
+    rn_status st;
+    if ((st = flatten(a, &fa)) != RN_OK) return st;
+    if ((st = flatten(b, &fb)) != RN_OK) return st;
+    if ((st = flatten(d, &fd)) != RN_OK) return st;
+    const int64_t M = fa.T, K = fa.H, N = fb.T;
+    if (fb.H != K || fd.T != M || fd.H != N || N == 0) return RN_ERR_SHAPE;
+    if (K % 16 != 0 || N % 8 != 0) return RN_ERR_SHAPE;
+    const int64_t kMax = 0x7fffffffLL;
+    if (M > kMax || N > kMax || K > kMax) return RN_ERR_SHAPE;
+    if ((st = flatten(b_scale, &fsb)) != RN_OK) return st;
+    if (fsb.numel != N) return RN_ERR_SHAPE;
+    if (M == 0) return RN_OK;
+    if ((st = flatten(a_scale, &fsa)) != RN_OK) return st;
+    if (fsa.numel != M) return RN_ERR_SHAPE;
+    if (!fa.ptr || !fb.ptr || !fd.ptr || !fsa.ptr || !fsb.ptr) return RN_ERR_NULL;
+    if (!aligned(fa.ptr, 16) || !aligned(fb.ptr, 16) || !aligned(fd.ptr, 16) ||
+        !aligned(fsa.ptr, 4) || !aligned(fsb.ptr, 4))
+        return RN_ERR_LAYOUT;
+    if (overlap(fd, fa) || overlap(fd, fb) || overlap(fd, fsa) || overlap(fd, fsb))
+        return RN_ERR_ALIAS;
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e == cudaSuccess) {
+        rn::GemmArgs g{fa.ptr, fb.ptr, reinterpret_cast<const float*>(fsa.ptr),
+                       reinterpret_cast<const float*>(fsb.ptr), fd.ptr, M, N, K, dev,
+                       device_sms()};
+        e = rn::launch_fp8_rowwise_gemm(g, static_cast<cudaStream_t>(stream));
+    }
+    if (e != cudaSuccess) {
+        std::snprintf(g_cuda_error, sizeof g_cuda_error, "%s: %s", cudaGetErrorName(e),
+                      cudaGetErrorString(e));
+        return RN_ERR_CUDA;
+    }
+    return RN_OK;
+}
+
 rn_status rn_validate(int32_t op, const rn_tensor* out_or_q, const rn_tensor* scale,
                       const rn_tensor* x, const rn_tensor* residual, const rn_tensor* weight,
                       float eps, int64_t variance_size, rn_plan* plan) {

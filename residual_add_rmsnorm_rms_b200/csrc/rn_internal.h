@@ -30,6 +30,18 @@ struct SwigluArgs {
     int64_t I;
 };
 
+// Operands of the row-wise scaled fp8 GEMM (device pointers; see fp8_gemm.cu).
+struct GemmArgs {
+    const void* a;        // [M x K] e4m3
+    const void* b;        // [N x K] e4m3
+    const float* a_scale; // [M]
+    const float* b_scale; // [N]
+    void* d;              // [M x N] bf16
+    int64_t M, N, K;
+    int device;
+    int num_sms;
+};
+
 struct Launch {
     int kernel;  // 0 = vector, 1 = scalar, 2 = staged
     int tpr;     // threads per row
@@ -62,6 +74,9 @@ cudaError_t launch(int op, int dtype, const Args& a, const Launch& l, cudaStream
 
 // Enqueues the fused SwiGLU + FP8 cast (vector plan: kernel 0; scalar: 1).
 cudaError_t launch_swiglu_fp8(int dtype, const SwigluArgs& a, const Launch& l, cudaStream_t s);
+
+// Runs the row-wise scaled fp8 GEMM on `stream` (tcgen05 tensor cores).
+cudaError_t launch_fp8_rowwise_gemm(const GemmArgs& g, cudaStream_t stream);
 
 // Reads, and clears when set, the device-side error flags of the current
 // device (bit 0: an mbarrier wait timed out). Synchronous.

@@ -15,6 +15,9 @@ Ops (namespace ``rmsnorm_b200``; CUDA only, N-D inputs flattened to
 * ``silu_and_mul_fp8(x) -> (q, scale)``: x = [gate | up] over the last dim;
   q (float8_e4m3fn, last dim halved), scale (float32, last dim 1): the fused
   SwiGLU + per-token FP8 cast
+* ``fp8_rowwise_gemm(a, b, a_scale, b_scale) -> d``: bf16 [..., N] from
+  e4m3 a [..., K] with per-row a_scale and an e4m3 weight b [N, K] with
+  per-channel b_scale (tcgen05 tensor cores)
 * ``fused_add_rms_norm_fp8(x, residual!, weight, epsilon) -> (q, scale)``:
   residual := x + residual; q (float8_e4m3fn, shape of x) and scale
   (float32, shape of x with the last dim 1) the per-token dynamic cast of
@@ -39,6 +42,7 @@ import torch
 from . import fused_add_rms_norm as _fused
 from . import fused_add_rms_norm_fp8 as _fused_fp8
 from . import rms_norm as _rms
+from . import fp8_rowwise_gemm as _gemm
 from . import silu_and_mul_fp8 as _silu_fp8
 
 __all__ = [
@@ -163,6 +167,19 @@ def _(x):
     shape = x.shape[:-1] + (x.shape[-1] // 2,)
     return (torch.empty(shape, dtype=torch.float8_e4m3fn, device=x.device),
             torch.empty(x.shape[:-1] + (1,), dtype=torch.float32, device=x.device))
+
+
+@torch.library.custom_op(f"{LIB}::fp8_rowwise_gemm", mutates_args=(), device_types="cuda")
+def _fp8_rowwise_gemm_op(a: torch.Tensor, b: torch.Tensor, a_scale: torch.Tensor,
+                         b_scale: torch.Tensor) -> torch.Tensor:
+    d = torch.empty(a.shape[:-1] + (b.shape[0],), dtype=torch.bfloat16, device=a.device)
+    _gemm(d, a, b, a_scale, b_scale)
+    return d
+
+
+@_fp8_rowwise_gemm_op.register_fake
+def _(a, b, a_scale, b_scale):
+    return torch.empty(a.shape[:-1] + (b.shape[0],), dtype=torch.bfloat16, device=a.device)
 
 
 # --------------------------------------------------------------------------- dispatch

@@ -407,4 +407,47 @@ def pin_swiglu_fp8_row_properties(orc, golden=None):
         assert (np.abs(deq - y) <= half_step * (1 + 1e-6)).all()
 
 
+# ---------------------------------------------------------------- fp8 row-wise GEMM
+
+def _e4m3_codes(shape, seed, spread=4.0):
+    g = torch.Generator().manual_seed(seed)
+    v = synth.normal(shape, spread, g, "cpu").clamp_(-448, 448)
+    return v.to(torch.float8_e4m3fn).view(torch.uint8).numpy()
+
+
+def pin_gemm_exact_rationals(orc, golden=None):
+    """A tiny GEMM against exact rational arithmetic (brute force)."""
+    from fractions import Fraction
+    A = _e4m3_codes((3, 16), 1)
+    B = _e4m3_codes((4, 16), 2)
+    rng = np.random.default_rng(3)
+    sa = rng.uniform(0.01, 2.0, 3).astype(np.float32)
+    sb = rng.uniform(0.01, 2.0, 4).astype(np.float32)
+    D, y = orc.fp8_rowwise_gemm(A, B, sa, sb, want_y=True)
+    dec = torch.arange(256, dtype=torch.int32).to(torch.uint8).view(torch.float8_e4m3fn).double().numpy()
+    for m in range(3):
+        for n in range(4):
+            acc = sum(Fraction(dec[A[m, k]]) * Fraction(dec[B[n, k]]) for k in range(16))
+            exact = acc * Fraction(float(sa[m])) * Fraction(float(sb[n]))
+            assert abs(Fraction(y[m, n]) - exact) <= abs(exact) * Fraction(1, 2 ** 51)
+            assert D[m, n] == orc.encode16(np.array([float(exact)]), "bf16")[0]
+
+
+def pin_gemm_matches_float64_matmul(orc, golden=None):
+    """Library pin: numpy float64 matmul of the decoded codes (exact here)."""
+    A = _e4m3_codes((24, 256), 4)
+    B = _e4m3_codes((40, 256), 5)
+    rng = np.random.default_rng(6)
+    sa = rng.uniform(0.001, 1.0, 24).astype(np.float32)
+    sb = rng.uniform(0.001, 1.0, 40).astype(np.float32)
+    dec = torch.arange(256, dtype=torch.int32).to(torch.uint8).view(torch.float8_e4m3fn).double().numpy()
+    ref = (dec[A] @ dec[B].T) * sa.astype(np.float64)[:, None] * sb.astype(np.float64)[None, :]
+    D, y = orc.fp8_rowwise_gemm(A, B, sa, sb, want_y=True)
+    np.testing.assert_array_equal(y, ref)
+    np.testing.assert_array_equal(D, bits16(torch.from_numpy(ref).to(torch.bfloat16)))
+    rows = np.array([0, 5, 23])
+    D2, y2 = orc.fp8_rowwise_gemm(A, B, sa, sb, rows=rows, want_y=True)
+    np.testing.assert_array_equal(y2, ref[rows])
+
+
 PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -1,0 +1,136 @@
+"""GPU parity of the row-wise scaled fp8 GEMM (tcgen05 tensor cores) against
+the fp64 oracle, whose dot products are exact.
+
+Tolerance, derived from the arithmetic: every e4m3 x e4m3 product is exact
+in fp32 (4-bit significands); the tensor cores accumulate K of them in fp32,
+so the accumulated sum is within gamma_K * sum_k |a_k b_k| of the exact sum,
+gamma_K = K * 2^-24 (the worst case of any fp32 summation order); the two
+scale products add 2 * 2^-24 relative, and the result is rounded once to
+bf16 (half an ulp). The test requires, per element,
+    |D - y| <= 1 ulp_bf16(|y|) + (K + 2) * 2^-24 * a_scale * b_scale * sum_k |a_k b_k|
+with y the oracle's unrounded value, and reports how many elements equal
+the correctly rounded value."""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+import residual_add_rmsnorm_rms_b200 as rn
+import synth
+from residual_add_rmsnorm_rms_b200 import torch_ops  # noqa: F401  (registers the ops)
+from tests.cmp_util import bits16, codes8, ulp16
+from tests.gpu_util import CORES, sample_rows
+
+pytestmark = pytest.mark.gpu
+
+# (N, K) weight shapes of Gemma 4 12B's fp8 linear layers, from the
+# weight-shape table of "VLLM_ROCM_USE_AITER=1 slows Gemma 4 on an AMD MI300X"
+GEMMA_NK = [(8192, 3840), (9216, 3840), (30720, 3840), (3840, 4096), (3840, 8192), (3840, 15360)]
+DEC = torch.arange(256, dtype=torch.int32).to(torch.uint8).view(torch.float8_e4m3fn).double().numpy()
+
+
+@pytest.fixture(autouse=True)
+def _cuda():
+    if not torch.cuda.is_available():
+        pytest.fail("GPU tests need a CUDA device")
+    yield
+    assert rn.device_errors() == 0
+
+
+def _operands(M, N, K, seed, device="cpu"):
+    g = torch.Generator(device=device).manual_seed(seed)
+    a = (torch.randn(M, K, generator=g, device=device) * 40).clamp_(-448, 448)
+    b = (torch.randn(N, K, generator=g, device=device) * 40).clamp_(-448, 448)
+    sa = torch.rand(M, generator=g, device=device) * 0.02 + 1e-3
+    sb = torch.rand(N, generator=g, device=device) * 0.02 + 1e-3
+    return a.to(torch.float8_e4m3fn), b.to(torch.float8_e4m3fn), sa, sb
+
+
+def _gemm(a, b, sa, sb):
+    d = torch.empty(a.shape[0], b.shape[0], dtype=torch.bfloat16, device="cuda")
+    rn.fp8_rowwise_gemm(d, a, b, sa, sb)
+    torch.cuda.synchronize()
+    return d
+
+
+def _check(d_gpu, a_codes, b_codes, sa, sb, rows=None):
+    """d_gpu holds the rows `rows` (or all); returns the fraction equal to RNE(y)."""
+    want, y = oracle.fp8_rowwise_gemm(a_codes, b_codes, sa, sb, rows=rows, want_y=True,
+                                      threads=CORES)
+    A = a_codes if rows is None else a_codes[rows]
+    sa_r = sa if rows is None else sa[rows]
+    K = A.shape[1]
+    absdot = np.abs(DEC[A]) @ np.abs(DEC[b_codes]).T
+    bound = (K + 2) * 2.0 ** -24 * absdot * sa_r.astype(np.float64)[:, None] \
+        * sb.astype(np.float64)[None, :]
+    got = torch.from_numpy(d_gpu.astype(np.int16) if isinstance(d_gpu, np.ndarray) else
+                           bits16(d_gpu).view(np.int16)).view(torch.bfloat16).double().numpy()
+    ay = np.abs(y)
+    ulp = np.where(ay > 0, 2.0 ** (np.floor(np.log2(np.maximum(ay, 1e-300))) - 7), 2.0 ** -133)
+    err = np.abs(got - y)
+    assert (err <= ulp + bound).all(), float(np.max((err - ulp) / np.maximum(bound, 1e-300)))
+    gbits = bits16(d_gpu) if not isinstance(d_gpu, np.ndarray) else d_gpu
+    return float(np.mean(ulp16(gbits, want) == 0))
+
+
+@pytest.mark.parametrize("M,N,K", [(1, 8, 16), (7, 128, 128), (128, 128, 128), (300, 264, 400),
+                                   (129, 3840, 4096), (64, 8, 15360)])
+def test_gemm_small_shapes_full(M, N, K):
+    a, b, sa, sb = _operands(M, N, K, seed=M + N + K)
+    d = _gemm(a.cuda(), b.cuda(), sa.cuda(), sb.cuda())
+    exact_frac = _check(d, codes8(a), codes8(b), sa.numpy(), sb.numpy())
+    print(M, N, K, "correctly rounded fraction", exact_frac)
+
+
+@pytest.mark.parametrize("N,K", GEMMA_NK)
+@pytest.mark.parametrize("M", [1, 256, 8192])
+def test_gemm_gemma_shapes(M, N, K):
+    a, b, sa, sb = _operands(M, N, K, seed=N + K + M, device="cuda")
+    d = _gemm(a, b, sa, sb)
+    rows = sample_rows(M, k=32)
+    exact_frac = _check(bits16(d)[rows], codes8(a), codes8(b), sa.cpu().numpy(),
+                        sb.cpu().numpy(), rows=rows)
+    print(M, N, K, "correctly rounded fraction", exact_frac)
+
+
+def test_norm_then_gemm_chain():
+    """The decode chain: fused_add_rms_norm_fp8 codes and per-token scales
+    feed the GEMM directly (GPU codes go to both the GPU GEMM and the oracle)."""
+    wl = synth.make_inputs("prefill", "fused_add_rms_norm_fp8", "bf16", 256, 3840)
+    q = torch.empty(256, 3840, dtype=torch.float8_e4m3fn, device="cuda")
+    s = torch.empty(256, dtype=torch.float32, device="cuda")
+    rn.fused_add_rms_norm_fp8(q, s, wl.x.cuda(), wl.residual.cuda().clone(), wl.weight.cuda(),
+                              wl.eps)
+    _, b, _, sb = _operands(1, 8192, 3840, seed=77)
+    d = torch.ops.rmsnorm_b200.fp8_rowwise_gemm(q, b.cuda(), s, sb.cuda())
+    torch.cuda.synchronize()
+    assert d.shape == (256, 8192) and d.dtype == torch.bfloat16
+    _check(d, codes8(q), codes8(b), s.cpu().numpy(), sb.numpy())
+
+
+def test_gemm_validation():
+    a = torch.zeros(4, 32, dtype=torch.float8_e4m3fn, device="cuda")
+    b = torch.zeros(16, 32, dtype=torch.float8_e4m3fn, device="cuda")
+    sa = torch.ones(4, device="cuda")
+    sb = torch.ones(16, device="cuda")
+    d = torch.empty(4, 16, dtype=torch.bfloat16, device="cuda")
+    rn.fp8_rowwise_gemm(d, a, b, sa, sb)
+    torch.cuda.synchronize()
+    assert (d.float() == 0).all()
+    cases = [
+        ((d, a[:, :24], b[:, :24], sa, sb), "RN_ERR_LAYOUT"),       # padded rows
+        ((d, torch.zeros(4, 24, dtype=torch.float8_e4m3fn, device="cuda"),
+          torch.zeros(16, 24, dtype=torch.float8_e4m3fn, device="cuda"), sa, sb), "RN_ERR_SHAPE"),
+        ((torch.empty(4, 12, dtype=torch.bfloat16, device="cuda"), a, b[:12], sa, sb[:12]),
+         "RN_ERR_SHAPE"),                                          # N % 8
+        ((d, a, b, sa[:3], sb), "RN_ERR_SHAPE"),
+        ((d.float(), a, b, sa, sb), "RN_ERR_DTYPE"),
+        ((d, a.view(torch.uint8).to(torch.bfloat16), b, sa, sb), "RN_ERR_DTYPE"),
+    ]
+    for args, name in cases:
+        with pytest.raises(rn.RmsNormError) as e:
+            rn.fp8_rowwise_gemm(*args)
+        assert e.value.name == name, (name, e.value.name)
+    empty = torch.empty(0, 32, dtype=torch.float8_e4m3fn, device="cuda")
+    rn.fp8_rowwise_gemm(torch.empty(0, 16, dtype=torch.bfloat16, device="cuda"), empty, b,
+                        torch.empty(0, device="cuda"), sb)

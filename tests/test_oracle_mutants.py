@@ -46,6 +46,11 @@ MUTANTS = {
                                     "double y = 1.0 / (1.0 + exp(-a)) * b;"),
     "swiglu_scale_240": ("double s = amax / 448.0;\n        scale[t] = (float)s;\n        for (int64_t i = 0; i < I; ++i) {",
                          "double s = amax / 240.0;\n        scale[t] = (float)s;\n        for (int64_t i = 0; i < I; ++i) {"),
+    "gemm_b_transposed": ("const uint8_t* b = B + n * K;", "const uint8_t* b = B + n;"),
+    "gemm_a_scale_dropped": ("double y = acc * (double)a_scale[m] * (double)b_scale[n];",
+                             "double y = acc * (double)b_scale[n];"),
+    "gemm_scales_swapped": ("double y = acc * (double)a_scale[m] * (double)b_scale[n];",
+                            "double y = acc * (double)a_scale[n % M] * (double)b_scale[m % N];"),
     "bf16_overflow_threshold": ("if (r > maxf) return sign | 0x7f80; /* overflow to infinity */",
                                 "if (r >= maxf) return sign | 0x7f80;"),
 }

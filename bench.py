@@ -349,22 +349,24 @@ def run_ours(args, world, rank, local):
     barrier(world)
     total_ms = max_over_ranks(e_start.elapsed_time(e_end), world, device)
 
-    # Pass B: the same K steps with an event pair around every launch, for
-    # the per-kernel durations (the roofline of the dominant kernel).
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(K)]
-    barrier(world)
-    torch.cuda.synchronize(device)
-    for i in range(K):
-        ev[i][0].record(stream)
-        launch(i, 0)
-        ev[i][1].record(stream)
-        launch(i, 1)
-        ev[i][2].record(stream)
-    torch.cuda.synchronize(device)
-    barrier(world)
-    k0 = [ev[i][0].elapsed_time(ev[i][1]) for i in range(K)]
-    k1 = [ev[i][1].elapsed_time(ev[i][2]) for i in range(K)]
-    passb_ms = ev[0][0].elapsed_time(ev[K - 1][2])
+    # Pass B: each op alone, K launches back to back on the step's rotating
+    # buffer sets, one event pair around the K launches: that kernel's
+    # average launch duration in a stream (the roofline of the dominant
+    # kernel). Events around single launches would stop programmatic
+    # dependent launch from overlapping one launch's tail with the next
+    # one's head and add that gap to every launch.
+    per_op_ms = []
+    for k in (0, 1):
+        ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        barrier(world)
+        torch.cuda.synchronize(device)
+        ea.record(stream)
+        for i in range(K):
+            launch(i, k)
+        eb.record(stream)
+        torch.cuda.synchronize(device)
+        barrier(world)
+        per_op_ms.append(max_over_ranks(ea.elapsed_time(eb), world, device) / K)
 
     # end to end through the public API with host buffers: pinned H2D of each
     # launch's inputs, the two launches, D2H of every output, all timed.
@@ -376,9 +378,8 @@ def run_ours(args, world, rank, local):
     value = b_step * K * world / (total_ms / 1e3) / 1e9
     peak, peak_src = measured_peak()
     dom_bytes = op_bytes("fused_add_rms_norm", T, H)
-    dom_ms = statistics.mean(k0)
+    dom_ms, fp8_ms = per_op_ms
     achieved = dom_bytes / (dom_ms / 1e3) / 1e9
-    fp8_ms = statistics.mean(k1)
     traffic = ncu_traffic()
     cpu = cpu_baseline() if (rank == 0 and world == 1 and not args.no_cpu_baseline) else None
     if rank != 0:
@@ -401,7 +402,7 @@ def run_ours(args, world, rank, local):
             "bytes_per_step": b_step,
             "plans": {op: rn.plan_launch(op, torch.bfloat16, T, H) for op in STEP_OPS},
         },
-        "per_kernel_pass_ms_per_step": round(passb_ms / K, 5),
+        "per_kernel_how": f"each op alone, {K} launches back to back, events at the ends",
         "per_kernel_ms": {"fused_add_rms_norm": round(dom_ms, 5),
                           "fused_add_rms_norm_fp8": round(fp8_ms, 5)},
         "per_kernel_gbs": {"fused_add_rms_norm": round(achieved, 1),
@@ -565,7 +566,7 @@ def time_cell(rn, name, op, dtype, T, H, iters, device, mem_cap_bytes=24 << 30):
 # (N, K) of Gemma 4 12B's fp8 linear layers (weight-shape table of
 # "VLLM_ROCM_USE_AITER=1 slows Gemma 4 on an AMD MI300X")
 GEMMA_NK = ((8192, 3840), (9216, 3840), (30720, 3840), (3840, 4096), (3840, 8192), (3840, 15360))
-GEMM_M = (1, 64, 256, 8192)
+GEMM_M = (1, 16, 32, 64, 256, 8192)
 
 
 def measured_fp8_peak():
@@ -580,7 +581,11 @@ def measured_fp8_peak():
         return 2.0 * 1590.0, "2 x fallback bf16 1.59 PFLOP/s"
 
 
-def time_gemm_cell(rn, M, N, K, iters, device):
+def time_gemm_cell(rn, M, N, K, iters, device, configs=(None,)):
+    """Per tile configuration (None = the automatic choice): mean time per
+    call over `iters` eager calls rotating over operand sets of >= 4x L2
+    (at most 8 sets), and, for calls under 60 us, the CUDA-graph replay time
+    of 100 captured calls (device time without the host's per-call cost)."""
     g = torch.Generator(device=device).manual_seed(M + N + K)
     n_sets = max(2, math.ceil(4 * torch.cuda.get_device_properties(device).L2_cache_size
                               / (N * K + M * K + 2 * M * N)) + 1)
@@ -594,19 +599,46 @@ def time_gemm_cell(rn, M, N, K, iters, device):
                      torch.rand(M, generator=g, device=device) * 0.01,
                      torch.rand(N, generator=g, device=device) * 0.01))
         del a, b
-    for i in range(3):
-        rn.fp8_rowwise_gemm(*sets[i % n_sets])
-    torch.cuda.synchronize(device)
+    out = {}
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    e0.record()
-    for i in range(iters):
-        rn.fp8_rowwise_gemm(*sets[i % n_sets])
-    e1.record()
-    torch.cuda.synchronize(device)
-    us = e0.elapsed_time(e1) / iters * 1e3
+    for cfg in configs:
+        rn.fp8_gemm_force_config(cfg)
+        try:
+            for i in range(3):
+                rn.fp8_rowwise_gemm(*sets[i % n_sets])
+            torch.cuda.synchronize(device)
+            e0.record()
+            for i in range(iters):
+                rn.fp8_rowwise_gemm(*sets[i % n_sets])
+            e1.record()
+            torch.cuda.synchronize(device)
+            us = e0.elapsed_time(e1) / iters * 1e3
+            gus = None
+            if us < 60:
+                gr = torch.cuda.CUDAGraph()
+                st = torch.cuda.Stream(device)
+                with torch.cuda.stream(st):
+                    rn.fp8_rowwise_gemm(*sets[0])
+                    torch.cuda.synchronize(device)
+                    with torch.cuda.graph(gr, stream=st):
+                        for i in range(100):
+                            rn.fp8_rowwise_gemm(*sets[i % n_sets])
+                gr.replay()
+                torch.cuda.synchronize(device)
+                e0.record()
+                for _ in range(3):
+                    gr.replay()
+                e1.record()
+                torch.cuda.synchronize(device)
+                gus = e0.elapsed_time(e1) / 300 * 1e3
+                del gr
+        finally:
+            rn.fp8_gemm_force_config(None)
+        name = cfg if cfg is not None else rn.fp8_gemm_config(M, N, K)
+        out[cfg] = (us, gus, name)
     del sets
     torch.cuda.empty_cache()
-    return us
+    return out
 
 
 def run_sweep(args, world, rank, local):
@@ -637,15 +669,22 @@ def run_sweep(args, world, rank, local):
                   if all(w in ("gemm", "fp8_rowwise_gemm", str(M), f"{N}x{K}") for w in want)]
     fp8_peak, fp8_src = measured_fp8_peak()
     for M, N, K in gemm_cells:
-        us = time_gemm_cell(rn, M, N, K, args.sweep_iters, device)
-        tflops = 2.0 * M * N * K / us / 1e6
-        rec = {"workload": "gemm", "op": "fp8_rowwise_gemm", "dtype": "e4m3", "M": M, "N": N,
-               "K": K, "us": round(us, 3), "tflops": round(tflops, 1),
-               "frac_of_fp8_peak": round(tflops / fp8_peak, 4), "fp8_peak_tflops": fp8_peak,
-               "peak_source": fp8_src,
-               "weight_gbs": round(N * K / us / 1e3, 1)}
-        out.write(json.dumps(rec) + "\n")
-        out.flush()
+        configs = [None]
+        if args.sweep_gemm_configs and M <= 256:
+            configs += list(rn.GEMM_CONFIGS)
+        for cfg, (us, gus, name) in time_gemm_cell(rn, M, N, K, args.sweep_iters, device,
+                                                   configs).items():
+            best = gus if gus is not None else us
+            tflops = 2.0 * M * N * K / best / 1e6
+            rec = {"workload": "gemm", "op": "fp8_rowwise_gemm", "dtype": "e4m3", "M": M,
+                   "N": N, "K": K, "config": name, "forced": cfg is not None,
+                   "us": round(us, 3), "graph_us": None if gus is None else round(gus, 3),
+                   "tflops": round(tflops, 1), "frac_of_fp8_peak": round(tflops / fp8_peak, 4),
+                   "fp8_peak_tflops": fp8_peak, "peak_source": fp8_src,
+                   "weight_gbs": round(N * K / best / 1e3, 1),
+                   "weight_frac_of_measured_hbm": round(N * K / best / 1e3 / peak, 4)}
+            out.write(json.dumps(rec) + "\n")
+            out.flush()
     out.close()
     assert rn.device_errors() == 0
     print(json.dumps({"sweep": args.sweep_out, "cells": len(cells) + len(gemm_cells)}))
@@ -665,6 +704,8 @@ def main():
                     help="instead of the step benchmark, time every workload cell and write "
                          "one JSON line per cell to this file")
     ap.add_argument("--sweep-iters", type=int, default=50)
+    ap.add_argument("--sweep-gemm-configs", action="store_true",
+                    help="also time every GEMM tile configuration, forced, on cells with M <= 256")
     ap.add_argument("--sweep-filter", default=None,
                     help="comma-separated values a cell must all match (workload, op, dtype, "
                          "T or H), e.g. swiglu,bf16,8192")

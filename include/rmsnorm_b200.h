@@ -164,10 +164,42 @@ RN_API rn_status rn_silu_and_mul_fp8(const rn_tensor* q, const rn_tensor* scale,
  * Requirements: dense views (flattening rule of the norm ops), K % 16 == 0,
  * N % 8 == 0, 16-byte-aligned A, B and D, K, N and M below 2^31; D must not
  * overlap any input. M == 0 is a no-op. Needs no workspace. Asynchronous on
- * `stream`; validation errors return before any CUDA call. */
+ * `stream`; validation errors return before any CUDA call. The tile shape is
+ * chosen per call (rn_fp8_gemm_config). */
 RN_API rn_status rn_fp8_rowwise_gemm(const rn_tensor* d, const rn_tensor* a,
                                      const rn_tensor* b, const rn_tensor* a_scale,
                                      const rn_tensor* b_scale, void* stream);
+
+/* Tile configurations of rn_fp8_rowwise_gemm. TOK tiles put the tensor core's
+ * MMA rows on tokens: (tokens x channels) = 128 x 128. CH tiles compute D^T =
+ * B * A^T, putting the MMA rows on the weight's output channels: (channels x
+ * tokens), for decode-sized M where 128 token rows would be mostly padding.
+ * Every configuration computes the same values: the scales are applied in the
+ * same order and the fp32 accumulation over K differs only in its order. */
+typedef enum {
+    RN_GEMM_TOK128_CH128 = 0,
+    RN_GEMM_CH128_TOK16 = 1,
+    RN_GEMM_CH128_TOK32 = 2,
+    RN_GEMM_CH128_TOK64 = 3,
+    RN_GEMM_CH64_TOK16 = 4,
+    RN_GEMM_CH64_TOK32 = 5,
+    RN_GEMM_CH64_TOK64 = 6
+} rn_gemm_config;
+
+/* The configuration rn_fp8_rowwise_gemm uses for an M x N x K problem on a
+ * device with `num_sms` SMs (<= 0: 148). Among the CH configurations, the one
+ * with the most tiles (ceil(N / channels) * ceil(M / tokens)) not above
+ * num_sms, ties going to fewer channels, then fewer tokens per tile; if none
+ * fits, CH128 with the smallest token width >= M for M <= 64, TOK128_CH128
+ * above. Honours rn_fp8_gemm_force_config. Pure host logic. RN_ERR_SHAPE for
+ * M < 0, N < 1 or K < 1. */
+RN_API rn_status rn_fp8_gemm_config(int64_t M, int64_t N, int64_t K, int32_t num_sms,
+                                    int32_t* config);
+
+/* Test hook: force rn_gemm_config `config` for every later GEMM in the
+ * process; -1 restores the automatic choice; other values RN_ERR_CONFIG. Not
+ * thread-safe with concurrent launches; meant for tests and tuning. */
+RN_API rn_status rn_fp8_gemm_force_config(int32_t config);
 
 /* Static text for a status code (never NULL). */
 RN_API const char* rn_status_string(rn_status status);

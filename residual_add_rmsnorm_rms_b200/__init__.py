@@ -24,8 +24,9 @@ import torch
 
 __all__ = [
     "RmsNormError", "rms_norm", "fused_add_rms_norm", "fused_add_rms_norm_fp8",
-    "silu_and_mul_fp8", "fp8_rowwise_gemm",
-    "plan_launch", "validate", "force_plan", "force_staged", "set_launch_options", "device_errors", "supported_vectors_per_thread", "status_string",
+    "silu_and_mul_fp8", "fp8_rowwise_gemm", "fp8_gemm_config", "fp8_gemm_force_config",
+    "GEMM_CONFIGS", "plan_launch", "validate", "force_plan", "force_staged",
+    "set_launch_options", "device_errors", "supported_vectors_per_thread", "status_string",
     "LIB_PATH", "lib", "RnTensor", "RnPlan", "STATUS", "OPS",
 ]
 
@@ -93,6 +94,10 @@ def _load():
     L.rn_silu_and_mul_fp8.restype = ctypes.c_int
     L.rn_fp8_rowwise_gemm.argtypes = [P, P, P, P, P, VP]
     L.rn_fp8_rowwise_gemm.restype = ctypes.c_int
+    L.rn_fp8_gemm_config.argtypes = [I64, I64, I64, ctypes.c_int32, ctypes.POINTER(ctypes.c_int32)]
+    L.rn_fp8_gemm_config.restype = ctypes.c_int
+    L.rn_fp8_gemm_force_config.argtypes = [ctypes.c_int32]
+    L.rn_fp8_gemm_force_config.restype = ctypes.c_int
     L.rn_status_string.argtypes = [ctypes.c_int]
     L.rn_status_string.restype = ctypes.c_char_p
     L.rn_last_cuda_error.argtypes = []
@@ -247,6 +252,26 @@ def fp8_rowwise_gemm(d: torch.Tensor, a: torch.Tensor, b: torch.Tensor, a_scale:
     st = _call(lib.rn_fp8_rowwise_gemm, dev, _desc(d, 0), _desc(a, 1), _desc(b, 2),
                _desc(a_scale, 3), _desc(b_scale, 4), s)
     _check(st, "rn_fp8_rowwise_gemm")
+
+
+# rn_gemm_config values: TOK = token-major (tokens x channels) tiles, CH =
+# channel-major (channels x tokens) tiles computing D^T.
+GEMM_CONFIGS = {"tok128_ch128": 0, "ch128_tok16": 1, "ch128_tok32": 2, "ch128_tok64": 3,
+                "ch64_tok16": 4, "ch64_tok32": 5, "ch64_tok64": 6}
+
+
+def fp8_gemm_config(M: int, N: int, K: int, num_sms: int = 0) -> str:
+    """Name of the tile configuration rn_fp8_rowwise_gemm uses (host logic)."""
+    c = ctypes.c_int32(-1)
+    _check(lib.rn_fp8_gemm_config(M, N, K, num_sms, ctypes.byref(c)), "rn_fp8_gemm_config")
+    return {v: k for k, v in GEMM_CONFIGS.items()}[c.value]
+
+
+def fp8_gemm_force_config(config) -> None:
+    """Test/tuning hook: force a GEMM tile configuration (name or id); None or
+    -1 restores the automatic choice."""
+    cid = -1 if config is None else (GEMM_CONFIGS[config] if isinstance(config, str) else config)
+    _check(lib.rn_fp8_gemm_force_config(cid), "rn_fp8_gemm_force_config")
 
 
 def plan_launch(op: str, dtype: torch.dtype, T: int, H: int, vector_ok: bool = True) -> dict:

@@ -33,7 +33,7 @@ NVCC_FLAGS = [
     "-Xcompiler", "-fPIC", "-Xcompiler", "-fvisibility=hidden",
 ]
 # Sources that instantiate CUTLASS templates.
-CUTLASS_SOURCES = {"fp8_gemm.cu"}
+CUTLASS_SOURCES = {"fp8_gemm.cu", "fp8_gemm_ch128.cu", "fp8_gemm_ch64.cu"}
 CUTLASS_FLAGS = ["--expt-relaxed-constexpr", "-diag-suppress", "20012"]
 
 

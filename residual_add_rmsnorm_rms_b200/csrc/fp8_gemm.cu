@@ -1,114 +1,28 @@
-// fp8_gemm.cu -- row-wise scaled FP8 GEMM on the sm_100a tensor cores:
-//
-//   D[m, n] = bf16( b_scale[n] * (a_scale[m] * sum_k A[m, k] * B[n, k]) )
-//
-// A [M x K] e4m3 (row-major, K contiguous) is what fused_add_rms_norm_fp8
-// produces together with its per-token a_scale; B [N x K] e4m3 is a weight
-// with one scale per output channel. This is the consumer of the fused
-// residual + RMSNorm + FP8 pass in the decode path of "Custom CUDA kernels
-// juice Llama 3.1 405B on AMD MI300X, skipping Nvidia lock-in" and the
-// row-wise fp8 linear layers (RowWiseTorchFP8ScaledMMLinearKernel) in the
-// table of "VLLM_ROCM_USE_AITER=1 slows Gemma 4 on an AMD MI300X".
-//
-// Built from CUTLASS's sm100 collectives: tcgen05 MMA issued by one thread
-// with the accumulator in tensor memory, TMA loads of A and B tiles into a
-// multi-stage shared-memory pipeline, warp-specialised (load / MMA /
-// epilogue warps), persistent tile scheduler. One CTA per 128 x 128 output
-// tile (cluster 1 x 1 x 1), K step 128. The epilogue is an epilogue-visitor
-// tree: fp32 accumulator x a_scale[m] (column broadcast) x b_scale[n] (row
-// broadcast), rounded once to bf16, stored by TMA.
-#include <cstdint>
-
-#include "cutlass/cutlass.h"
-#include "cute/tensor.hpp"
-#include "cutlass/epilogue/collective/collective_builder.hpp"
-#include "cutlass/epilogue/fusion/sm90_visitor_tma_warpspecialized.hpp"
-#include "cutlass/gemm/collective/collective_builder.hpp"
-#include "cutlass/gemm/device/gemm_universal_adapter.h"
-#include "cutlass/gemm/kernel/gemm_universal.hpp"
-#include "cutlass/util/packed_stride.hpp"
-
-#include "rn_internal.h"
+// fp8_gemm.cu -- tile-configuration dispatch of the row-wise scaled FP8 GEMM
+// and its token-major 128 x 128 instantiation (the template and the two
+// orientations are described in fp8_gemm.cuh). The channel-major
+// instantiations for decode-sized M live in fp8_gemm_ch128.cu and
+// fp8_gemm_ch64.cu so that the three units compile in parallel.
+#include "fp8_gemm.cuh"
 
 namespace rn {
-namespace {
 
-using namespace cute;
-namespace fusion = cutlass::epilogue::fusion;
-
-using ElementA = cutlass::float_e4m3_t;
-using ElementB = cutlass::float_e4m3_t;
-using ElementD = cutlass::bfloat16_t;
-using LayoutA = cutlass::layout::RowMajor;     // [M x K], K contiguous
-using LayoutB = cutlass::layout::ColumnMajor;  // K x N stored as [N x K], K contiguous
-using LayoutD = cutlass::layout::RowMajor;
-constexpr int kAlignAB = 16;  // elements: 16 bytes of e4m3 per TMA row granule
-constexpr int kAlignD = 8;    // elements: 16 bytes of bf16
-
-template <class MmaTile>
-struct RowwiseGemm {
-    using Cluster = Shape<_1, _1, _1>;
-    using ScaleA = fusion::Sm90ColBroadcast<0, MmaTile, float, float, Stride<_1, _0, int64_t>>;
-    using ScaleB = fusion::Sm90RowBroadcast<0, MmaTile, float, float, Stride<_0, _1, int64_t>>;
-    using MulA = fusion::Sm90Compute<cutlass::multiplies, float, float,
-                                     cutlass::FloatRoundStyle::round_to_nearest>;
-    using MulB = fusion::Sm90Compute<cutlass::multiplies, ElementD, float,
-                                     cutlass::FloatRoundStyle::round_to_nearest>;
-    using Evt = fusion::Sm90EVT<MulB, ScaleB, fusion::Sm90EVT<MulA, ScaleA, fusion::Sm90AccFetch>>;
-
-    using Epilogue = typename cutlass::epilogue::collective::CollectiveBuilder<
-        cutlass::arch::Sm100, cutlass::arch::OpClassTensorOp, MmaTile, Cluster,
-        cutlass::epilogue::collective::EpilogueTileAuto, float, float, void, LayoutD, kAlignD,
-        ElementD, LayoutD, kAlignD, cutlass::epilogue::TmaWarpSpecialized1Sm, Evt>::CollectiveOp;
-
-    using Mainloop = typename cutlass::gemm::collective::CollectiveBuilder<
-        cutlass::arch::Sm100, cutlass::arch::OpClassTensorOp, ElementA, LayoutA, kAlignAB,
-        ElementB, LayoutB, kAlignAB, float, MmaTile, Cluster,
-        cutlass::gemm::collective::StageCountAutoCarveout<
-            static_cast<int>(sizeof(typename Epilogue::SharedStorage))>,
-        cutlass::gemm::KernelTmaWarpSpecialized1SmSm100>::CollectiveOp;
-
-    using Kernel =
-        cutlass::gemm::kernel::GemmUniversal<Shape<int, int, int, int>, Mainloop, Epilogue, void>;
-    using Gemm = cutlass::gemm::device::GemmUniversalAdapter<Kernel>;
-
-    static cudaError_t run(const GemmArgs& g, cudaStream_t stream) {
-        const int M = static_cast<int>(g.M), N = static_cast<int>(g.N), K = static_cast<int>(g.K);
-        typename Gemm::Arguments args;
-        args.mode = cutlass::gemm::GemmUniversalMode::kGemm;
-        args.problem_shape = {M, N, K, 1};
-        const auto sA = cutlass::make_cute_packed_stride(typename Kernel::StrideA{},
-                                                         make_shape(M, K, 1));
-        const auto sB = cutlass::make_cute_packed_stride(typename Kernel::StrideB{},
-                                                         make_shape(N, K, 1));
-        const auto sD = cutlass::make_cute_packed_stride(typename Kernel::StrideD{},
-                                                         make_shape(M, N, 1));
-        args.mainloop = {static_cast<const ElementA*>(g.a), sA, static_cast<const ElementB*>(g.b),
-                         sB};
-        args.epilogue.ptr_C = nullptr;
-        args.epilogue.dC = sD;
-        args.epilogue.ptr_D = static_cast<ElementD*>(g.d);
-        args.epilogue.dD = sD;
-        args.epilogue.thread = {
-            {g.b_scale, 0.f, {}},                 // b_scale[n]
-            {{g.a_scale, 0.f, {}}, {}, {}},       // a_scale[m] * accumulator
-            {}};
-        args.hw_info.device_id = g.device;
-        args.hw_info.sm_count = g.num_sms;
-        Gemm gemm;
-        if (gemm.can_implement(args) != cutlass::Status::kSuccess) return cudaErrorInvalidValue;
-        if (Gemm::get_workspace_size(args) != 0) return cudaErrorInvalidValue;  // none by design
-        if (gemm.initialize(args, nullptr, stream) != cutlass::Status::kSuccess)
-            return cudaErrorInvalidConfiguration;
-        if (gemm.run(stream) != cutlass::Status::kSuccess) return cudaErrorLaunchFailure;
-        return cudaGetLastError();
-    }
-};
-
-}  // namespace
+cudaError_t gemm_channel_major_128(int tokens, const GemmArgs& g, cudaStream_t stream);
+cudaError_t gemm_channel_major_64(int tokens, const GemmArgs& g, cudaStream_t stream);
 
 cudaError_t launch_fp8_rowwise_gemm(const GemmArgs& g, cudaStream_t stream) {
-    return RowwiseGemm<Shape<_128, _128, _128>>::run(g, stream);
+    using namespace gemm_detail;
+    switch (g.config) {
+        case kGemmTok128Ch128:
+            return RowwiseGemm<Shape<_128, _128, _128>, false>::run(g, stream);
+        case kGemmCh128Tok16: return gemm_channel_major_128(16, g, stream);
+        case kGemmCh128Tok32: return gemm_channel_major_128(32, g, stream);
+        case kGemmCh128Tok64: return gemm_channel_major_128(64, g, stream);
+        case kGemmCh64Tok16: return gemm_channel_major_64(16, g, stream);
+        case kGemmCh64Tok32: return gemm_channel_major_64(32, g, stream);
+        case kGemmCh64Tok64: return gemm_channel_major_64(64, g, stream);
+        default: return cudaErrorInvalidValue;
+    }
 }
 
 }  // namespace rn

@@ -28,6 +28,7 @@ std::atomic<int> g_force_staged_s{0};
 std::atomic<int> g_force_staged_t{0};
 std::atomic<int> g_pdl{-1};              // -1 default, 0 off, 1 on
 std::atomic<long long> g_max_grid{0};    // 0: no cap
+std::atomic<int> g_force_gemm{-1};       // fp8 GEMM tile configuration; -1: automatic
 // Launch defaults, measured on B200 (prefill [8192 x 3840], two ops
 // alternating in one stream): programmatic dependent launch lets the next
 // kernel's blocks start as this one drains (+4-5 %), and capping the vector
@@ -300,6 +301,42 @@ int device_sms() {
     return n;
 }
 
+// Tile configuration of the fp8 GEMM for an [M x K] x [N x K]^T problem.
+// A decode-sized GEMM is bound by streaming the weight, and a CTA streams
+// only its own tiles, so the choice maximises the tiles in flight: among the
+// channel-major shapes (channels x tokens: 64 or 128 x 16, 32 or 64), the one
+// with the most tiles that still fit in one wave (ties: fewer channels, then
+// fewer tokens per tile). When none fits, up to 64 tokens take the 128-channel
+// tile of the smallest token width >= M (fewest tiles), larger M the
+// token-major 128 x 128 tile. Measured on B200 over the Gemma 4 12B weight
+// shapes, this picks the fastest configuration or one within 5 % of it.
+int gemm_auto_config(int64_t M, int64_t N, int num_sms) {
+    struct Shape { int config, ch, tok; };
+    static constexpr Shape kChannelMajor[] = {
+        {rn::kGemmCh64Tok16, 64, 16},   {rn::kGemmCh64Tok32, 64, 32},
+        {rn::kGemmCh64Tok64, 64, 64},   {rn::kGemmCh128Tok16, 128, 16},
+        {rn::kGemmCh128Tok32, 128, 32}, {rn::kGemmCh128Tok64, 128, 64}};
+    int best = -1;
+    int64_t best_tiles = 0;
+    for (const Shape& c : kChannelMajor) {
+        const int64_t tiles = ((N + c.ch - 1) / c.ch) * ((M + c.tok - 1) / c.tok);
+        if (tiles <= num_sms && tiles > best_tiles) {
+            best = c.config;
+            best_tiles = tiles;
+        }
+    }
+    if (best >= 0) return best;
+    if (M <= 16) return rn::kGemmCh128Tok16;
+    if (M <= 32) return rn::kGemmCh128Tok32;
+    if (M <= 64) return rn::kGemmCh128Tok64;
+    return rn::kGemmTok128Ch128;
+}
+
+int gemm_config(int64_t M, int64_t N, int num_sms) {
+    const int f = g_force_gemm.load();
+    return f >= 0 ? f : gemm_auto_config(M, N, num_sms);
+}
+
 struct Common {
     Flat x, out, res, q, scale, w;
     bool has_w = false;
@@ -561,7 +598,8 @@ rn_status rn_fp8_rowwise_gemm(const rn_tensor* d, const rn_tensor* a, const rn_t
     if (e == cudaSuccess) {
         rn::GemmArgs g{fa.ptr, fb.ptr, reinterpret_cast<const float*>(fsa.ptr),
                        reinterpret_cast<const float*>(fsb.ptr), fd.ptr, M, N, K, dev,
-                       device_sms()};
+                       device_sms(), 0};
+        g.config = gemm_config(M, N, g.num_sms);
         e = rn::launch_fp8_rowwise_gemm(g, static_cast<cudaStream_t>(stream));
     }
     if (e != cudaSuccess) {
@@ -671,6 +709,20 @@ int32_t rn_supported_vectors_per_thread(int32_t* out, int32_t cap) {
     return rn::kNumVpt;
 }
 
-const char* rn_version(void) { return "0.2.0"; }
+rn_status rn_fp8_gemm_config(int64_t M, int64_t N, int64_t K, int32_t num_sms,
+                             int32_t* config) {
+    if (!config) return RN_ERR_NULL;
+    if (M < 0 || N < 1 || K < 1) return RN_ERR_SHAPE;
+    *config = gemm_config(M, N, num_sms > 0 ? num_sms : kDefaultSms);
+    return RN_OK;
+}
+
+rn_status rn_fp8_gemm_force_config(int32_t config) {
+    if (config < -1 || config >= rn::kNumGemmConfigs) return RN_ERR_CONFIG;
+    g_force_gemm.store(config);
+    return RN_OK;
+}
+
+const char* rn_version(void) { return "0.3.0"; }
 
 }  // extern "C"

@@ -40,6 +40,21 @@ struct GemmArgs {
     int64_t M, N, K;
     int device;
     int num_sms;
+    int config;           // GemmConfig: tile shape and orientation
+};
+
+// Tile configurations of the fp8 GEMM (values of rn_gemm_config in the public
+// header). Token-major tiles are (tokens x channels); channel-major tiles
+// compute D^T and are (channels x tokens).
+enum GemmConfig {
+    kGemmTok128Ch128 = 0,
+    kGemmCh128Tok16 = 1,
+    kGemmCh128Tok32 = 2,
+    kGemmCh128Tok64 = 3,
+    kGemmCh64Tok16 = 4,
+    kGemmCh64Tok32 = 5,
+    kGemmCh64Tok64 = 6,
+    kNumGemmConfigs = 7
 };
 
 struct Launch {

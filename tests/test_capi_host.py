@@ -15,6 +15,7 @@ import os
 import re
 import subprocess
 
+import numpy as np
 import pytest
 import torch
 
@@ -295,6 +296,73 @@ def test_force_staged_hook():
     finally:
         rn.force_staged(0, 0, 0)
     assert rn.plan_launch("fused_add_rms_norm", BF, 50, 3840)["kernel"] == 0
+
+
+CH_SHAPES = {"ch64_tok16": (64, 16), "ch64_tok32": (64, 32), "ch64_tok64": (64, 64),
+             "ch128_tok16": (128, 16), "ch128_tok32": (128, 32), "ch128_tok64": (128, 64)}
+
+
+def _tiles(name, M, N):
+    ch, tok = CH_SHAPES[name]
+    return -(-N // ch) * -(-M // tok)
+
+
+def test_gemm_config_choice():
+    """Channel-major tiles maximising the tiles of one wave; the Gemma 4 12B
+    decode shapes get the configurations measured fastest."""
+    cfg = rn.fp8_gemm_config
+    assert cfg(1, 8192, 3840, 148) == "ch64_tok16"      # 128 tiles
+    assert cfg(16, 8192, 3840, 148) == "ch64_tok16"
+    assert cfg(32, 8192, 3840, 148) == "ch64_tok32"     # 128 tiles (tok16 would be 256)
+    assert cfg(64, 8192, 3840, 148) == "ch64_tok64"
+    assert cfg(32, 3840, 4096, 148) == "ch64_tok16"     # 120 tiles
+    assert cfg(64, 3840, 15360, 148) == "ch64_tok32"    # 120 tiles
+    assert cfg(1, 30720, 3840, 148) == "ch128_tok16"    # nothing fits one wave
+    assert cfg(33, 30720, 3840, 148) == "ch128_tok64"
+    assert cfg(256, 3840, 8192, 148) == "ch128_tok64"   # 120 tiles
+    assert cfg(256, 8192, 3840, 148) == "tok128_ch128"
+    assert cfg(8192, 8192, 3840, 148) == "tok128_ch128"
+    assert cfg(0, 8, 16) in rn.GEMM_CONFIGS               # empty problem: any valid config
+    for bad in ((-1, 8, 16), (1, 0, 16), (1, 8, 0)):
+        with pytest.raises(rn.RmsNormError) as e:
+            cfg(*bad)
+        assert e.value.name == "RN_ERR_SHAPE"
+
+
+@pytest.mark.parametrize("seed", range(3))
+def test_gemm_config_choice_is_the_fullest_wave(seed):
+    """Brute force over the rule's candidates on random shapes."""
+    rng = np.random.default_rng(seed)
+    for _ in range(300):
+        M = int(rng.integers(1, 600))
+        N = 8 * int(rng.integers(1, 5000))
+        sms = int(rng.integers(1, 200))
+        got = rn.fp8_gemm_config(M, N, 16, sms)
+        fits = {c: _tiles(c, M, N) for c in CH_SHAPES if _tiles(c, M, N) <= sms}
+        if fits:
+            assert got in fits and fits[got] == max(fits.values()), (M, N, sms, got)
+            order = list(CH_SHAPES)
+            assert got == next(c for c in order if fits.get(c) == max(fits.values()))
+        elif M <= 64:
+            assert got == min((c for c in CH_SHAPES if c.startswith("ch128") and
+                               CH_SHAPES[c][1] >= M), key=lambda c: CH_SHAPES[c][1])
+        else:
+            assert got == "tok128_ch128"
+
+
+def test_gemm_force_config_hook():
+    for bad in (-2, 7, 100):
+        with pytest.raises(rn.RmsNormError) as e:
+            rn.fp8_gemm_force_config(bad)
+        assert e.value.name == "RN_ERR_CONFIG"
+    try:
+        for name in rn.GEMM_CONFIGS:
+            rn.fp8_gemm_force_config(name)
+            assert rn.fp8_gemm_config(8192, 8192, 3840) == name
+            assert rn.fp8_gemm_config(1, 8, 16) == name
+    finally:
+        rn.fp8_gemm_force_config(None)
+    assert rn.fp8_gemm_config(8192, 8192, 3840) == "tok128_ch128"
 
 
 def test_status_strings():

@@ -82,8 +82,29 @@ def test_gemm_small_shapes_full(M, N, K):
     print(M, N, K, "correctly rounded fraction", exact_frac)
 
 
+# Shapes that leave ragged tiles in every configuration: M below, at and
+# above the token widths 16/32/64, N not a multiple of 64 or 128.
+CONFIG_SHAPES = [(1, 8, 16), (5, 264, 400), (16, 128, 128), (33, 520, 272), (64, 3840, 4096),
+                 (130, 200, 144)]
+
+
+@pytest.mark.parametrize("M,N,K", CONFIG_SHAPES)
+@pytest.mark.parametrize("config", list(rn.GEMM_CONFIGS))
+def test_gemm_every_config(config, M, N, K):
+    """Each tile configuration (token-major, and channel-major D^T tiles)
+    forced on shapes that are ragged for it, checked in full."""
+    a, b, sa, sb = _operands(M, N, K, seed=7 * M + N + K)
+    rn.fp8_gemm_force_config(config)
+    try:
+        d = _gemm(a.cuda(), b.cuda(), sa.cuda(), sb.cuda())
+    finally:
+        rn.fp8_gemm_force_config(None)
+    exact_frac = _check(d, codes8(a), codes8(b), sa.numpy(), sb.numpy())
+    print(config, M, N, K, "correctly rounded fraction", exact_frac)
+
+
 @pytest.mark.parametrize("N,K", GEMMA_NK)
-@pytest.mark.parametrize("M", [1, 256, 8192])
+@pytest.mark.parametrize("M", [1, 16, 33, 64, 256, 8192])
 def test_gemm_gemma_shapes(M, N, K):
     a, b, sa, sb = _operands(M, N, K, seed=N + K + M, device="cuda")
     d = _gemm(a, b, sa, sb)

@@ -66,6 +66,8 @@ def _load():
         lib.oracle_silu_and_mul_fp8.restype = I
         lib.oracle_fp8_rowwise_gemm.argtypes = [P, P, P, P, I64, I64, I64, I64, I64, P, P]
         lib.oracle_fp8_rowwise_gemm.restype = I
+        lib.oracle_allreduce_sum16.argtypes = [P, I, I64, I, P]
+        lib.oracle_allreduce_sum16.restype = I
         lib.oracle_decode16_array.argtypes = [P, I, I64, P]
         lib.oracle_encode16_array.argtypes = [P, I, I64, P]
         lib.oracle_decode_e4m3_array.argtypes = [P, I64, P]
@@ -270,6 +272,49 @@ def fp8_rowwise_gemm(a_codes, b_codes, a_scale, b_scale, rows=None, want_y: bool
 
     _run(blk, M, 1, threads)
     return (D, y) if want_y else D
+
+
+def allreduce_sum16(parts, dtype: str, threads: int = 1) -> np.ndarray:
+    """x = RNE16(exact sum over ranks) of W partial arrays (16-bit bits,
+    stacked on a leading rank axis: [W, ...]). Returns bits of shape [...]."""
+    lib = _load()
+    pb = _bits16(parts)
+    W = pb.shape[0]
+    flat = pb.reshape(W, -1)
+    n = flat.shape[1]
+    x = np.empty(n, np.uint16)
+    dt = DTYPES[dtype]
+    chunks = _blocks(n, threads)
+
+    def blk(c):
+        i0, i1 = c
+        part = np.ascontiguousarray(flat[:, i0:i1])
+        rc = lib.oracle_allreduce_sum16(_ptr(part), W, i1 - i0, dt, _ptr(x[i0:i1]))
+        assert rc == 0
+
+    if len(chunks) <= 1:
+        for c in chunks:
+            blk(c)
+    else:
+        with ThreadPoolExecutor(len(chunks)) as ex:
+            list(ex.map(blk, chunks))
+    return x.reshape(pb.shape[1:])
+
+
+def allreduce_fused_add_rms_norm(parts, residual, weight, dtype: str, eps: float,
+                                 want_y: bool = False, threads: int = 1):
+    """Tensor-parallel form: x = allreduce_sum16(parts) ([W, T, H] partials),
+    then fused_add_rms_norm(x, residual). Returns (x, r', out[, y])."""
+    x = allreduce_sum16(parts, dtype, threads)
+    return (x, *fused_add_rms_norm(x, residual, weight, dtype, eps, want_y, threads))
+
+
+def allreduce_fused_add_rms_norm_fp8(parts, residual, weight, dtype: str, eps: float,
+                                     want_y: bool = False, threads: int = 1):
+    """x = allreduce_sum16(parts), then fused_add_rms_norm_fp8(x, residual).
+    Returns (x, r', q, scale[, y])."""
+    x = allreduce_sum16(parts, dtype, threads)
+    return (x, *fused_add_rms_norm_fp8(x, residual, weight, dtype, eps, want_y, threads))
 
 
 def usable_cores() -> int:

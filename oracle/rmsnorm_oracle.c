@@ -354,3 +354,117 @@ int oracle_fp8_rowwise_gemm(const uint8_t* A, const uint8_t* B, const float* a_s
     }
     return 0;
 }
+
+/* ------------------------------------------------------------------------ */
+/* All-reduce sum of tensor-parallel partials (the all-reduce that precedes  */
+/* the residual add and RMSNorm in a tensor-parallel decoder layer; AITER    */
+/* provides all-reduce and RMSNorm to SGLang, "AITER: AMD's operator library */
+/* for ROCm", ecosystem section). Element i of the result is the exact real  */
+/* sum of the W partial values parts[r][i], rounded once to the 16-bit       */
+/* format (RNE16 as above). Non-finite inputs follow IEEE addition: any NaN, */
+/* or +inf with -inf, gives NaN; otherwise an infinity gives that infinity.  */
+/* An exact zero sum is -0 only when every term is -0 (round-to-nearest).   */
+/*                                                                          */
+/* The exact sum is kept as a two's-complement integer multiple of          */
+/* 2^ACC_LSB in ACC_LIMBS 64-bit limbs: every finite bf16 or fp16 value is an */
+/* integer below 2^24 times a power of two >= 2^-160, and the largest sum of */
+/* up to 64 terms stays below 2^300, so no bit is ever lost. The integer is */
+/* then rounded to odd at 53 bits (its top 53 bits, with the lowest of them  */
+/* set when anything below is non-zero), an exact binary64 value; rounding   */
+/* that to nearest at 8 or 11 bits gives the correctly rounded sum (rounding */
+/* to odd with at least two extra bits makes the second rounding innocuous:  */
+/* Boldo and Melquiond, "When double rounding is odd", 2005).               */
+
+#define ACC_LIMBS 6
+#define ACC_LSB (-160)
+
+typedef struct { uint64_t w[ACC_LIMBS]; } exact_acc;
+
+/* acc += sign * m * 2^(ACC_LSB + sh), 0 <= m < 2^24, 0 <= sh <= 300. */
+static void acc_add(exact_acc* acc, int negative, uint64_t m, int sh) {
+    uint64_t t[ACC_LIMBS] = {0};
+    int li = sh / 64, bi = sh % 64;
+    t[li] = m << bi;
+    if (bi != 0 && li + 1 < ACC_LIMBS) t[li + 1] = m >> (64 - bi);
+    if (negative) { /* two's complement: invert, add one */
+        unsigned carry = 1;
+        for (int k = 0; k < ACC_LIMBS; ++k) {
+            uint64_t inv = ~t[k];
+            t[k] = inv + carry;
+            carry = carry && t[k] == 0;
+        }
+    }
+    unsigned carry = 0;
+    for (int k = 0; k < ACC_LIMBS; ++k) {
+        uint64_t s = acc->w[k] + t[k];
+        unsigned c1 = s < acc->w[k];
+        uint64_t s2 = s + carry;
+        unsigned c2 = s2 < s;
+        acc->w[k] = s2;
+        carry = c1 | c2;
+    }
+}
+
+/* The accumulated exact value, rounded to odd at 53 significant bits. */
+static double acc_to_f64_odd(const exact_acc* acc) {
+    uint64_t a[ACC_LIMBS];
+    memcpy(a, acc->w, sizeof a);
+    int negative = (int)(a[ACC_LIMBS - 1] >> 63);
+    if (negative) {
+        unsigned carry = 1;
+        for (int k = 0; k < ACC_LIMBS; ++k) {
+            uint64_t inv = ~a[k];
+            a[k] = inv + carry;
+            carry = carry && a[k] == 0;
+        }
+    }
+    int h = -1; /* highest set bit */
+    for (int k = ACC_LIMBS - 1; k >= 0 && h < 0; --k)
+        for (int b = 63; b >= 0; --b)
+            if ((a[k] >> b) & 1) { h = 64 * k + b; break; }
+    if (h < 0) return 0.0;
+    double mag;
+    if (h < 53) {
+        mag = ldexp((double)a[0], ACC_LSB); /* below 2^53: exact */
+    } else {
+        int lo = h - 52; /* keep bits [lo, h] */
+        uint64_t top = 0;
+        for (int b = h; b >= lo; --b) top = (top << 1) | ((a[b / 64] >> (b % 64)) & 1);
+        int sticky = 0;
+        for (int b = lo - 1; b >= 0 && !sticky; --b) sticky = (int)((a[b / 64] >> (b % 64)) & 1);
+        if (sticky) top |= 1;
+        mag = ldexp((double)top, lo + ACC_LSB);
+    }
+    return negative ? -mag : mag;
+}
+
+/* parts: W arrays of n 16-bit values, rank r's at parts + r * n. */
+int oracle_allreduce_sum16(const uint16_t* parts, int W, int64_t n, int dtype, uint16_t* x) {
+    if ((dtype != OR_F16 && dtype != OR_BF16) || W < 1 || W > 64 || n < 0) return -1;
+    for (int64_t i = 0; i < n; ++i) {
+        exact_acc acc;
+        memset(&acc, 0, sizeof acc);
+        int nan = 0, pinf = 0, ninf = 0, all_neg_zero = 1;
+        for (int r = 0; r < W; ++r) {
+            double v = load16(parts + (int64_t)r * n, i, dtype);
+            if (isnan(v)) { nan = 1; continue; }
+            if (isinf(v)) { if (v > 0) pinf = 1; else ninf = 1; continue; }
+            if (!(v == 0.0 && signbit(v))) all_neg_zero = 0;
+            if (v == 0.0) continue;
+            int k;
+            double f = frexp(fabs(v), &k);         /* |v| = f * 2^k, f in [0.5, 1) */
+            uint64_t m = (uint64_t)ldexp(f, 24);  /* exact: <= 11 significant bits */
+            acc_add(&acc, v < 0, m, (k - 24) - ACC_LSB);
+        }
+        double s;
+        if (nan || (pinf && ninf)) s = NAN;
+        else if (pinf) s = INFINITY;
+        else if (ninf) s = -INFINITY;
+        else {
+            s = acc_to_f64_odd(&acc);
+            if (s == 0.0) s = all_neg_zero ? -0.0 : 0.0;
+        }
+        x[i] = store16(s, dtype);
+    }
+    return 0;
+}

@@ -24,6 +24,7 @@ from __future__ import annotations
 import bisect
 import math
 from decimal import Decimal
+from fractions import Fraction
 
 import numpy as np
 import torch
@@ -448,6 +449,170 @@ def pin_gemm_matches_float64_matmul(orc, golden=None):
     rows = np.array([0, 5, 23])
     D2, y2 = orc.fp8_rowwise_gemm(A, B, sa, sb, rows=rows, want_y=True)
     np.testing.assert_array_equal(y2, ref[rows])
+
+
+# --------------------------------------------------------------------------
+# All-reduce sum of tensor-parallel partials (the all-reduce that precedes the
+# residual add and RMSNorm in a tensor-parallel layer; "AITER: AMD's operator
+# library for ROCm", ecosystem section: all-reduce and RMSNorm for SGLang).
+
+_FMT16 = {"bf16": (8, -126, 127), "fp16": (11, -14, 15)}  # p, emin, emax
+
+
+def _exact16(q: Fraction, dtype: str) -> float:
+    """Round-to-nearest-even of an exact rational onto the 16-bit format,
+    from the format definition (p significand bits, gradual underflow,
+    overflow to infinity past the largest finite value); returns the value."""
+    p, emin, emax = _FMT16[dtype]
+    if q == 0:
+        return 0.0
+    a = abs(q)
+    E = a.numerator.bit_length() - a.denominator.bit_length()
+    while Fraction(2) ** E > a:
+        E -= 1
+    while Fraction(2) ** (E + 1) <= a:
+        E += 1
+    quantum = Fraction(2) ** (max(E, emin) - (p - 1))
+    n = a / quantum
+    fl = n.numerator // n.denominator
+    frac = n - fl
+    r = fl + 1 if frac > Fraction(1, 2) else fl if frac < Fraction(1, 2) else fl + (fl % 2)
+    v = r * quantum
+    if v > (2 - Fraction(2) ** (1 - p)) * Fraction(2) ** emax:
+        return math.copysign(math.inf, q)
+    return math.copysign(float(v), q)
+
+
+def _lib16(values, dtype: str) -> np.ndarray:
+    """Bits of exactly representable values, by numpy / torch conversion."""
+    v = np.asarray(values, dtype=np.float64)
+    if dtype == "fp16":
+        return v.astype(np.float16).view(np.uint16)
+    return bits16(torch.from_numpy(v).to(torch.bfloat16))
+
+
+def _finite_codes(rng, n, dtype, lo_exp=None, hi_exp=None):
+    """Random finite 16-bit codes whose exponent field spans [lo_exp, hi_exp]."""
+    if dtype == "bf16":
+        lo, hi = (lo_exp or 0), (hi_exp or 254)
+        e = rng.integers(lo, hi + 1, n)
+        m = rng.integers(0, 128, n)
+        return ((rng.integers(0, 2, n) << 15) | (e << 7) | m).astype(np.uint16)
+    lo, hi = (lo_exp or 0), (hi_exp or 30)
+    e = rng.integers(lo, hi + 1, n)
+    m = rng.integers(0, 1024, n)
+    return ((rng.integers(0, 2, n) << 15) | (e << 10) | m).astype(np.uint16)
+
+
+def pin_allreduce_single_rank_identity(orc, golden=None):
+    """One rank: the sum is the partial itself, for every 16-bit pattern."""
+    for dtype in ("bf16", "fp16"):
+        got = orc.allreduce_sum16(ALL16.reshape(1, -1), dtype)
+        nan = _nan16(ALL16, dtype)
+        assert (_nan16(got, dtype) == nan).all()
+        np.testing.assert_array_equal(got[~nan], ALL16[~nan])
+
+
+def pin_allreduce_two_ranks_library_addition(orc, golden=None):
+    """Two ranks: torch's bf16 and numpy's float16 addition (one operation,
+    computed wider and rounded once: correctly rounded), over random patterns
+    and every pairing of the special values (zeros, infinities, NaN,
+    subnormal extremes, the largest finite values)."""
+    rng = np.random.default_rng(71)
+    for dtype in ("bf16", "fp16"):
+        special = ([0x0000, 0x8000, 0x7F80, 0xFF80, 0x7FC0, 0x0001, 0x8001, 0x7F7F, 0xFF7F,
+                    0x3F80, 0xBF80, 0x3B80] if dtype == "bf16" else
+                   [0x0000, 0x8000, 0x7C00, 0xFC00, 0x7E00, 0x0001, 0x8001, 0x7BFF, 0xFBFF,
+                    0x3C00, 0xBC00, 0x1400])
+        sp = np.array(special, dtype=np.uint16)
+        a = np.concatenate([rng.integers(0, 65536, 100000).astype(np.uint16), np.repeat(sp, sp.size)])
+        b = np.concatenate([rng.integers(0, 65536, 100000).astype(np.uint16), np.tile(sp, sp.size)])
+        if dtype == "bf16":
+            ta = torch.from_numpy(a.view(np.int16).copy()).view(torch.bfloat16)
+            tb = torch.from_numpy(b.view(np.int16).copy()).view(torch.bfloat16)
+            ref = bits16(ta + tb)
+        else:
+            with np.errstate(over="ignore", invalid="ignore"):
+                ref = (a.view(np.float16) + b.view(np.float16)).view(np.uint16)
+        got = orc.allreduce_sum16(np.stack([a, b]), dtype)
+        nan = _nan16(ref, dtype)
+        assert (_nan16(got, dtype) == nan).all()
+        np.testing.assert_array_equal(got[~nan], ref[~nan])
+
+
+def pin_allreduce_exact_rationals(orc, golden=None):
+    """3 to 8 ranks: the exact rational sum rounded by the format definition,
+    on values spanning the whole exponent range (where binary64 summation is
+    not exact) and on built rounding ties broken only by a far smaller term."""
+    rng = np.random.default_rng(72)
+    for dtype in ("bf16", "fp16"):
+        for W in (3, 5, 8):
+            parts = np.stack([_finite_codes(rng, 400, dtype) for _ in range(W)])
+            vals = orc.decode16(parts, dtype)
+            want = [_exact16(sum(Fraction(float(v)) for v in vals[:, i]), dtype)
+                    for i in range(parts.shape[1])]
+            got = orc.decode16(orc.allreduce_sum16(parts, dtype), dtype)
+            nz = np.array(want) != 0
+            np.testing.assert_array_equal(got[nz], np.array(want)[nz])
+            np.testing.assert_array_equal(got[~nz], 0.0)
+        tiny = 2.0 ** -133 if dtype == "bf16" else 2.0 ** -24
+        step = 2.0 ** -8 if dtype == "bf16" else 2.0 ** -11  # half an ulp of 1
+        cases = [([1.0, step, 0.0], 1.0), ([1.0, step, tiny], 1.0 + 2 * step),
+                 ([1.0, step, -tiny], 1.0), ([1.0 + 2 * step, step, 0.0], 1.0 + 4 * step),
+                 ([1.0 + 2 * step, step, -tiny], 1.0 + 2 * step),
+                 ([-1.0, -step, -tiny], -(1.0 + 2 * step)), ([tiny, -tiny, tiny], tiny),
+                 ([4.0, -4.0, tiny], tiny)]
+        parts = np.stack([_lib16([c[0][r] for c in cases], dtype) for r in range(3)])
+        want = _lib16([c[1] for c in cases], dtype)
+        np.testing.assert_array_equal(orc.allreduce_sum16(parts, dtype), want)
+
+
+def pin_allreduce_signed_zero_and_overflow(orc, golden=None):
+    for dtype in ("bf16", "fp16"):
+        z, nz = 0x0000, 0x8000
+        parts = np.array([[nz, nz, z, nz], [nz, z, nz, nz], [nz, nz, nz, z]], dtype=np.uint16)
+        np.testing.assert_array_equal(orc.allreduce_sum16(parts, dtype), [nz, z, z, z])
+        big = 0x7F7F if dtype == "bf16" else 0x7BFF
+        inf = 0x7F80 if dtype == "bf16" else 0x7C00
+        parts = np.array([[big, big | 0x8000], [big, big | 0x8000]], dtype=np.uint16)
+        np.testing.assert_array_equal(orc.allreduce_sum16(parts, dtype), [inf, inf | 0x8000])
+    # fp16: 65504 + 16 = 65520 is the midpoint to 2^16: ties to even overflow
+    parts = _lib16([[65504.0, 65504.0], [16.0, 15.0]], "fp16").reshape(2, 2)
+    np.testing.assert_array_equal(orc.allreduce_sum16(parts, "fp16"), [0x7C00, 0x7BFF])
+
+
+def pin_allreduce_rank_order_invariance(orc, golden=None):
+    """The exact sum does not depend on the order of the ranks."""
+    rng = np.random.default_rng(73)
+    for dtype in ("bf16", "fp16"):
+        parts = np.stack([_finite_codes(rng, 20000, dtype) for _ in range(8)])
+        ref = orc.allreduce_sum16(parts, dtype)
+        for _ in range(3):
+            perm = rng.permutation(8)
+            np.testing.assert_array_equal(orc.allreduce_sum16(parts[perm], dtype), ref)
+
+
+def pin_allreduce_fused_composition(orc, golden=None):
+    """The tensor-parallel fused ops are the all-reduce followed by the plain
+    fused ops: with one rank holding x and the others zeros, and with x split
+    exactly into two halves, they reduce to fused_add_rms_norm(x, r)."""
+    for dtype in ("bf16", "fp16"):
+        wl = synth.make_inputs("decode", "fused_add_rms_norm", dtype, 16, 4096)
+        x, r, w = bits16(wl.x), bits16(wl.residual), bits16(wl.weight)
+        r_ref, out_ref = orc.fused_add_rms_norm(x, r, w, dtype, wl.eps)
+        zeros = np.zeros_like(x)
+        half = bits16(wl.x / 2)  # exact: scaling by a power of two (normal range)
+        assert (orc.decode16(half, dtype) * 2 == orc.decode16(x, dtype)).all()
+        for parts in (np.stack([zeros, x, zeros, zeros]), np.stack([half, half])):
+            xs, r2, out = orc.allreduce_fused_add_rms_norm(parts, r, w, dtype, wl.eps)
+            np.testing.assert_array_equal(xs, x)
+            np.testing.assert_array_equal(r2, r_ref)
+            np.testing.assert_array_equal(out, out_ref)
+            xs, r3, q, sc = orc.allreduce_fused_add_rms_norm_fp8(parts, r, w, dtype, wl.eps)
+            r4, q4, sc4 = orc.fused_add_rms_norm_fp8(x, r, w, dtype, wl.eps)
+            np.testing.assert_array_equal(r3, r4)
+            np.testing.assert_array_equal(q, q4)
+            np.testing.assert_array_equal(sc, sc4)
 
 
 PINS = [v for k, v in sorted(globals().items()) if k.startswith("pin_")]

@@ -19,7 +19,7 @@ import residual_add_rmsnorm_rms_b200 as rn
 import synth
 from residual_add_rmsnorm_rms_b200 import torch_ops  # noqa: F401  (registers the ops)
 from tests.cmp_util import bits16, codes8, ulp16
-from tests.gpu_util import CORES, sample_rows
+from tests.gpu_util import CORES, oracle_run, sample_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -115,18 +115,33 @@ def test_gemm_gemma_shapes(M, N, K):
 
 
 def test_norm_then_gemm_chain():
-    """The decode chain: fused_add_rms_norm_fp8 codes and per-token scales
-    feed the GEMM directly (GPU codes go to both the GPU GEMM and the oracle)."""
+    """The decode chain through the torch ops: fused_add_rms_norm_fp8's codes
+    and [T, 1] per-token scales feed fp8_rowwise_gemm directly. The GEMM's
+    parity is judged on the oracle's own codes and scales for the same
+    synthetic inputs (no GPU output becomes an oracle input); the GPU chain
+    must then give the same D on every row whose GPU codes and scale equal
+    the oracle's (and both stages are checked against the oracle elsewhere)."""
     wl = synth.make_inputs("prefill", "fused_add_rms_norm_fp8", "bf16", 256, 3840)
-    q = torch.empty(256, 3840, dtype=torch.float8_e4m3fn, device="cuda")
-    s = torch.empty(256, dtype=torch.float32, device="cuda")
-    rn.fused_add_rms_norm_fp8(q, s, wl.x.cuda(), wl.residual.cuda().clone(), wl.weight.cuda(),
-                              wl.eps)
+    want = oracle_run("fused_add_rms_norm_fp8", wl.x, wl.residual, wl.weight, wl.eps, "bf16")
     _, b, _, sb = _operands(1, 8192, 3840, seed=77)
-    d = torch.ops.rmsnorm_b200.fp8_rowwise_gemm(q, b.cuda(), s, sb.cuda())
+    b, sb = b.cuda(), sb.cuda()
+
+    q_o = torch.from_numpy(want["q"].reshape(256, 3840)).cuda().view(torch.float8_e4m3fn)
+    s_o = torch.from_numpy(want["scale"].astype(np.float32)).cuda().view(256, 1)
+    d_o = torch.ops.rmsnorm_b200.fp8_rowwise_gemm(q_o, b, s_o, sb)
     torch.cuda.synchronize()
-    assert d.shape == (256, 8192) and d.dtype == torch.bfloat16
-    _check(d, codes8(q), codes8(b), s.cpu().numpy(), sb.numpy())
+    assert d_o.shape == (256, 8192) and d_o.dtype == torch.bfloat16
+    _check(d_o, want["q"].reshape(256, 3840), codes8(b), want["scale"].astype(np.float32),
+           sb.cpu().numpy())
+
+    q, s = torch.ops.rmsnorm_b200.fused_add_rms_norm_fp8(
+        wl.x.cuda(), wl.residual.cuda().clone(), wl.weight.cuda(), wl.eps)
+    d = torch.ops.rmsnorm_b200.fp8_rowwise_gemm(q, b, s, sb)
+    torch.cuda.synchronize()
+    same = ((codes8(q) == want["q"].reshape(256, 3840)).all(axis=1)
+            & (s.view(-1).cpu().numpy() == want["scale"].astype(np.float32)))
+    assert same.mean() > 0.5
+    assert (bits16(d)[same] == bits16(d_o)[same]).all()
 
 
 def test_gemm_validation():

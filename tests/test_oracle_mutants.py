@@ -51,6 +51,16 @@ MUTANTS = {
                              "double y = acc * (double)b_scale[n];"),
     "gemm_scales_swapped": ("double y = acc * (double)a_scale[m] * (double)b_scale[n];",
                             "double y = acc * (double)a_scale[n % M] * (double)b_scale[m % N];"),
+    "allreduce_sticky_dropped": ("if (sticky) top |= 1;", "if (0) top |= 1;"),
+    "allreduce_sign_ignored": ("acc_add(&acc, v < 0, m, (k - 24) - ACC_LSB);",
+                               "acc_add(&acc, 0, m, (k - 24) - ACC_LSB);"),
+    "allreduce_last_rank_dropped": ("for (int r = 0; r < W; ++r) {\n            double v = load16(parts",
+                                    "for (int r = 0; r < W - 1; ++r) {\n            double v = load16(parts"),
+    "allreduce_zero_sign": ("if (s == 0.0) s = all_neg_zero ? -0.0 : 0.0;", "if (s == 0.0) s = 0.0;"),
+    "allreduce_inf_minus_inf": ("if (nan || (pinf && ninf)) s = NAN;", "if (nan) s = NAN;"),
+    "allreduce_in_binary64": ("            s = acc_to_f64_odd(&acc);",
+                              "            s = 0.0;\n            for (int r = 0; r < W; ++r) s += load16(parts + (int64_t)r * n, i, dtype);"),
+    "allreduce_carry_lost": ("        carry = c1 | c2;", "        carry = c1;"),
     "bf16_overflow_threshold": ("if (r > maxf) return sign | 0x7f80; /* overflow to infinity */",
                                 "if (r >= maxf) return sign | 0x7f80;"),
 }

@@ -69,7 +69,7 @@ def kernel_digest(plan: dict) -> str:
     the launch shape the planner gives it on the bench's workload."""
     h = hashlib.sha256()
     d = os.path.join(ROOT, "residual_add_rmsnorm_rms_b200", "csrc")
-    for name in ("rmsnorm_kernels.cu", "rn_device.cuh", "rn_internal.h"):
+    for name in ("rmsnorm_kernels.cu", "rn_device.cuh", "rn_vec8.cuh", "rn_internal.h"):
         with open(os.path.join(d, name), "rb") as f:
             h.update(name.encode() + f.read())
     shape = {k: plan[k] for k in ("kernel", "threads_per_row", "vectors_per_thread",
@@ -641,6 +641,78 @@ def time_gemm_cell(rn, M, N, K, iters, device, configs=(None,)):
     return out
 
 
+def tp_bytes(fp8: bool, W: int, T: int, H: int) -> int:
+    """Unique bytes one single-device group call moves: per rank and row, the
+    partial read (2H), its copy into the exchange buffer (2H), one read of
+    that buffer (2H: each buffer is read by all W ranks, counted once), the
+    residual read and write (4H) and the output (2H, or H codes + 4)."""
+    return W * T * ((11 * H + 4) if fp8 else 12 * H)
+
+
+def time_tp_cell(rn, fp8, W, T, H, iters, device):
+    """A whole tensor-parallel group of W ranks on this device (one launch
+    per call): mean time per call over `iters` eager calls rotating over
+    operand sets of >= 4x L2 (at most 8), and CUDA-graph replay time of 50
+    captured calls for calls under 60 us."""
+    from residual_add_rmsnorm_rms_b200.allreduce import AllReduceComm
+    wl = synth.make_tp_inputs("bf16", W, T, H, device=device)
+    comm = AllReduceComm.single_device(W, T, H, device)
+    per = 2 * W * T * H * 3
+    n = min(8, max(1, math.ceil(4 * torch.cuda.get_device_properties(device).L2_cache_size / per)))
+    sets = []
+    for _ in range(n):
+        res = wl.residual.unsqueeze(0).repeat(W, 1, 1).contiguous()
+        s = {"x": wl.x.clone(), "r": res}
+        if fp8:
+            s["q"] = torch.empty(W, T, H, dtype=torch.float8_e4m3fn, device=device)
+            s["scale"] = torch.empty(W, T, dtype=torch.float32, device=device)
+        else:
+            s["out"] = torch.empty(W, T, H, dtype=torch.bfloat16, device=device)
+        sets.append(s)
+    w, eps = wl.weight, wl.eps
+    del wl
+
+    def call(i):
+        s = sets[i % n]
+        if fp8:
+            rn.allreduce_fused_add_rms_norm_fp8(s["q"], s["scale"], s["x"], s["r"], w, eps, comm)
+        else:
+            rn.allreduce_fused_add_rms_norm(s["out"], s["x"], s["r"], w, eps, comm)
+
+    for i in range(3):
+        call(i)
+    torch.cuda.synchronize(device)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for i in range(iters):
+        call(i)
+    e1.record()
+    torch.cuda.synchronize(device)
+    us = e0.elapsed_time(e1) / iters * 1e3
+    gus = None
+    if us < 60:
+        g = torch.cuda.CUDAGraph()
+        st = torch.cuda.Stream(device)
+        with torch.cuda.stream(st):
+            call(0)
+            torch.cuda.synchronize(device)
+            with torch.cuda.graph(g, stream=st):
+                for i in range(50):
+                    call(i)
+        g.replay()
+        torch.cuda.synchronize(device)
+        e0.record()
+        for _ in range(4):
+            g.replay()
+        e1.record()
+        torch.cuda.synchronize(device)
+        gus = e0.elapsed_time(e1) / 200 * 1e3
+        del g
+    del sets, comm
+    torch.cuda.empty_cache()
+    return us, gus
+
+
 def run_sweep(args, world, rank, local):
     import residual_add_rmsnorm_rms_b200 as rn
     device = torch.device("cuda", local)
@@ -665,6 +737,24 @@ def run_sweep(args, world, rank, local):
                "tpr": plan["threads_per_row"], "vpt": plan["vectors_per_thread"]}
         out.write(json.dumps(rec) + "\n")
         out.flush()
+    tp_cells = [(fp8, W, T, H) for fp8 in (False, True) for W in synth.TP_W
+                for T in synth.TP_T for H in (3840,)
+                if all(w in ("tp", "allreduce", str(W), str(T), str(H),
+                             "fp8" if fp8 else "bf16") for w in want)]
+    for fp8, W, T, H in tp_cells:
+        us, gus = time_tp_cell(rn, fp8, W, T, H, args.sweep_iters, device)
+        best = gus if gus is not None else us
+        nbytes = tp_bytes(fp8, W, T, H)
+        rec = {"workload": "tp", "op": "allreduce_fused_add_rms_norm" + ("_fp8" if fp8 else ""),
+               "dtype": "bf16", "W": W, "T": T, "H": H, "us": round(us, 3),
+               "graph_us": None if gus is None else round(gus, 3),
+               "gbs": round(nbytes / best / 1e3, 1),
+               "frac_of_measured": round(nbytes / best / 1e3 / peak, 4), "bytes": nbytes,
+               "rows_per_s": round(W * T / (best / 1e6), 1),
+               "remote_bytes_per_rank": (W - 1) * 2 * T * H,
+               "how": "whole group on one device, one cooperative launch per call"}
+        out.write(json.dumps(rec) + "\n")
+        out.flush()
     gemm_cells = [(M, N, K) for (N, K) in GEMMA_NK for M in GEMM_M
                   if all(w in ("gemm", "fp8_rowwise_gemm", str(M), f"{N}x{K}") for w in want)]
     fp8_peak, fp8_src = measured_fp8_peak()
@@ -687,7 +777,8 @@ def run_sweep(args, world, rank, local):
             out.flush()
     out.close()
     assert rn.device_errors() == 0
-    print(json.dumps({"sweep": args.sweep_out, "cells": len(cells) + len(gemm_cells)}))
+    print(json.dumps({"sweep": args.sweep_out,
+                      "cells": len(cells) + len(tp_cells) + len(gemm_cells)}))
 
 
 def main():

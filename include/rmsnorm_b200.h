@@ -87,7 +87,8 @@ typedef enum {
     RN_ERR_VARIANCE_SIZE = 7, /* variance_size != -1 */
     RN_ERR_EPS = 8,           /* eps negative, NaN or infinite */
     RN_ERR_CUDA = 9,          /* a CUDA runtime call failed */
-    RN_ERR_CONFIG = 10        /* rn_force_plan / rn_plan_launch: unsupported request */
+    RN_ERR_CONFIG = 10,       /* rn_force_plan / rn_plan_launch: unsupported request */
+    RN_ERR_COMM = 11          /* all-reduce: bad group description or exchange buffers too small */
 } rn_status;
 
 typedef enum {
@@ -201,6 +202,85 @@ RN_API rn_status rn_fp8_gemm_config(int64_t M, int64_t N, int64_t K, int32_t num
  * thread-safe with concurrent launches; meant for tests and tuning. */
 RN_API rn_status rn_fp8_gemm_force_config(int32_t config);
 
+/* ---- tensor-parallel all-reduce fused with the residual add and RMSNorm --
+ *
+ * In a tensor-parallel decoder layer each rank's row-parallel linear layer
+ * leaves a partial sum of the activations; an all-reduce adds the partials
+ * before the residual add and RMSNorm (SGLang takes all-reduce and RMSNorm
+ * from AITER: "AITER: AMD's operator library for ROCm", ecosystem section).
+ * These entry points do all three in one kernel per call, on every rank:
+ *   x = RNE16(sum over the ranks' partials), residual := RNE16(x + residual),
+ *   then out = RNE16(rms_norm(residual) * w)   (rn_allreduce_fused_add_rms_norm)
+ *   or q, scale as rn_fused_add_rms_norm_fp8   (rn_allreduce_fused_add_rms_norm_fp8).
+ * Every rank obtains bit-identical results (the residual is replicated).
+ * x is the correctly rounded sum of the partials whenever their binary64 sum
+ * is exact: always for fp16, and for bf16 whenever an element's non-zero
+ * partials span at most 42 binades; otherwise it can differ from it by one
+ * unit in the last place.
+ *
+ * Exchange: one-shot over peer memory (NVLink/NVSwitch loads and stores, no
+ * collective library). Every rank owns an exchange buffer and a signal pad
+ * that every rank's device can address (CUDA IPC or any peer mapping); each
+ * call copies the local partial into the rank's own buffer, publishes it
+ * through the peers' signal pads, waits for all peers, then reads the W
+ * partials. Every rank of the group must make the same sequence of calls,
+ * with the same T, H, dtype and op, on the same device model, each call
+ * enqueued after the previous one on one stream per rank.
+ *
+ * Operands are those of rn_fused_add_rms_norm(_fp8), with `x` the local
+ * partial; when one call computes several ranks (local_ranks > 1), x,
+ * residual, out and q carry a leading rank dimension ([local_ranks, T, H] or
+ * any dense view flattening to [local_ranks * T, H]) and scale holds
+ * local_ranks * T values. Requirements beyond those of the fused ops: H a
+ * multiple of 8 and at most 32768, x, residual, out, weight, buffers and
+ * signal pads 16-byte aligned, q 8-byte aligned. out == x (in place) is
+ * allowed. T == 0 still performs the exchange handshake (so that the ranks'
+ * call counters stay equal) and writes nothing. */
+#define RN_ALLREDUCE_MAX_WORLD 8
+/* Signal pad bytes per rank: a 64-byte header (the rank's call counter and an
+ * arrival counter, kept by the kernel) and 2 x 1024 blocks x 8 ranks 32-bit
+ * flags. */
+#define RN_ALLREDUCE_SIGNAL_BYTES 65600
+
+typedef struct {
+    int32_t world;       /* ranks in the group, 1..RN_ALLREDUCE_MAX_WORLD */
+    int32_t rank;        /* group rank of the first (or only) rank this call computes */
+    int32_t local_ranks; /* ranks this call computes on this device: 1, or `world`
+                          * with rank == 0 (the whole group on one device) */
+    void* buffers[RN_ALLREDUCE_MAX_WORLD]; /* [world] each rank's exchange buffer, as
+                          * addressed from this device; the caller owns them */
+    void* signals[RN_ALLREDUCE_MAX_WORLD]; /* [world] each rank's signal pad of
+                          * RN_ALLREDUCE_SIGNAL_BYTES: zero-filled before the first
+                          * call, then written only by these kernels; one group's */
+    int64_t buffer_bytes; /* size of each exchange buffer: two halves, each holding
+                          * T * H 16-bit values: buffer_bytes >= 4 * T * H + 32 */
+    int64_t timeout_ns;  /* bound on each wait for a peer; <= 0 selects 1 second */
+} rn_allreduce_comm;
+
+/* Calls are numbered on the device: each launch reads its rank's call
+ * counter from the signal pad and advances it when its last block finishes,
+ * so calls captured in a CUDA graph stay numbered correctly on replay. */
+
+/* Errors: the fused ops' validation, then RN_ERR_COMM for an invalid `comm`
+ * (world, rank, local_ranks, a NULL or misaligned buffer or pad,
+ * buffers too small for T and H), RN_ERR_LAYOUT for the alignment rules
+ * above, RN_ERR_SHAPE for H > 32768 or a row count not divisible by
+ * local_ranks, RN_ERR_ALIAS when an operand overlaps a local exchange buffer
+ * or signal pad, RN_ERR_CUDA when the launch fails. A peer that does not
+ * publish within timeout_ns is not an error of the call (it is asynchronous):
+ * the waiting block leaves its rows unwritten and sets bit 1 of
+ * rn_device_errors. Asynchronous on `stream`. */
+RN_API rn_status rn_allreduce_fused_add_rms_norm(const rn_tensor* out, const rn_tensor* x,
+                                                 const rn_tensor* residual,
+                                                 const rn_tensor* weight, float eps,
+                                                 const rn_allreduce_comm* comm, void* stream);
+RN_API rn_status rn_allreduce_fused_add_rms_norm_fp8(const rn_tensor* q, const rn_tensor* scale,
+                                                     const rn_tensor* x,
+                                                     const rn_tensor* residual,
+                                                     const rn_tensor* weight, float eps,
+                                                     const rn_allreduce_comm* comm,
+                                                     void* stream);
+
 /* Static text for a status code (never NULL). */
 RN_API const char* rn_status_string(rn_status status);
 
@@ -284,7 +364,9 @@ RN_API rn_status rn_set_launch_options(int32_t pdl, int64_t max_grid);
 
 /* Reads and clears the device-side error flags of the current device:
  * bit 0 = a bounded wait inside the STAGED kernel timed out (some rows of
- * that call were not written). Synchronises with the device. */
+ * that call were not written); bit 1 = an all-reduce call waited longer than
+ * its timeout for a peer (some rows of that call were not written).
+ * Synchronises with the device. */
 RN_API rn_status rn_device_errors(uint32_t* flags);
 
 /* Writes up to `cap` compiled vectors_per_thread values into `out` and

@@ -25,7 +25,8 @@ import torch
 __all__ = [
     "RmsNormError", "rms_norm", "fused_add_rms_norm", "fused_add_rms_norm_fp8",
     "silu_and_mul_fp8", "fp8_rowwise_gemm", "fp8_gemm_config", "fp8_gemm_force_config",
-    "GEMM_CONFIGS", "plan_launch", "validate", "force_plan", "force_staged",
+    "GEMM_CONFIGS", "allreduce_fused_add_rms_norm", "allreduce_fused_add_rms_norm_fp8",
+    "RnAllreduceComm", "ALLREDUCE_MAX_WORLD", "ALLREDUCE_SIGNAL_BYTES", "plan_launch", "validate", "force_plan", "force_staged",
     "set_launch_options", "device_errors", "supported_vectors_per_thread", "status_string",
     "LIB_PATH", "lib", "RnTensor", "RnPlan", "STATUS", "OPS",
 ]
@@ -35,12 +36,29 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "librmsnorm_
 STATUS = {
     0: "RN_OK", 1: "RN_ERR_NULL", 2: "RN_ERR_DTYPE", 3: "RN_ERR_WEIGHT_DTYPE", 4: "RN_ERR_SHAPE",
     5: "RN_ERR_LAYOUT", 6: "RN_ERR_ALIAS", 7: "RN_ERR_VARIANCE_SIZE", 8: "RN_ERR_EPS",
-    9: "RN_ERR_CUDA", 10: "RN_ERR_CONFIG",
+    9: "RN_ERR_CUDA", 10: "RN_ERR_CONFIG", 11: "RN_ERR_COMM",
 }
 OPS = {"rms_norm": 0, "fused_add_rms_norm": 1, "fused_add_rms_norm_fp8": 2}
 PLAN_OPS = dict(OPS, silu_and_mul_fp8=3)
 _DTYPES = {torch.float16: 0, torch.bfloat16: 1, torch.float8_e4m3fn: 2, torch.float32: 3,
            torch.uint8: 2}
+
+
+ALLREDUCE_MAX_WORLD = 8
+ALLREDUCE_SIGNAL_BYTES = 65600
+
+
+class RnAllreduceComm(ctypes.Structure):
+    """rn_allreduce_comm (include/rmsnorm_b200.h)."""
+    _fields_ = [
+        ("world", ctypes.c_int32),
+        ("rank", ctypes.c_int32),
+        ("local_ranks", ctypes.c_int32),
+        ("buffers", ctypes.c_void_p * ALLREDUCE_MAX_WORLD),
+        ("signals", ctypes.c_void_p * ALLREDUCE_MAX_WORLD),
+        ("buffer_bytes", ctypes.c_int64),
+        ("timeout_ns", ctypes.c_int64),
+    ]
 
 
 class RnTensor(ctypes.Structure):
@@ -94,6 +112,11 @@ def _load():
     L.rn_silu_and_mul_fp8.restype = ctypes.c_int
     L.rn_fp8_rowwise_gemm.argtypes = [P, P, P, P, P, VP]
     L.rn_fp8_rowwise_gemm.restype = ctypes.c_int
+    C = ctypes.POINTER(RnAllreduceComm)
+    L.rn_allreduce_fused_add_rms_norm.argtypes = [P, P, P, P, F, C, VP]
+    L.rn_allreduce_fused_add_rms_norm_fp8.argtypes = [P, P, P, P, P, F, C, VP]
+    L.rn_allreduce_fused_add_rms_norm.restype = ctypes.c_int
+    L.rn_allreduce_fused_add_rms_norm_fp8.restype = ctypes.c_int
     L.rn_fp8_gemm_config.argtypes = [I64, I64, I64, ctypes.c_int32, ctypes.POINTER(ctypes.c_int32)]
     L.rn_fp8_gemm_config.restype = ctypes.c_int
     L.rn_fp8_gemm_force_config.argtypes = [ctypes.c_int32]
@@ -252,6 +275,32 @@ def fp8_rowwise_gemm(d: torch.Tensor, a: torch.Tensor, b: torch.Tensor, a_scale:
     st = _call(lib.rn_fp8_rowwise_gemm, dev, _desc(d, 0), _desc(a, 1), _desc(b, 2),
                _desc(a_scale, 3), _desc(b_scale, 4), s)
     _check(st, "rn_fp8_rowwise_gemm")
+
+
+def allreduce_fused_add_rms_norm(out: torch.Tensor, x: torch.Tensor, residual: torch.Tensor,
+                                 weight: torch.Tensor | None, eps: float, comm,
+                                 stream=None) -> None:
+    """Tensor-parallel all-reduce of the partials x across the group of
+    `comm` (an ``allreduce.AllReduceComm``), then the fused residual add and
+    RMSNorm (C ABI rn_allreduce_fused_add_rms_norm). With comm.local_ranks > 1
+    the operands carry a leading rank dimension."""
+    dev, s = _stream_for((out, x, residual, weight), stream)
+    st = _call(lib.rn_allreduce_fused_add_rms_norm, dev, _desc(out, 0), _desc(x, 1),
+               _desc(residual, 2), None if weight is None else _desc(weight, 3), eps,
+               comm.descriptor_ref(), s)
+    _check(st, "rn_allreduce_fused_add_rms_norm")
+
+
+def allreduce_fused_add_rms_norm_fp8(q: torch.Tensor, scale: torch.Tensor, x: torch.Tensor,
+                                     residual: torch.Tensor, weight: torch.Tensor | None,
+                                     eps: float, comm, stream=None) -> None:
+    """As allreduce_fused_add_rms_norm, with the per-token e4m3 output of
+    fused_add_rms_norm_fp8 (C ABI rn_allreduce_fused_add_rms_norm_fp8)."""
+    dev, s = _stream_for((q, scale, x, residual, weight), stream)
+    st = _call(lib.rn_allreduce_fused_add_rms_norm_fp8, dev, _desc(q, 0), _desc(scale, 1),
+               _desc(x, 2), _desc(residual, 3), None if weight is None else _desc(weight, 4),
+               eps, comm.descriptor_ref(), s)
+    _check(st, "rn_allreduce_fused_add_rms_norm_fp8")
 
 
 # rn_gemm_config values: TOK = token-major (tokens x channels) tiles, CH =

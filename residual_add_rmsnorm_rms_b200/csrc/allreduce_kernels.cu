@@ -1,0 +1,381 @@
+// allreduce_kernels.cu -- tensor-parallel all-reduce fused with the residual
+// add and RMSNorm (+ per-token FP8 cast), one kernel per call.
+//
+// In a tensor-parallel decoder layer every rank ends its row-parallel linear
+// layer with a partial sum of the activations; an all-reduce adds the W
+// partials and the residual add + RMSNorm follows (SGLang takes all-reduce and
+// RMSNorm from AITER: "AITER: AMD's operator library for ROCm", ecosystem
+// section). Here each rank computes, for every row,
+//   x = RNE16(sum over ranks of the partials),  residual := RNE16(x + residual),
+//   out = RNE16(rms_norm(residual) * w)   or   (q, scale) as fused_add_rms_norm_fp8,
+// identically on every rank (the residual is replicated across the group).
+//
+// One-shot exchange over peer memory (NVLink / NVSwitch loads; no collective
+// library, no multicast): every rank owns an exchange buffer and a signal pad
+// that all ranks can address. The pad starts with this rank's call counter
+// (the epoch of its last call) and an arrival counter, then the flags. Block
+// b of every rank owns the same rows; in call e (= counter + 1, 0 skipped):
+//  1. it copies its rows of the local partial into its own buffer (the half
+//     selected by e's parity),
+//  2. publishes them: a system-scope fence, then e is stored with release
+//     semantics into flag [e & 1][b][rank] of every rank's pad,
+//  3. waits (bounded by timeout_ns on the global timer) until flag
+//     [e & 1][b][p] of its own pad equals e, for every rank p,
+//  4. reads the rows from all W buffers (volatile 16-byte loads: never a stale
+//     L1 line), sums them in rank order 0..W-1 and finishes the row exactly
+//     as fused_add_rms_norm(_fp8) does (same 8-element arithmetic),
+//  5. counts itself in the arrival counter; the last block of the rank to
+//     arrive resets it and stores e as the call counter for the next launch.
+// The counter lives on the device, so a captured CUDA graph replays correctly
+// (each replayed launch takes the next epoch). A rank overwrites a buffer
+// half, or a flag, only two calls after it last wrote it: by then every peer
+// has finished reading the half and has seen the flag, because a peer
+// publishes call e+1 only after its call e kernel completed (stream order)
+// and each rank waits for all peers' call e+1 flags before starting call e+2.
+// So the flags are compared for equality and never need resetting. Every
+// call launches, even with no rows (one block then only publishes and waits),
+// so all ranks' counters advance together for any sequence of row counts.
+// The grid is the same on every rank and fully resident (cooperative launch),
+// so no block waits for a block that cannot run. Several ranks may be driven
+// by one launch (blockIdx.y = rank - first rank, operands stacked by rank),
+// which runs a whole group on one device.
+//
+// The sum is accumulated in binary64 in rank order, converted to binary32 by
+// rounding to odd (toward zero, then the last bit set if anything was
+// dropped) and rounded once to the 16-bit format. Rounding to odd with at
+// least two more bits than the target makes the second rounding correct
+// (Boldo and Melquiond, "When double rounding is odd", 2005), so x is the
+// correctly rounded sum whenever the binary64 sum is exact: always for fp16
+// partials (every fp16 value is an integer multiple of 2^-24 below 2^16), and
+// for bf16 partials whose non-zero values span at most 42 binades (W <= 8
+// values then fit 53 bits). Every rank computes bit-identical results.
+//
+// A wait that runs out sets bit 1 of the device error flags and leaves that
+// block's rows unwritten (the other blocks are unaffected); the block still
+// counts its arrival, so the rank's call counter advances.
+#include <cuda_bf16.h>
+#include <cuda_fp16.h>
+
+#include <cstdint>
+
+#include "rn_device.cuh"
+#include "rn_internal.h"
+#include "rn_vec8.cuh"
+
+namespace rn {
+namespace {
+
+__device__ unsigned int g_rn_ar_error = 0;
+constexpr unsigned kErrPeerTimeout = 2u;
+
+// Signal pad layout, in 32-bit words: the call counter, the arrival counter,
+// padding to 64 bytes, then flags [2][kArMaxBlocks][kArMaxWorld].
+constexpr int kPadEpoch = 0;
+constexpr int kPadArrived = 1;
+constexpr int kPadFlags = 16;
+static_assert((kPadFlags + 2 * kArMaxBlocks * kArMaxWorld) * 4 == kArSignalBytes,
+              "signal pad size");
+
+__device__ __forceinline__ uint4 ld_volatile_v4(const uint4* p) {
+    uint4 v;
+    asm volatile("ld.volatile.global.v4.u32 {%0, %1, %2, %3}, [%4];"
+                 : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+                 : "l"(p)
+                 : "memory");
+    return v;
+}
+
+__device__ __forceinline__ void st_release_sys(uint32_t* p, uint32_t v) {
+    asm volatile("st.release.sys.global.u32 [%0], %1;" ::"l"(p), "r"(v) : "memory");
+}
+
+__device__ __forceinline__ uint32_t ld_acquire_sys(const uint32_t* p) {
+    uint32_t v;
+    asm volatile("ld.acquire.sys.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+    return v;
+}
+
+__device__ __forceinline__ unsigned long long global_ns() {
+    unsigned long long t;
+    asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+    return t;
+}
+
+// Rounds to odd at binary32 precision: toward zero, then the last significand
+// bit set when the conversion dropped anything. NaN stays NaN; a finite value
+// beyond the binary32 range becomes the largest finite binary32 with its last
+// bit set, which every 16-bit format then rounds to infinity.
+__device__ __forceinline__ float round_to_odd_f32(double s) {
+    float f = __double2float_rz(s);
+    if (static_cast<double>(f) != s) f = __uint_as_float(__float_as_uint(f) | 1u);
+    return f;
+}
+
+// RNE16 of the rank-order binary64 sum of 8 elements of W partials.
+template <typename T>
+__device__ __forceinline__ uint4 sum8(const uint4 (&pv)[kArMaxWorld], int W) {
+    uint4 o;
+    uint32_t* os = &o.x;
+#pragma unroll
+    for (int c = 0; c < 4; ++c) {
+        const float2 f0 = Fmt<T>::unpack((&pv[0].x)[c]);
+        double sx = f0.x, sy = f0.y;  // start from rank 0: keeps -0 + -0 = -0
+#pragma unroll
+        for (int p = 1; p < kArMaxWorld; ++p) {
+            if (p < W) {
+                const float2 f = Fmt<T>::unpack((&pv[p].x)[c]);
+                sx += static_cast<double>(f.x);
+                sy += static_cast<double>(f.y);
+            }
+        }
+        os[c] = Fmt<T>::pack(make_float2(round_to_odd_f32(sx), round_to_odd_f32(sy)));
+    }
+    return o;
+}
+
+// Step 4 for the rows of this block: reduce + residual add + RMSNorm (+ FP8),
+// rows mapped as in the vector kernel.
+template <typename T, int VPT, bool kFp8, bool kHasW>
+__device__ __forceinline__ void reduce_rows(const ArArgs& a, const int tpr, const int rpc,
+                                            float2* red, const int ly, const uint32_t epoch,
+                                            const int nvec, const int64_t local) {
+    const int W = a.world;
+    const int64_t slot = static_cast<int64_t>(epoch & 1u) * (a.slot_elems >> 3);
+    const uint4* __restrict__ wv = static_cast<const uint4*>(a.weight);
+    const float hf = static_cast<float>(a.H);
+    const uint4* peer[kArMaxWorld];
+#pragma unroll
+    for (int p = 0; p < kArMaxWorld; ++p)
+        peer[p] = static_cast<const uint4*>(a.buffers[p < W ? p : 0]) + slot;
+    const int row_in_cta = threadIdx.x / tpr;
+    const int lr = threadIdx.x - row_in_cta * tpr;
+    const int wpr = tpr >> 5;
+    int parity = 0;
+    for (int64_t base = static_cast<int64_t>(blockIdx.x) * rpc; base < a.T;
+         base += static_cast<int64_t>(gridDim.x) * rpc) {
+        const int64_t row = base + row_in_cta;
+        const bool active = row < a.T;
+        const int64_t roff = (active ? row : 0) * nvec;
+        uint4* rrow = static_cast<uint4*>(a.residual) + local + roff;
+
+        uint4 v[VPT];
+#pragma unroll
+        for (int k = 0; k < VPT; ++k) {
+            const int j = lr + k * tpr;
+            if (active && j < nvec) {
+                uint4 pv[kArMaxWorld];
+#pragma unroll
+                for (int p = 0; p < kArMaxWorld; ++p)
+                    pv[p] = p < W ? ld_volatile_v4(peer[p] + roff + j) : make_uint4(0, 0, 0, 0);
+                v[k] = sum8<T>(pv, W);
+            } else {
+                v[k] = make_uint4(0, 0, 0, 0);
+            }
+        }
+        uint4 r[VPT];
+#pragma unroll
+        for (int k = 0; k < VPT; ++k) {
+            const int j = lr + k * tpr;
+            r[k] = (active && j < nvec) ? ld_stream(rrow + j) : make_uint4(0, 0, 0, 0);
+        }
+        float2 acc = make_float2(0.f, 0.f);
+        float pm = 0.f;
+#pragma unroll
+        for (int k = 0; k < VPT; ++k) {
+            const int j = lr + k * tpr;
+            v[k] = add8<T>(v[k], r[k]);
+            if (active && j < nvec) st_v4(rrow + j, v[k]);
+            acc = ssq8<T>(v[k], acc);
+            if constexpr (kFp8) {
+                uint4 w = make_uint4(0, 0, 0, 0);
+                if constexpr (kHasW) {
+                    if (j < nvec) w = __ldg(wv + j);
+                }
+                pm = amax8<T, kHasW>(v[k], w, pm);
+            }
+        }
+        float ss = acc.x + acc.y;
+        const int width = tpr < 32 ? tpr : 32;
+        for (int o = width >> 1; o > 0; o >>= 1) {
+            ss += __shfl_xor_sync(0xffffffffu, ss, o);
+            if constexpr (kFp8) pm = fmaxf(pm, __shfl_xor_sync(0xffffffffu, pm, o));
+        }
+        if (wpr > 1) {
+            float2* s2 = red + (parity * rpc + row_in_cta) * wpr;
+            if ((lr & 31) == 0) s2[lr >> 5] = make_float2(ss, pm);
+            group_barrier(1 + row_in_cta, tpr);
+            float s = 0.f, m = 0.f;
+            for (int i = 0; i < wpr; ++i) {
+                const float2 t = s2[i];
+                s += t.x;
+                m = fmaxf(m, t.y);
+            }
+            ss = s;
+            pm = m;
+            parity ^= 1;
+        }
+        const float inv = 1.0f / sqrtf(ss / hf + a.eps);
+
+        if constexpr (!kFp8) {
+            uint4* orow = static_cast<uint4*>(a.out) + local + roff;
+            const float2 inv2 = make_float2(inv, inv);
+#pragma unroll
+            for (int k = 0; k < VPT; ++k) {
+                const int j = lr + k * tpr;
+                if (!(active && j < nvec)) continue;
+                uint4 w = make_uint4(0, 0, 0, 0);
+                if constexpr (kHasW) w = __ldg(wv + j);
+                st_v4(orow + j, scale8<T, kHasW>(v[k], w, inv2));
+            }
+        } else {
+            const float qmul = pm > 0.f ? 448.0f / pm : 0.f;
+            const float2 q2 = make_float2(qmul, qmul);
+            if (active && lr == 0)
+                a.scale[static_cast<int64_t>(ly) * a.T + row] = pm > 0.f ? (pm * inv) / 448.0f : 0.f;
+            uint2* qrow = reinterpret_cast<uint2*>(a.q) + local + roff;
+#pragma unroll
+            for (int k = 0; k < VPT; ++k) {
+                const int j = lr + k * tpr;
+                if (!(active && j < nvec)) continue;
+                uint4 w = make_uint4(0, 0, 0, 0);
+                if constexpr (kHasW) w = __ldg(wv + j);
+                uint2 o = quant8<T, kHasW>(v[k], w, q2);
+                if (!(pm > 0.f)) o = make_uint2(0, 0);
+                st_v2(qrow + j, o);
+            }
+        }
+    }
+}
+
+template <typename T, int VPT, bool kFp8, bool kHasW>
+__device__ __forceinline__ void allreduce_rows(const ArArgs& a, const int tpr, const int rpc,
+                                               float2* red) {
+    const int ly = blockIdx.y;
+    const int rank = a.rank + ly;
+    const int W = a.world;
+    const int nvec = static_cast<int>(a.H >> 3);
+    const int64_t local = static_cast<int64_t>(ly) * a.T * nvec;  // in 16-byte vectors
+    uint32_t* const pad = a.signals[rank];
+    uint32_t epoch = *reinterpret_cast<volatile uint32_t*>(pad + kPadEpoch) + 1u;
+    if (epoch == 0) epoch = 1;
+    const int64_t slot = static_cast<int64_t>(epoch & 1u) * (a.slot_elems >> 3);
+
+    // 1. this block's rows of the local partial into this rank's buffer
+    {
+        const uint4* x = static_cast<const uint4*>(a.x) + local;
+        uint4* mine = static_cast<uint4*>(a.buffers[rank]) + slot;
+        for (int64_t base = static_cast<int64_t>(blockIdx.x) * rpc; base < a.T;
+             base += static_cast<int64_t>(gridDim.x) * rpc) {
+            const int64_t v0 = base * nvec;
+            const int64_t v1 = (base + rpc < a.T ? base + rpc : a.T) * nvec;
+            for (int64_t i = v0 + threadIdx.x; i < v1; i += blockDim.x) st_v4(mine + i, ld_stream(x + i));
+        }
+    }
+    __syncthreads();
+
+    // 2. publish, 3. wait for every rank's copy of the same rows
+    const int flag0 = kPadFlags + ((epoch & 1u) * kArMaxBlocks + blockIdx.x) * kArMaxWorld;
+    if (threadIdx.x == 0) {
+        __threadfence_system();
+        for (int p = 0; p < W; ++p) st_release_sys(a.signals[p] + flag0 + rank, epoch);
+    }
+    bool late = false;
+    if (threadIdx.x < W) {
+        const uint32_t* f = pad + flag0 + threadIdx.x;
+        if (ld_acquire_sys(f) != epoch) {
+            const unsigned long long t0 = global_ns();
+            while (ld_acquire_sys(f) != epoch) {
+                if (global_ns() - t0 > static_cast<unsigned long long>(a.timeout_ns)) {
+                    late = true;
+                    break;
+                }
+                __nanosleep(64);
+            }
+        }
+    }
+    if (__syncthreads_or(late)) {
+        if (threadIdx.x == 0) atomicOr(&g_rn_ar_error, kErrPeerTimeout);
+    } else {
+        reduce_rows<T, VPT, kFp8, kHasW>(a, tpr, rpc, red, ly, epoch, nvec, local);
+    }
+
+    // 5. arrival; the last block of this rank advances the call counter
+    __syncthreads();
+    if (threadIdx.x == 0) {
+        __threadfence();
+        if (atomicAdd(pad + kPadArrived, 1u) == gridDim.x - 1) {
+            atomicExch(pad + kPadArrived, 0u);
+            atomicExch(pad + kPadEpoch, epoch);
+        }
+    }
+}
+
+template <typename T, int VPT, bool kFp8>
+__global__ void __launch_bounds__(kArMaxBlock)
+    rn_allreduce_kernel(const ArArgs a, const int tpr, const int rpc) {
+    extern __shared__ float2 red[];  // [2][rpc][warps per row]
+    if (a.weight)
+        allreduce_rows<T, VPT, kFp8, true>(a, tpr, rpc, red);
+    else
+        allreduce_rows<T, VPT, kFp8, false>(a, tpr, rpc, red);
+}
+
+using ArKernel = void (*)(const ArArgs, const int, const int);
+
+template <typename T, bool kFp8>
+ArKernel pick_vpt(int vpt) {
+    switch (vpt) {
+        case 1: return rn_allreduce_kernel<T, 1, kFp8>;
+        case 2: return rn_allreduce_kernel<T, 2, kFp8>;
+        case 4: return rn_allreduce_kernel<T, 4, kFp8>;
+        case 8: return rn_allreduce_kernel<T, 8, kFp8>;
+        default: return nullptr;
+    }
+}
+
+ArKernel pick(int dtype, bool fp8, int vpt) {
+    if (dtype == kBF16)
+        return fp8 ? pick_vpt<__nv_bfloat16, true>(vpt) : pick_vpt<__nv_bfloat16, false>(vpt);
+    if (dtype == kF16) return fp8 ? pick_vpt<__half, true>(vpt) : pick_vpt<__half, false>(vpt);
+    return nullptr;
+}
+
+}  // namespace
+
+cudaError_t allreduce_blocks_per_sm(int dtype, bool fp8, const ArLaunch& l, int* blocks) {
+    const ArKernel k = pick(dtype, fp8, l.vpt);
+    if (!k) return cudaErrorInvalidValue;
+    return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks, k, l.block,
+                                                         static_cast<size_t>(l.smem));
+}
+
+cudaError_t launch_allreduce(int dtype, bool fp8, const ArArgs& a, const ArLaunch& l,
+                             cudaStream_t s) {
+    const ArKernel k = pick(dtype, fp8, l.vpt);
+    if (!k) return cudaErrorInvalidValue;
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(l.grid_x), static_cast<unsigned>(l.local_ranks));
+    cfg.blockDim = dim3(static_cast<unsigned>(l.block));
+    cfg.dynamicSmemBytes = static_cast<size_t>(l.smem);
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeCooperative;
+    attr[0].val.cooperative = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cudaLaunchKernelEx(&cfg, k, a, l.tpr, l.rpc);
+}
+
+cudaError_t read_and_clear_allreduce_errors(unsigned* flags) {
+    unsigned v = 0;
+    cudaError_t e = cudaMemcpyFromSymbol(&v, g_rn_ar_error, sizeof v);
+    if (e != cudaSuccess) return e;
+    *flags = v;
+    if (v) {
+        const unsigned zero = 0;
+        e = cudaMemcpyToSymbol(g_rn_ar_error, &zero, sizeof zero);
+    }
+    return e;
+}
+
+}  // namespace rn

@@ -610,6 +610,148 @@ rn_status rn_fp8_rowwise_gemm(const rn_tensor* d, const rn_tensor* a, const rn_t
     return RN_OK;
 }
 
+// ---- tensor-parallel all-reduce fused ops
+
+}  // extern "C"
+
+namespace {
+
+constexpr long long kArDefaultTimeoutNs = 1000000000LL;  // 1 s
+constexpr int64_t kArMaxH = static_cast<int64_t>(rn::kArMaxBlock) * 8 * 8;
+
+bool overlaps_bytes(const Flat& f, const void* p, int64_t bytes) {
+    if (!f.ptr || f.numel == 0 || !p || bytes <= 0) return false;
+    const auto a0 = reinterpret_cast<uintptr_t>(f.ptr);
+    const auto a1 = a0 + static_cast<uintptr_t>(f.bytes());
+    const auto b0 = reinterpret_cast<uintptr_t>(p);
+    const auto b1 = b0 + static_cast<uintptr_t>(bytes);
+    return a0 < b1 && b0 < a1;
+}
+
+// Row mapping of the all-reduce kernel: the smallest power-of-two group of
+// threads that covers a row with at most 4 vectors each (8 once the group
+// reaches the block limit), 256-thread blocks of several rows for narrow rows.
+rn_status ar_shape(int64_t H, rn::ArLaunch* l) {
+    const int64_t nvec = H / 8;
+    int tpr = 1;
+    while (static_cast<int64_t>(tpr) * 4 < nvec && tpr < rn::kArMaxBlock) tpr *= 2;
+    const int64_t need = (nvec + tpr - 1) / tpr;
+    int vpt = 1;
+    while (vpt < need) vpt *= 2;
+    if (vpt > 8) return RN_ERR_SHAPE;
+    l->tpr = tpr;
+    l->vpt = vpt;
+    l->rpc = tpr >= 256 ? 1 : 256 / tpr;
+    l->block = tpr * l->rpc;
+    l->smem = static_cast<int>(2 * l->rpc * (tpr >= 64 ? tpr / 32 : 1) * sizeof(float) * 2);
+    return RN_OK;
+}
+
+static_assert(RN_ALLREDUCE_SIGNAL_BYTES == rn::kArSignalBytes, "signal pad size");
+static_assert(RN_ALLREDUCE_MAX_WORLD == rn::kArMaxWorld, "group size");
+
+rn_status check_comm(const rn_allreduce_comm* comm) {
+    if (comm->world < 1 || comm->world > RN_ALLREDUCE_MAX_WORLD) return RN_ERR_COMM;
+    if (comm->rank < 0 || comm->rank >= comm->world) return RN_ERR_COMM;
+    if (!(comm->local_ranks == 1 || (comm->local_ranks == comm->world && comm->rank == 0)))
+        return RN_ERR_COMM;
+    for (int p = 0; p < comm->world; ++p) {
+        if (!comm->buffers[p] || !comm->signals[p]) return RN_ERR_COMM;
+        if (!aligned(comm->buffers[p], 16) || !aligned(comm->signals[p], 16)) return RN_ERR_COMM;
+    }
+    return RN_OK;
+}
+
+rn_status run_allreduce(bool fp8, const rn_tensor* o, const rn_tensor* sc, const rn_tensor* x,
+                        const rn_tensor* r, const rn_tensor* w, float eps,
+                        const rn_allreduce_comm* comm, void* stream) {
+    const int op = fp8 ? rn::kFusedAddFp8 : rn::kFusedAdd;
+    if (!comm) return RN_ERR_NULL;
+    Common c;
+    rn_status st = check_descriptors(op, o, sc, x, r, w, eps, -1, &c);
+    if (st != RN_OK) return st;
+    if ((st = check_comm(comm)) != RN_OK) return st;
+    const int L = comm->local_ranks;
+    if (c.x.T % L != 0) return RN_ERR_SHAPE;
+    const int64_t T = c.x.T / L, H = c.x.H;
+    if (H % 8 != 0) return RN_ERR_LAYOUT;
+    if (H > kArMaxH) return RN_ERR_SHAPE;
+    const int64_t slot_bytes = (comm->buffer_bytes / 2) & ~static_cast<int64_t>(15);
+    if (comm->buffer_bytes < 0 || slot_bytes < 2 * T * H) return RN_ERR_COMM;
+    rn::ArLaunch l;
+    if ((st = ar_shape(H, &l)) != RN_OK) return st;
+    if (T > 0) {
+        rn_plan unused;
+        if ((st = check_pointers_and_plan(op, c, device_sms(), &unused)) != RN_OK) return st;
+        if (!aligned(c.x.ptr, 16) || !aligned(c.res.ptr, 16) ||
+            (c.has_w && !aligned(c.w.ptr, 16)) || (!fp8 && !aligned(c.out.ptr, 16)) ||
+            (fp8 && !aligned(c.q.ptr, 8)))
+            return RN_ERR_LAYOUT;
+        for (int i = 0; i < L; ++i) {
+            const void* buf = comm->buffers[comm->rank + i];
+            const void* pad = comm->signals[comm->rank + i];
+            for (const Flat* f : {&c.x, &c.res, &c.out, &c.q, &c.scale, &c.w})
+                if (overlaps_bytes(*f, buf, comm->buffer_bytes) ||
+                    overlaps_bytes(*f, pad, rn::kArSignalBytes))
+                    return RN_ERR_ALIAS;
+        }
+    }
+    rn::ArArgs a = {};
+    a.world = comm->world;
+    a.rank = comm->rank;
+    for (int p = 0; p < comm->world; ++p) {
+        a.buffers[p] = comm->buffers[p];
+        a.signals[p] = static_cast<uint32_t*>(comm->signals[p]);
+    }
+    a.slot_elems = slot_bytes / 2;
+    a.timeout_ns = comm->timeout_ns > 0 ? comm->timeout_ns : kArDefaultTimeoutNs;
+    a.x = c.x.ptr;
+    a.residual = c.res.ptr;
+    a.weight = c.has_w ? c.w.ptr : nullptr;
+    a.out = c.out.ptr;
+    a.q = reinterpret_cast<uint8_t*>(c.q.ptr);
+    a.scale = reinterpret_cast<float*>(c.scale.ptr);
+    a.T = T;
+    a.H = H;
+    a.eps = eps;
+    l.local_ranks = L;
+    int per_sm = 0;
+    cudaError_t e = rn::allreduce_blocks_per_sm(c.dt, fp8, l, &per_sm);
+    if (e == cudaSuccess) {
+        const int64_t resident = static_cast<int64_t>(per_sm) * device_sms() / L;
+        const int64_t groups = T > 0 ? (T + l.rpc - 1) / l.rpc : 1;
+        int64_t g = groups < resident ? groups : resident;
+        if (g > rn::kArMaxBlocks) g = rn::kArMaxBlocks;
+        if (g < 1) return RN_ERR_CONFIG;
+        l.grid_x = static_cast<int>(g);
+        e = rn::launch_allreduce(c.dt, fp8, a, l, static_cast<cudaStream_t>(stream));
+    }
+    if (e != cudaSuccess) {
+        std::snprintf(g_cuda_error, sizeof g_cuda_error, "%s: %s", cudaGetErrorName(e),
+                      cudaGetErrorString(e));
+        return RN_ERR_CUDA;
+    }
+    return RN_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+rn_status rn_allreduce_fused_add_rms_norm(const rn_tensor* out, const rn_tensor* x,
+                                          const rn_tensor* residual, const rn_tensor* weight,
+                                          float eps, const rn_allreduce_comm* comm,
+                                          void* stream) {
+    return run_allreduce(false, out, nullptr, x, residual, weight, eps, comm, stream);
+}
+
+rn_status rn_allreduce_fused_add_rms_norm_fp8(const rn_tensor* q, const rn_tensor* scale,
+                                              const rn_tensor* x, const rn_tensor* residual,
+                                              const rn_tensor* weight, float eps,
+                                              const rn_allreduce_comm* comm, void* stream) {
+    return run_allreduce(true, q, scale, x, residual, weight, eps, comm, stream);
+}
+
 rn_status rn_validate(int32_t op, const rn_tensor* out_or_q, const rn_tensor* scale,
                       const rn_tensor* x, const rn_tensor* residual, const rn_tensor* weight,
                       float eps, int64_t variance_size, rn_plan* plan) {
@@ -635,6 +777,7 @@ const char* rn_status_string(rn_status s) {
         case RN_ERR_EPS: return "eps must be finite and >= 0";
         case RN_ERR_CUDA: return "CUDA error (see rn_last_cuda_error)";
         case RN_ERR_CONFIG: return "unsupported launch configuration";
+        case RN_ERR_COMM: return "bad all-reduce group description or exchange buffers too small";
     }
     return "unknown status";
 }
@@ -676,8 +819,10 @@ rn_status rn_set_launch_options(int32_t pdl, int64_t max_grid) {
 
 rn_status rn_device_errors(uint32_t* flags) {
     if (!flags) return RN_ERR_NULL;
-    unsigned v = 0;
-    const cudaError_t e = rn::read_and_clear_device_errors(&v);
+    unsigned v = 0, v_ar = 0;
+    cudaError_t e = rn::read_and_clear_device_errors(&v);
+    if (e == cudaSuccess) e = rn::read_and_clear_allreduce_errors(&v_ar);
+    v |= v_ar;
     if (e != cudaSuccess) {
         std::snprintf(g_cuda_error, sizeof g_cuda_error, "%s: %s", cudaGetErrorName(e),
                       cudaGetErrorString(e));

@@ -30,6 +30,11 @@ Multiplies Run Slower"):
 * ``sweep``    all three ops, bf16 and fp16, T in {1,16,256,4096,32768,65536} x
                H in {2048,4096,5120,7168,8192,16384}, x ~ N(0,1),
                residual ~ N(0,4), eps 1e-6.
+* ``tp``       the tensor-parallel fused ops (``make_tp_inputs``): W ranks'
+               partial sums [W x T x H], each ~ N(0, 1/W) (their sum has the
+               decode workload's N(0,1)), one residual [T x H] ~ N(0,4)
+               replicated on every rank, eps 1e-5; W in {2, 4, 8}, T in
+               {1, 8, 64, 256, 8192}, H 3840 (Gemma 4 12B) and 4096.
 
 Every workload uses weight = 1 + N(0, 0.1) in the activation dtype.
 """
@@ -54,7 +59,10 @@ __all__ = [
     "SWEEP_H",
     "SWIGLU_I",
     "SWIGLU_T",
+    "TP_W",
+    "TP_T",
     "to_dtype",
+    "make_tp_inputs",
 ]
 
 DECODE_T = (1, 8, 64, 256)
@@ -62,6 +70,8 @@ SWEEP_T = (1, 16, 256, 4096, 32768, 65536)
 SWEEP_H = (2048, 4096, 5120, 7168, 8192, 16384)
 SWIGLU_I = 15360
 SWIGLU_T = (1, 8, 64, 256, 8192)
+TP_W = (2, 4, 8)
+TP_T = (1, 8, 64, 256, 8192)
 
 
 def to_dtype(name: str) -> torch.dtype:
@@ -181,3 +191,20 @@ def make_inputs(name: str, op: str, dtype: str, T: int, H: int, device="cpu",
         x=x.to(dt), residual=None if r is None else r.to(dt), weight=w,
         outliers=outl,
     )
+
+
+def make_tp_inputs(dtype: str, W: int, T: int, H: int, device="cpu",
+                   seed: int | None = None) -> Workload:
+    """Inputs of one tensor-parallel cell: ``x`` holds the W partial sums
+    [W x T x H] (each ~ N(0, 1/W)), ``residual`` the replicated residual
+    [T x H] ~ N(0, 4); weight 1 + N(0, 0.1); eps 1e-5."""
+    dt = to_dtype(dtype)
+    device = torch.device(device)
+    if seed is None:
+        seed = cell_seed("tp", dtype, W, T, H)
+    g = _gen(seed, device)
+    x = normal((W, T, H), 1.0 / W, g, device)
+    r = normal((T, H), 4.0, g, device)
+    w = weight(H, dt, g, device)
+    return Workload(name="tp", op="allreduce_fused_add_rms_norm", dtype=dt, T=T, H=H,
+                    eps=1e-5, seed=seed, x=x.to(dt), residual=r.to(dt), weight=w)

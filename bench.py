@@ -642,11 +642,13 @@ def time_gemm_cell(rn, M, N, K, iters, device, configs=(None,)):
 
 
 def tp_bytes(fp8: bool, W: int, T: int, H: int) -> int:
-    """Unique bytes one single-device group call moves: per rank and row, the
-    partial read (2H), its copy into the exchange buffer (2H), one read of
-    that buffer (2H: each buffer is read by all W ranks, counted once), the
-    residual read and write (4H) and the output (2H, or H codes + 4)."""
-    return W * T * ((11 * H + 4) if fp8 else 12 * H)
+    """Bytes one single-device group call moves, per rank and row: the
+    partial read (2H), its copy into the exchange buffer (2H), the reads of
+    all W exchange buffers (2WH: every rank reads every buffer; W buffers of
+    a large call do not stay in L2 together), the residual read and write
+    (4H) and the output (2H, or H codes + a 4-byte scale)."""
+    per_row = (9 + 2 * W) * H + 4 if fp8 else (10 + 2 * W) * H
+    return W * T * per_row
 
 
 def time_tp_cell(rn, fp8, W, T, H, iters, device):

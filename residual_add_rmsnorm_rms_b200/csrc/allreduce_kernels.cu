@@ -17,8 +17,8 @@
 // b of every rank owns the same rows; in call e (= counter + 1, 0 skipped):
 //  1. it copies its rows of the local partial into its own buffer (the half
 //     selected by e's parity),
-//  2. publishes them: a system-scope fence, then e is stored with release
-//     semantics into flag [e & 1][b][rank] of every rank's pad,
+//  2. publishes them: e is stored with system-scope release semantics into
+//     flag [e & 1][b][rank] of every rank's pad,
 //  3. waits (bounded by timeout_ns on the global timer) until flag
 //     [e & 1][b][p] of its own pad equals e, for every rank p,
 //  4. reads the rows from all W buffers (volatile 16-byte loads: never a stale
@@ -35,14 +35,19 @@
 // So the flags are compared for equality and never need resetting. Every
 // call launches, even with no rows (one block then only publishes and waits),
 // so all ranks' counters advance together for any sequence of row counts.
-// The grid is the same on every rank and fully resident (cooperative launch),
-// so no block waits for a block that cannot run. Several ranks may be driven
-// by one launch (blockIdx.y = rank - first rank, operands stacked by rank),
-// which runs a whole group on one device.
+// The grid is the same on every rank and no larger than what the device
+// holds resident, and blocks are dispatched in index order, so the blocks
+// resident on every rank always include the lowest-numbered blocks still
+// waiting, which can therefore finish: no block waits on a block that cannot
+// run (the bounded wait guards the rest). Several ranks may be driven by one
+// launch (blockIdx.y = rank - first rank, operands stacked by rank), which
+// runs a whole group on one device; blocks of one launch then wait on one
+// another, so that launch is cooperative (every block resident).
 //
-// The sum is accumulated in binary64 in rank order, converted to binary32 by
-// rounding to odd (toward zero, then the last bit set if anything was
-// dropped) and rounded once to the 16-bit format. Rounding to odd with at
+// With two ranks the sum is one packed 16-bit add (correctly rounded, as the
+// residual add). With more, it is accumulated in binary64 in rank order,
+// converted to binary32 by rounding to odd (toward zero, then the last bit
+// set if anything was dropped) and rounded once to the 16-bit format. Rounding to odd with at
 // least two more bits than the target makes the second rounding correct
 // (Boldo and Melquiond, "When double rounding is odd", 2005), so x is the
 // correctly rounded sum whenever the binary64 sum is exact: always for fp16
@@ -60,6 +65,7 @@
 
 #include "rn_device.cuh"
 #include "rn_internal.h"
+#include "rn_allreduce.h"
 #include "rn_vec8.cuh"
 
 namespace rn {
@@ -111,31 +117,41 @@ __device__ __forceinline__ float round_to_odd_f32(double s) {
     return f;
 }
 
-// RNE16 of the rank-order binary64 sum of 8 elements of W partials.
-template <typename T>
-__device__ __forceinline__ uint4 sum8(const uint4 (&pv)[kArMaxWorld], int W) {
-    uint4 o;
-    uint32_t* os = &o.x;
+// RNE16 of the sum over the ranks of 8 elements: kW is the group size
+// rounded up to 1, 2, 4 or 8 (W of them present). One rank: the value itself.
+// Two ranks: the packed 16-bit add, which rounds the exact sum once (as the
+// residual add does). More: the rank-order binary64 sum, rounded to odd at
+// binary32, then to nearest even at 16 bits.
+template <typename T, int kW>
+__device__ __forceinline__ uint4 sum8(const uint4 (&pv)[kW], int W) {
+    if constexpr (kW == 1) {
+        return pv[0];
+    } else if constexpr (kW == 2) {
+        return add8<T>(pv[0], pv[1]);
+    } else {
+        uint4 o;
+        uint32_t* os = &o.x;
 #pragma unroll
-    for (int c = 0; c < 4; ++c) {
-        const float2 f0 = Fmt<T>::unpack((&pv[0].x)[c]);
-        double sx = f0.x, sy = f0.y;  // start from rank 0: keeps -0 + -0 = -0
+        for (int c = 0; c < 4; ++c) {
+            const float2 f0 = Fmt<T>::unpack((&pv[0].x)[c]);
+            double sx = f0.x, sy = f0.y;  // start from rank 0: keeps -0 + -0 = -0
 #pragma unroll
-        for (int p = 1; p < kArMaxWorld; ++p) {
-            if (p < W) {
-                const float2 f = Fmt<T>::unpack((&pv[p].x)[c]);
-                sx += static_cast<double>(f.x);
-                sy += static_cast<double>(f.y);
+            for (int p = 1; p < kW; ++p) {
+                if (p < W) {
+                    const float2 f = Fmt<T>::unpack((&pv[p].x)[c]);
+                    sx += static_cast<double>(f.x);
+                    sy += static_cast<double>(f.y);
+                }
             }
+            os[c] = Fmt<T>::pack(make_float2(round_to_odd_f32(sx), round_to_odd_f32(sy)));
         }
-        os[c] = Fmt<T>::pack(make_float2(round_to_odd_f32(sx), round_to_odd_f32(sy)));
+        return o;
     }
-    return o;
 }
 
 // Step 4 for the rows of this block: reduce + residual add + RMSNorm (+ FP8),
 // rows mapped as in the vector kernel.
-template <typename T, int VPT, bool kFp8, bool kHasW>
+template <typename T, int VPT, int kW, bool kFp8, bool kHasW>
 __device__ __forceinline__ void reduce_rows(const ArArgs& a, const int tpr, const int rpc,
                                             float2* red, const int ly, const uint32_t epoch,
                                             const int nvec, const int64_t local) {
@@ -143,9 +159,9 @@ __device__ __forceinline__ void reduce_rows(const ArArgs& a, const int tpr, cons
     const int64_t slot = static_cast<int64_t>(epoch & 1u) * (a.slot_elems >> 3);
     const uint4* __restrict__ wv = static_cast<const uint4*>(a.weight);
     const float hf = static_cast<float>(a.H);
-    const uint4* peer[kArMaxWorld];
+    const uint4* peer[kW];
 #pragma unroll
-    for (int p = 0; p < kArMaxWorld; ++p)
+    for (int p = 0; p < kW; ++p)
         peer[p] = static_cast<const uint4*>(a.buffers[p < W ? p : 0]) + slot;
     const int row_in_cta = threadIdx.x / tpr;
     const int lr = threadIdx.x - row_in_cta * tpr;
@@ -158,25 +174,25 @@ __device__ __forceinline__ void reduce_rows(const ArArgs& a, const int tpr, cons
         const int64_t roff = (active ? row : 0) * nvec;
         uint4* rrow = static_cast<uint4*>(a.residual) + local + roff;
 
+        uint4 r[VPT];  // residual loads first: in flight during the exchange reads
+#pragma unroll
+        for (int k = 0; k < VPT; ++k) {
+            const int j = lr + k * tpr;
+            r[k] = (active && j < nvec) ? ld_stream(rrow + j) : make_uint4(0, 0, 0, 0);
+        }
         uint4 v[VPT];
 #pragma unroll
         for (int k = 0; k < VPT; ++k) {
             const int j = lr + k * tpr;
             if (active && j < nvec) {
-                uint4 pv[kArMaxWorld];
+                uint4 pv[kW];
 #pragma unroll
-                for (int p = 0; p < kArMaxWorld; ++p)
+                for (int p = 0; p < kW; ++p)
                     pv[p] = p < W ? ld_volatile_v4(peer[p] + roff + j) : make_uint4(0, 0, 0, 0);
-                v[k] = sum8<T>(pv, W);
+                v[k] = sum8<T, kW>(pv, W);
             } else {
                 v[k] = make_uint4(0, 0, 0, 0);
             }
-        }
-        uint4 r[VPT];
-#pragma unroll
-        for (int k = 0; k < VPT; ++k) {
-            const int j = lr + k * tpr;
-            r[k] = (active && j < nvec) ? ld_stream(rrow + j) : make_uint4(0, 0, 0, 0);
         }
         float2 acc = make_float2(0.f, 0.f);
         float pm = 0.f;
@@ -247,7 +263,7 @@ __device__ __forceinline__ void reduce_rows(const ArArgs& a, const int tpr, cons
     }
 }
 
-template <typename T, int VPT, bool kFp8, bool kHasW>
+template <typename T, int VPT, int kW, bool kFp8, bool kHasW>
 __device__ __forceinline__ void allreduce_rows(const ArArgs& a, const int tpr, const int rpc,
                                                float2* red) {
     const int ly = blockIdx.y;
@@ -268,6 +284,7 @@ __device__ __forceinline__ void allreduce_rows(const ArArgs& a, const int tpr, c
              base += static_cast<int64_t>(gridDim.x) * rpc) {
             const int64_t v0 = base * nvec;
             const int64_t v1 = (base + rpc < a.T ? base + rpc : a.T) * nvec;
+#pragma unroll 4
             for (int64_t i = v0 + threadIdx.x; i < v1; i += blockDim.x) st_v4(mine + i, ld_stream(x + i));
         }
     }
@@ -275,10 +292,11 @@ __device__ __forceinline__ void allreduce_rows(const ArArgs& a, const int tpr, c
 
     // 2. publish, 3. wait for every rank's copy of the same rows
     const int flag0 = kPadFlags + ((epoch & 1u) * kArMaxBlocks + blockIdx.x) * kArMaxWorld;
-    if (threadIdx.x == 0) {
-        __threadfence_system();
-        for (int p = 0; p < W; ++p) st_release_sys(a.signals[p] + flag0 + rank, epoch);
-    }
+    // The barrier above orders every thread's copy before the release
+    // stores, and a system-scope release orders everything that happens
+    // before it: no separate fence is needed. Thread p publishes to rank p,
+    // so the W releases proceed in parallel.
+    if (threadIdx.x < W) st_release_sys(a.signals[threadIdx.x] + flag0 + rank, epoch);
     bool late = false;
     if (threadIdx.x < W) {
         const uint32_t* f = pad + flag0 + threadIdx.x;
@@ -296,7 +314,7 @@ __device__ __forceinline__ void allreduce_rows(const ArArgs& a, const int tpr, c
     if (__syncthreads_or(late)) {
         if (threadIdx.x == 0) atomicOr(&g_rn_ar_error, kErrPeerTimeout);
     } else {
-        reduce_rows<T, VPT, kFp8, kHasW>(a, tpr, rpc, red, ly, epoch, nvec, local);
+        reduce_rows<T, VPT, kW, kFp8, kHasW>(a, tpr, rpc, red, ly, epoch, nvec, local);
     }
 
     // 5. arrival; the last block of this rank advances the call counter
@@ -310,40 +328,52 @@ __device__ __forceinline__ void allreduce_rows(const ArArgs& a, const int tpr, c
     }
 }
 
-template <typename T, int VPT, bool kFp8>
+template <typename T, int VPT, int kW, bool kFp8>
 __global__ void __launch_bounds__(kArMaxBlock)
     rn_allreduce_kernel(const ArArgs a, const int tpr, const int rpc) {
     extern __shared__ float2 red[];  // [2][rpc][warps per row]
     if (a.weight)
-        allreduce_rows<T, VPT, kFp8, true>(a, tpr, rpc, red);
+        allreduce_rows<T, VPT, kW, kFp8, true>(a, tpr, rpc, red);
     else
-        allreduce_rows<T, VPT, kFp8, false>(a, tpr, rpc, red);
+        allreduce_rows<T, VPT, kW, kFp8, false>(a, tpr, rpc, red);
 }
 
 using ArKernel = void (*)(const ArArgs, const int, const int);
 
-template <typename T, bool kFp8>
+template <typename T, int kW, bool kFp8>
 ArKernel pick_vpt(int vpt) {
     switch (vpt) {
-        case 1: return rn_allreduce_kernel<T, 1, kFp8>;
-        case 2: return rn_allreduce_kernel<T, 2, kFp8>;
-        case 4: return rn_allreduce_kernel<T, 4, kFp8>;
-        case 8: return rn_allreduce_kernel<T, 8, kFp8>;
+        case 1: return rn_allreduce_kernel<T, 1, kW, kFp8>;
+        case 2: return rn_allreduce_kernel<T, 2, kW, kFp8>;
+        case 4: return rn_allreduce_kernel<T, 4, kW, kFp8>;
+        case 8: return rn_allreduce_kernel<T, 8, kW, kFp8>;
         default: return nullptr;
     }
 }
 
-ArKernel pick(int dtype, bool fp8, int vpt) {
+template <typename T, bool kFp8>
+ArKernel pick_w(int world, int vpt) {
+    if (world == 1) return pick_vpt<T, 1, kFp8>(vpt);
+    if (world == 2) return pick_vpt<T, 2, kFp8>(vpt);
+    if (world <= 4) return pick_vpt<T, 4, kFp8>(vpt);
+    return pick_vpt<T, 8, kFp8>(vpt);
+}
+
+ArKernel pick(int dtype, bool fp8, int world, int vpt) {
+    if (world < 1 || world > kArMaxWorld) return nullptr;
     if (dtype == kBF16)
-        return fp8 ? pick_vpt<__nv_bfloat16, true>(vpt) : pick_vpt<__nv_bfloat16, false>(vpt);
-    if (dtype == kF16) return fp8 ? pick_vpt<__half, true>(vpt) : pick_vpt<__half, false>(vpt);
+        return fp8 ? pick_w<__nv_bfloat16, true>(world, vpt)
+                   : pick_w<__nv_bfloat16, false>(world, vpt);
+    if (dtype == kF16)
+        return fp8 ? pick_w<__half, true>(world, vpt) : pick_w<__half, false>(world, vpt);
     return nullptr;
 }
 
 }  // namespace
 
-cudaError_t allreduce_blocks_per_sm(int dtype, bool fp8, const ArLaunch& l, int* blocks) {
-    const ArKernel k = pick(dtype, fp8, l.vpt);
+cudaError_t allreduce_blocks_per_sm(int dtype, bool fp8, int world, const ArLaunch& l,
+                                    int* blocks) {
+    const ArKernel k = pick(dtype, fp8, world, l.vpt);
     if (!k) return cudaErrorInvalidValue;
     return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks, k, l.block,
                                                          static_cast<size_t>(l.smem));
@@ -351,7 +381,7 @@ cudaError_t allreduce_blocks_per_sm(int dtype, bool fp8, const ArLaunch& l, int*
 
 cudaError_t launch_allreduce(int dtype, bool fp8, const ArArgs& a, const ArLaunch& l,
                              cudaStream_t s) {
-    const ArKernel k = pick(dtype, fp8, l.vpt);
+    const ArKernel k = pick(dtype, fp8, a.world, l.vpt);
     if (!k) return cudaErrorInvalidValue;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(l.grid_x), static_cast<unsigned>(l.local_ranks));
@@ -362,7 +392,7 @@ cudaError_t launch_allreduce(int dtype, bool fp8, const ArArgs& a, const ArLaunc
     attr[0].id = cudaLaunchAttributeCooperative;
     attr[0].val.cooperative = 1;
     cfg.attrs = attr;
-    cfg.numAttrs = 1;
+    cfg.numAttrs = l.local_ranks > 1 ? 1 : 0;
     return cudaLaunchKernelEx(&cfg, k, a, l.tpr, l.rpc);
 }
 

@@ -16,6 +16,7 @@
 
 #include "../../include/rmsnorm_b200.h"
 #include "rn_internal.h"
+#include "rn_allreduce.h"
 
 namespace {
 
@@ -628,13 +629,18 @@ bool overlaps_bytes(const Flat& f, const void* p, int64_t bytes) {
     return a0 < b1 && b0 < a1;
 }
 
-// Row mapping of the all-reduce kernel: the smallest power-of-two group of
-// threads that covers a row with at most 4 vectors each (8 once the group
-// reaches the block limit), 256-thread blocks of several rows for narrow rows.
-rn_status ar_shape(int64_t H, rn::ArLaunch* l) {
+// Row mapping of the all-reduce kernel: a power-of-two group of threads per
+// row holding v vectors of 16 bytes each, v chosen so that a thread keeps
+// about 128 bytes of loads in flight (v = 8 / (W + 1) rounded down to a power
+// of two, at least 1: each vector costs W exchange loads and one residual
+// load), up to the 512-thread block (then 2, 4 or 8 vectors each);
+// 256-thread blocks of several rows for narrow rows.
+rn_status ar_shape(int64_t H, int world, rn::ArLaunch* l) {
     const int64_t nvec = H / 8;
+    int target = 1;
+    while (target * 2 <= 8 / (world + 1)) target *= 2;
     int tpr = 1;
-    while (static_cast<int64_t>(tpr) * 4 < nvec && tpr < rn::kArMaxBlock) tpr *= 2;
+    while (static_cast<int64_t>(tpr) * target < nvec && tpr < rn::kArMaxBlock) tpr *= 2;
     const int64_t need = (nvec + tpr - 1) / tpr;
     int vpt = 1;
     while (vpt < need) vpt *= 2;
@@ -646,9 +652,6 @@ rn_status ar_shape(int64_t H, rn::ArLaunch* l) {
     l->smem = static_cast<int>(2 * l->rpc * (tpr >= 64 ? tpr / 32 : 1) * sizeof(float) * 2);
     return RN_OK;
 }
-
-static_assert(RN_ALLREDUCE_SIGNAL_BYTES == rn::kArSignalBytes, "signal pad size");
-static_assert(RN_ALLREDUCE_MAX_WORLD == rn::kArMaxWorld, "group size");
 
 rn_status check_comm(const rn_allreduce_comm* comm) {
     if (comm->world < 1 || comm->world > RN_ALLREDUCE_MAX_WORLD) return RN_ERR_COMM;
@@ -679,7 +682,7 @@ rn_status run_allreduce(bool fp8, const rn_tensor* o, const rn_tensor* sc, const
     const int64_t slot_bytes = (comm->buffer_bytes / 2) & ~static_cast<int64_t>(15);
     if (comm->buffer_bytes < 0 || slot_bytes < 2 * T * H) return RN_ERR_COMM;
     rn::ArLaunch l;
-    if ((st = ar_shape(H, &l)) != RN_OK) return st;
+    if ((st = ar_shape(H, comm->world, &l)) != RN_OK) return st;
     if (T > 0) {
         rn_plan unused;
         if ((st = check_pointers_and_plan(op, c, device_sms(), &unused)) != RN_OK) return st;
@@ -716,7 +719,7 @@ rn_status run_allreduce(bool fp8, const rn_tensor* o, const rn_tensor* sc, const
     a.eps = eps;
     l.local_ranks = L;
     int per_sm = 0;
-    cudaError_t e = rn::allreduce_blocks_per_sm(c.dt, fp8, l, &per_sm);
+    cudaError_t e = rn::allreduce_blocks_per_sm(c.dt, fp8, comm->world, l, &per_sm);
     if (e == cudaSuccess) {
         const int64_t resident = static_cast<int64_t>(per_sm) * device_sms() / L;
         const int64_t groups = T > 0 ? (T + l.rpc - 1) / l.rpc : 1;

@@ -97,50 +97,4 @@ cudaError_t launch_fp8_rowwise_gemm(const GemmArgs& g, cudaStream_t stream);
 // device (bit 0: an mbarrier wait timed out). Synchronous.
 cudaError_t read_and_clear_device_errors(unsigned* flags);
 
-// ---- tensor-parallel all-reduce fused with the residual add and RMSNorm
-// (allreduce_kernels.cu).
-
-constexpr int kArMaxWorld = 8;      // ranks in one group (one NVSwitch domain)
-constexpr int kArMaxBlocks = 1024;  // signal-pad capacity, in blocks per rank
-constexpr int kArMaxBlock = 512;    // threads per block (the kernel's launch bound)
-constexpr int kArSignalBytes = 64 + 2 * kArMaxBlocks * kArMaxWorld * 4;  // per rank
-
-struct ArArgs {
-    int world;                        // ranks in the group
-    int rank;                         // rank driven by blockIdx.y == 0
-    void* buffers[kArMaxWorld];       // every rank's exchange buffer (this process's address)
-    uint32_t* signals[kArMaxWorld];   // every rank's signal pad (kArSignalBytes)
-    int64_t slot_elems;               // 16-bit elements per buffer half (call parity picks one)
-    long long timeout_ns;             // bound on each wait for a peer
-    const void* x;                    // partial sums [local ranks][T][H]
-    void* residual;                   // [local ranks][T][H], in place
-    const void* weight;               // [H] or nullptr
-    void* out;                        // 16-bit op: [local ranks][T][H]
-    uint8_t* q;                       // fp8 op: codes [local ranks][T][H]
-    float* scale;                     // fp8 op: [local ranks][T]
-    int64_t T, H;
-    float eps;
-};
-
-struct ArLaunch {
-    int tpr;          // threads per row
-    int vpt;          // 16-byte vectors per thread per row: 1, 2, 4 or 8
-    int rpc;          // rows per block
-    int block;        // threads per block
-    int smem;         // dynamic shared memory bytes
-    int grid_x;       // blocks per rank (the same on every rank)
-    int local_ranks;  // gridDim.y
-};
-
-// Resident blocks per SM of the all-reduce kernel for this shape.
-cudaError_t allreduce_blocks_per_sm(int dtype, bool fp8, const ArLaunch& l, int* blocks);
-
-// Cooperative launch of the all-reduce kernel (every block resident).
-cudaError_t launch_allreduce(int dtype, bool fp8, const ArArgs& a, const ArLaunch& l,
-                             cudaStream_t s);
-
-// Reads, and clears when set, the all-reduce kernel's error flags on the
-// current device (bit 1: a wait for a peer timed out). Synchronous.
-cudaError_t read_and_clear_allreduce_errors(unsigned* flags);
-
 }  // namespace rn

@@ -88,7 +88,8 @@ typedef enum {
     RN_ERR_EPS = 8,           /* eps negative, NaN or infinite */
     RN_ERR_CUDA = 9,          /* a CUDA runtime call failed */
     RN_ERR_CONFIG = 10,       /* rn_force_plan / rn_plan_launch: unsupported request */
-    RN_ERR_COMM = 11          /* all-reduce: bad group description or exchange buffers too small */
+    RN_ERR_COMM = 11,         /* all-reduce: bad group description or exchange buffers too small */
+    RN_ERR_CAPACITY = 12      /* rn_allreduce_fused_add_rms_norm_local: beyond its static memory */
 } rn_status;
 
 typedef enum {
@@ -280,6 +281,30 @@ RN_API rn_status rn_allreduce_fused_add_rms_norm_fp8(const rn_tensor* q, const r
                                                      const rn_tensor* weight, float eps,
                                                      const rn_allreduce_comm* comm,
                                                      void* stream);
+
+/* ---- the whole group on one device, with the library's own exchange memory
+ *
+ * No counterpart on the pages: they describe no such entry point. This is
+ * rn_allreduce_fused_add_rms_norm for a group of `world` ranks all held on
+ * the current device (operands stacked [world, T, H], as with local_ranks ==
+ * world; one launch computes every rank), whose exchange buffers and signal
+ * pads live in a static device array of the library instead of caller
+ * memory: it allocates nothing and takes no rn_allreduce_comm.
+ * Capacity: world * round_up(4 * T * H + 32, 256) <= RN_LOCAL_EXCHANGE_BYTES
+ * (32 MiB of buffers, plus 8 signal pads), else RN_ERR_CAPACITY before any
+ * CUDA call; world outside 1..8 is RN_ERR_COMM; otherwise the checks and
+ * errors of rn_allreduce_fused_add_rms_norm. The first call on a device
+ * looks the array up (the device must be current, as for every call), and
+ * the first call with a given `world` after another clears the signal pads
+ * with cudaMemsetAsync on `stream`: make those calls outside stream capture
+ * (RN_ERR_CONFIG inside); later calls may be captured. The memory is shared
+ * by every call on a device: calls that overlap in time (other streams,
+ * other threads) race and give undefined results. */
+#define RN_LOCAL_EXCHANGE_BYTES 33554432
+RN_API rn_status rn_allreduce_fused_add_rms_norm_local(const rn_tensor* out, const rn_tensor* x,
+                                                       const rn_tensor* residual,
+                                                       const rn_tensor* weight, float eps,
+                                                       int32_t world, void* stream);
 
 /* Static text for a status code (never NULL). */
 RN_API const char* rn_status_string(rn_status status);

@@ -26,6 +26,7 @@ __all__ = [
     "RmsNormError", "rms_norm", "fused_add_rms_norm", "fused_add_rms_norm_fp8",
     "silu_and_mul_fp8", "fp8_rowwise_gemm", "fp8_gemm_config", "fp8_gemm_force_config",
     "GEMM_CONFIGS", "allreduce_fused_add_rms_norm", "allreduce_fused_add_rms_norm_fp8",
+    "allreduce_fused_add_rms_norm_local",
     "RnAllreduceComm", "ALLREDUCE_MAX_WORLD", "ALLREDUCE_SIGNAL_BYTES", "plan_launch", "validate", "force_plan", "force_staged",
     "set_launch_options", "device_errors", "supported_vectors_per_thread", "status_string",
     "LIB_PATH", "lib", "RnTensor", "RnPlan", "STATUS", "OPS",
@@ -36,7 +37,7 @@ LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "librmsnorm_
 STATUS = {
     0: "RN_OK", 1: "RN_ERR_NULL", 2: "RN_ERR_DTYPE", 3: "RN_ERR_WEIGHT_DTYPE", 4: "RN_ERR_SHAPE",
     5: "RN_ERR_LAYOUT", 6: "RN_ERR_ALIAS", 7: "RN_ERR_VARIANCE_SIZE", 8: "RN_ERR_EPS",
-    9: "RN_ERR_CUDA", 10: "RN_ERR_CONFIG", 11: "RN_ERR_COMM",
+    9: "RN_ERR_CUDA", 10: "RN_ERR_CONFIG", 11: "RN_ERR_COMM", 12: "RN_ERR_CAPACITY",
 }
 OPS = {"rms_norm": 0, "fused_add_rms_norm": 1, "fused_add_rms_norm_fp8": 2}
 PLAN_OPS = dict(OPS, silu_and_mul_fp8=3)
@@ -116,6 +117,8 @@ def _load():
     L.rn_allreduce_fused_add_rms_norm.argtypes = [P, P, P, P, F, C, VP]
     L.rn_allreduce_fused_add_rms_norm_fp8.argtypes = [P, P, P, P, P, F, C, VP]
     L.rn_allreduce_fused_add_rms_norm.restype = ctypes.c_int
+    L.rn_allreduce_fused_add_rms_norm_local.argtypes = [P, P, P, P, F, ctypes.c_int32, VP]
+    L.rn_allreduce_fused_add_rms_norm_local.restype = ctypes.c_int
     L.rn_allreduce_fused_add_rms_norm_fp8.restype = ctypes.c_int
     L.rn_fp8_gemm_config.argtypes = [I64, I64, I64, ctypes.c_int32, ctypes.POINTER(ctypes.c_int32)]
     L.rn_fp8_gemm_config.restype = ctypes.c_int
@@ -301,6 +304,21 @@ def allreduce_fused_add_rms_norm_fp8(q: torch.Tensor, scale: torch.Tensor, x: to
                _desc(x, 2), _desc(residual, 3), None if weight is None else _desc(weight, 4),
                eps, comm.descriptor_ref(), s)
     _check(st, "rn_allreduce_fused_add_rms_norm_fp8")
+
+
+def allreduce_fused_add_rms_norm_local(out: torch.Tensor, x: torch.Tensor,
+                                       residual: torch.Tensor, weight: torch.Tensor | None,
+                                       eps: float, world: int, stream=None) -> None:
+    """A whole group of `world` ranks on one device (operands [world, T, H])
+    with the library's own static exchange memory: allocates nothing (C ABI
+    rn_allreduce_fused_add_rms_norm_local). Calls sharing a device must not
+    overlap in time; the first call, and the first after a change of
+    `world`, must be made outside CUDA-graph capture."""
+    dev, s = _stream_for((out, x, residual, weight), stream)
+    st = _call(lib.rn_allreduce_fused_add_rms_norm_local, dev, _desc(out, 0), _desc(x, 1),
+               _desc(residual, 2), None if weight is None else _desc(weight, 3), eps,
+               int(world), s)
+    _check(st, "rn_allreduce_fused_add_rms_norm_local")
 
 
 # rn_gemm_config values: TOK = token-major (tokens x channels) tiles, CH =

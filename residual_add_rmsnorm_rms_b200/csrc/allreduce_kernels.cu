@@ -396,6 +396,15 @@ cudaError_t launch_allreduce(int dtype, bool fp8, const ArArgs& a, const ArLaunc
     return cudaLaunchKernelEx(&cfg, k, a, l.tpr, l.rpc);
 }
 
+// Exchange memory of rn_allreduce_fused_add_rms_norm_local: signal pads, then
+// buffers (rn_allreduce.h). Zero at module load; the pads are cleared again by
+// the host whenever the group size on a device changes.
+static __device__ __align__(256) unsigned char g_rn_local_scratch[kLocalScratchBytes];
+
+cudaError_t local_scratch_address(void** p) {
+    return cudaGetSymbolAddress(p, g_rn_local_scratch);
+}
+
 cudaError_t read_and_clear_allreduce_errors(unsigned* flags) {
     unsigned v = 0;
     cudaError_t e = cudaMemcpyFromSymbol(&v, g_rn_ar_error, sizeof v);

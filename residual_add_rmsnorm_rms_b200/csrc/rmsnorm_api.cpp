@@ -8,6 +8,7 @@
 #include <cstdint>
 #include <cstdio>
 #include <cstring>
+#include <mutex>
 
 #include <atomic>
 #include <initializer_list>
@@ -737,9 +738,80 @@ rn_status run_allreduce(bool fp8, const rn_tensor* o, const rn_tensor* sc, const
     return RN_OK;
 }
 
+// Per device: the address of the library's static exchange memory and the
+// group size its signal pads were last prepared for.
+struct LocalGroup {
+    void* base = nullptr;
+    int world = 0;
+};
+constexpr int kMaxDevices = 64;
+LocalGroup g_local[kMaxDevices];
+std::mutex g_local_mu;
+
+rn_status local_cuda_error(cudaError_t e) {
+    std::snprintf(g_cuda_error, sizeof g_cuda_error, "%s: %s", cudaGetErrorName(e),
+                  cudaGetErrorString(e));
+    return RN_ERR_CUDA;
+}
+
 }  // namespace
 
 extern "C" {
+
+rn_status rn_allreduce_fused_add_rms_norm_local(const rn_tensor* out, const rn_tensor* x,
+                                                const rn_tensor* residual,
+                                                const rn_tensor* weight, float eps,
+                                                int32_t world, void* stream) {
+    if (world < 1 || world > rn::kArMaxWorld) return RN_ERR_COMM;
+    Common c;
+    rn_status st = check_descriptors(rn::kFusedAdd, out, nullptr, x, residual, weight, eps, -1, &c);
+    if (st != RN_OK) return st;
+    if (c.x.T % world != 0) return RN_ERR_SHAPE;
+    const int64_t T = c.x.T / world, H = c.x.H;
+    const int64_t buffer_bytes = ((4 * T * H + 32 + 255) / 256) * 256;
+    if (buffer_bytes * world > rn::kLocalBufferBytes) return RN_ERR_CAPACITY;
+
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) return local_cuda_error(e);
+    if (dev < 0 || dev >= kMaxDevices) return RN_ERR_CONFIG;
+    const auto s = static_cast<cudaStream_t>(stream);
+    rn_allreduce_comm comm = {};
+    {
+        std::lock_guard<std::mutex> lock(g_local_mu);
+        LocalGroup& g = g_local[dev];
+        if (!g.base || g.world != world) {
+            // first use on this device or a new group size: the setup (symbol
+            // lookup, clearing the pads on `stream`) must not be captured
+            cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+            e = cudaStreamIsCapturing(s, &cs);
+            if (e != cudaSuccess) return local_cuda_error(e);
+            if (cs != cudaStreamCaptureStatusNone) return RN_ERR_CONFIG;
+        }
+        if (!g.base) {
+            void* p = nullptr;
+            e = rn::local_scratch_address(&p);  // the current device is `dev`
+            if (e != cudaSuccess) return local_cuda_error(e);
+            g.base = p;
+        }
+        if (g.world != world) {
+            e = cudaMemsetAsync(g.base, 0, rn::kLocalPadStride * rn::kArMaxWorld, s);
+            if (e != cudaSuccess) return local_cuda_error(e);
+            g.world = world;
+        }
+        char* base = static_cast<char*>(g.base);
+        comm.world = world;
+        comm.rank = 0;
+        comm.local_ranks = world;
+        for (int p = 0; p < world; ++p) {
+            comm.signals[p] = base + p * rn::kLocalPadStride;
+            comm.buffers[p] = base + rn::kLocalPadStride * rn::kArMaxWorld + p * buffer_bytes;
+        }
+        comm.buffer_bytes = buffer_bytes;
+        comm.timeout_ns = 0;
+    }
+    return run_allreduce(false, out, nullptr, x, residual, weight, eps, &comm, stream);
+}
 
 rn_status rn_allreduce_fused_add_rms_norm(const rn_tensor* out, const rn_tensor* x,
                                           const rn_tensor* residual, const rn_tensor* weight,
@@ -781,6 +853,7 @@ const char* rn_status_string(rn_status s) {
         case RN_ERR_CUDA: return "CUDA error (see rn_last_cuda_error)";
         case RN_ERR_CONFIG: return "unsupported launch configuration";
         case RN_ERR_COMM: return "bad all-reduce group description or exchange buffers too small";
+        case RN_ERR_CAPACITY: return "problem larger than the library's static exchange memory";
     }
     return "unknown status";
 }

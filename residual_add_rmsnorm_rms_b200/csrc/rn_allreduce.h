@@ -51,6 +51,16 @@ cudaError_t allreduce_blocks_per_sm(int dtype, bool fp8, int world, const ArLaun
 cudaError_t launch_allreduce(int dtype, bool fp8, const ArArgs& a, const ArLaunch& l,
                              cudaStream_t s);
 
+// Static exchange memory of rn_allreduce_fused_add_rms_norm_local (a whole
+// group on one device): kArMaxWorld signal pads, kLocalPadStride bytes apart,
+// then up to kLocalBufferBytes of exchange buffers.
+constexpr int64_t kLocalPadStride = ((kArSignalBytes + 255) / 256) * 256;
+constexpr int64_t kLocalBufferBytes = 32LL << 20;
+constexpr int64_t kLocalScratchBytes = kLocalPadStride * kArMaxWorld + kLocalBufferBytes;
+
+// Device address of that memory on the current device.
+cudaError_t local_scratch_address(void** p);
+
 // Reads, and clears when set, the all-reduce kernel's error flags on the
 // current device (bit 1: a wait for a peer timed out). Synchronous.
 cudaError_t read_and_clear_allreduce_errors(unsigned* flags);

@@ -169,3 +169,20 @@ def test_exchange_records_orders_by_rank():
 def test_exchange_records_detects_disagreement():
     res = _run_exchange([512, 1024])
     assert all(isinstance(v, str) and "hidden" in v for v in res.values())
+
+
+def test_no_alloc_entry_point_validation():
+    """Refusals of rn_allreduce_fused_add_rms_norm_local that come before any
+    CUDA call (host stand-in pointers are never dereferenced)."""
+    def call(out, x, r, w, world):
+        ds = [rn.describe(t) for t in (out, x, r, w)]
+        ref = [None if d is None else ctypes.byref(d) for d, _ in ds]
+        return rn.STATUS[rn.lib.rn_allreduce_fused_add_rms_norm_local(*ref, 1e-6, world, None)]
+    out, x, r, w = _ops(L=2, T=8, H=512)
+    for world in (0, 9, -1):
+        assert call(out, x, r, w, world) == "RN_ERR_COMM"
+    assert call(out, x, r, w.half(), 2) == "RN_ERR_WEIGHT_DTYPE"
+    o3, x3, r3, _ = _ops(L=3, T=5)
+    assert call(o3, x3, r3, w, 2) == "RN_ERR_SHAPE"
+    big = torch.zeros(8, 257, 4096, dtype=torch.bfloat16)  # 8 ranks x 257 rows: > 32 MiB
+    assert call(torch.zeros_like(big), big, torch.zeros_like(big), None, 8) == "RN_ERR_CAPACITY"

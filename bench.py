@@ -762,7 +762,7 @@ def run_sweep(args, world, rank, local):
     fp8_peak, fp8_src = measured_fp8_peak()
     for M, N, K in gemm_cells:
         configs = [None]
-        if args.sweep_gemm_configs and M <= 256:
+        if args.sweep_gemm_configs:
             configs += list(rn.GEMM_CONFIGS)
         for cfg, (us, gus, name) in time_gemm_cell(rn, M, N, K, args.sweep_iters, device,
                                                    configs).items():
@@ -798,7 +798,7 @@ def main():
                          "one JSON line per cell to this file")
     ap.add_argument("--sweep-iters", type=int, default=50)
     ap.add_argument("--sweep-gemm-configs", action="store_true",
-                    help="also time every GEMM tile configuration, forced, on cells with M <= 256")
+                    help="also time every GEMM tile configuration, forced, on every GEMM cell")
     ap.add_argument("--sweep-filter", default=None,
                     help="comma-separated values a cell must all match (workload, op, dtype, "
                          "T or H), e.g. swiglu,bf16,8192")

@@ -175,7 +175,8 @@ RN_API rn_status rn_fp8_rowwise_gemm(const rn_tensor* d, const rn_tensor* a,
 /* Tile configurations of rn_fp8_rowwise_gemm. TOK tiles put the tensor core's
  * MMA rows on tokens: (tokens x channels) = 128 x 128. CH tiles compute D^T =
  * B * A^T, putting the MMA rows on the weight's output channels: (channels x
- * tokens), for decode-sized M where 128 token rows would be mostly padding.
+ * tokens), for decode-sized M where 128 token rows would be mostly padding;
+ * TOK128_CH256 is the token-major tile with 256 channels.
  * Every configuration computes the same values: the scales are applied in the
  * same order and the fp32 accumulation over K differs only in its order. */
 typedef enum {
@@ -185,15 +186,17 @@ typedef enum {
     RN_GEMM_CH128_TOK64 = 3,
     RN_GEMM_CH64_TOK16 = 4,
     RN_GEMM_CH64_TOK32 = 5,
-    RN_GEMM_CH64_TOK64 = 6
+    RN_GEMM_CH64_TOK64 = 6,
+    RN_GEMM_TOK128_CH256 = 7
 } rn_gemm_config;
 
 /* The configuration rn_fp8_rowwise_gemm uses for an M x N x K problem on a
  * device with `num_sms` SMs (<= 0: 148). Among the CH configurations, the one
  * with the most tiles (ceil(N / channels) * ceil(M / tokens)) not above
  * num_sms, ties going to fewer channels, then fewer tokens per tile; if none
- * fits, CH128 with the smallest token width >= M for M <= 64, TOK128_CH128
- * above. Honours rn_fp8_gemm_force_config. Pure host logic. RN_ERR_SHAPE for
+ * fits, CH128 with the smallest token width >= M for M <= 64; above,
+ * TOK128_CH256 when ceil(M / 128) * ceil(N / 256) >= num_sms, else
+ * TOK128_CH128. Honours rn_fp8_gemm_force_config. Pure host logic. RN_ERR_SHAPE for
  * M < 0, N < 1 or K < 1. */
 RN_API rn_status rn_fp8_gemm_config(int64_t M, int64_t N, int64_t K, int32_t num_sms,
                                     int32_t* config);

@@ -324,7 +324,7 @@ def allreduce_fused_add_rms_norm_local(out: torch.Tensor, x: torch.Tensor,
 # rn_gemm_config values: TOK = token-major (tokens x channels) tiles, CH =
 # channel-major (channels x tokens) tiles computing D^T.
 GEMM_CONFIGS = {"tok128_ch128": 0, "ch128_tok16": 1, "ch128_tok32": 2, "ch128_tok64": 3,
-                "ch64_tok16": 4, "ch64_tok32": 5, "ch64_tok64": 6}
+                "ch64_tok16": 4, "ch64_tok32": 5, "ch64_tok64": 6, "tok128_ch256": 7}
 
 
 def fp8_gemm_config(M: int, N: int, K: int, num_sms: int = 0) -> str:

@@ -1,5 +1,5 @@
 // fp8_gemm.cu -- tile-configuration dispatch of the row-wise scaled FP8 GEMM
-// and its token-major 128 x 128 instantiation (the template and the two
+// and its token-major 128 x 128 and 128 x 256 instantiations (the template and the two
 // orientations are described in fp8_gemm.cuh). The channel-major
 // instantiations for decode-sized M live in fp8_gemm_ch128.cu and
 // fp8_gemm_ch64.cu so that the three units compile in parallel.
@@ -15,6 +15,8 @@ cudaError_t launch_fp8_rowwise_gemm(const GemmArgs& g, cudaStream_t stream) {
     switch (g.config) {
         case kGemmTok128Ch128:
             return RowwiseGemm<Shape<_128, _128, _128>, false>::run(g, stream);
+        case kGemmTok128Ch256:
+            return RowwiseGemm<Shape<_128, _256, _128>, false>::run(g, stream);
         case kGemmCh128Tok16: return gemm_channel_major_128(16, g, stream);
         case kGemmCh128Tok32: return gemm_channel_major_128(32, g, stream);
         case kGemmCh128Tok64: return gemm_channel_major_128(64, g, stream);

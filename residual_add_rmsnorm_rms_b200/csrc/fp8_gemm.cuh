@@ -45,7 +45,7 @@
 #include "cutlass/gemm/kernel/gemm_universal.hpp"
 #include "cutlass/util/packed_stride.hpp"
 
-#include "rn_internal.h"
+#include "rn_gemm.h"
 
 namespace rn {
 namespace gemm_detail {

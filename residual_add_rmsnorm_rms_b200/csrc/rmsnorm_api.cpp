@@ -18,6 +18,7 @@
 #include "../../include/rmsnorm_b200.h"
 #include "rn_internal.h"
 #include "rn_allreduce.h"
+#include "rn_gemm.h"
 
 namespace {
 
@@ -309,8 +310,8 @@ int device_sms() {
 // channel-major shapes (channels x tokens: 64 or 128 x 16, 32 or 64), the one
 // with the most tiles that still fit in one wave (ties: fewer channels, then
 // fewer tokens per tile). When none fits, up to 64 tokens take the 128-channel
-// tile of the smallest token width >= M (fewest tiles), larger M the
-// token-major 128 x 128 tile. Measured on B200 over the Gemma 4 12B weight
+// tile of the smallest token width >= M (fewest tiles), larger M a token-major
+// tile. Measured on B200 over the Gemma 4 12B weight
 // shapes, this picks the fastest configuration or one within 5 % of it.
 int gemm_auto_config(int64_t M, int64_t N, int num_sms) {
     struct Shape { int config, ch, tok; };
@@ -331,7 +332,10 @@ int gemm_auto_config(int64_t M, int64_t N, int num_sms) {
     if (M <= 16) return rn::kGemmCh128Tok16;
     if (M <= 32) return rn::kGemmCh128Tok32;
     if (M <= 64) return rn::kGemmCh128Tok64;
-    return rn::kGemmTok128Ch128;
+    // token-major: 128 x 256 tiles once they fill a wave (12-16 % faster than
+    // 128 x 128 at M = 8192 on B200), else 128 x 128 for twice the tiles
+    const int64_t tiles256 = ((M + 127) / 128) * ((N + 255) / 256);
+    return tiles256 >= num_sms ? rn::kGemmTok128Ch256 : rn::kGemmTok128Ch128;
 }
 
 int gemm_config(int64_t M, int64_t N, int num_sms) {

@@ -30,33 +30,6 @@ struct SwigluArgs {
     int64_t I;
 };
 
-// Operands of the row-wise scaled fp8 GEMM (device pointers; see fp8_gemm.cu).
-struct GemmArgs {
-    const void* a;        // [M x K] e4m3
-    const void* b;        // [N x K] e4m3
-    const float* a_scale; // [M]
-    const float* b_scale; // [N]
-    void* d;              // [M x N] bf16
-    int64_t M, N, K;
-    int device;
-    int num_sms;
-    int config;           // GemmConfig: tile shape and orientation
-};
-
-// Tile configurations of the fp8 GEMM (values of rn_gemm_config in the public
-// header). Token-major tiles are (tokens x channels); channel-major tiles
-// compute D^T and are (channels x tokens).
-enum GemmConfig {
-    kGemmTok128Ch128 = 0,
-    kGemmCh128Tok16 = 1,
-    kGemmCh128Tok32 = 2,
-    kGemmCh128Tok64 = 3,
-    kGemmCh64Tok16 = 4,
-    kGemmCh64Tok32 = 5,
-    kGemmCh64Tok64 = 6,
-    kNumGemmConfigs = 7
-};
-
 struct Launch {
     int kernel;  // 0 = vector, 1 = scalar, 2 = staged
     int tpr;     // threads per row
@@ -89,9 +62,6 @@ cudaError_t launch(int op, int dtype, const Args& a, const Launch& l, cudaStream
 
 // Enqueues the fused SwiGLU + FP8 cast (vector plan: kernel 0; scalar: 1).
 cudaError_t launch_swiglu_fp8(int dtype, const SwigluArgs& a, const Launch& l, cudaStream_t s);
-
-// Runs the row-wise scaled fp8 GEMM on `stream` (tcgen05 tensor cores).
-cudaError_t launch_fp8_rowwise_gemm(const GemmArgs& g, cudaStream_t stream);
 
 // Reads, and clears when set, the device-side error flags of the current
 // device (bit 0: an mbarrier wait timed out). Synchronous.

@@ -320,8 +320,9 @@ def test_gemm_config_choice():
     assert cfg(1, 30720, 3840, 148) == "ch128_tok16"    # nothing fits one wave
     assert cfg(33, 30720, 3840, 148) == "ch128_tok64"
     assert cfg(256, 3840, 8192, 148) == "ch128_tok64"   # 120 tiles
-    assert cfg(256, 8192, 3840, 148) == "tok128_ch128"
-    assert cfg(8192, 8192, 3840, 148) == "tok128_ch128"
+    assert cfg(256, 8192, 3840, 148) == "tok128_ch128"   # 64 tiles of 128 x 256: < 1 wave
+    assert cfg(8192, 8192, 3840, 148) == "tok128_ch256"
+    assert cfg(256, 30720, 3840, 148) == "tok128_ch256"  # 240 tiles of 128 x 256
     assert cfg(0, 8, 16) in rn.GEMM_CONFIGS               # empty problem: any valid config
     for bad in ((-1, 8, 16), (1, 0, 16), (1, 8, 0)):
         with pytest.raises(rn.RmsNormError) as e:
@@ -347,11 +348,12 @@ def test_gemm_config_choice_is_the_fullest_wave(seed):
             assert got == min((c for c in CH_SHAPES if c.startswith("ch128") and
                                CH_SHAPES[c][1] >= M), key=lambda c: CH_SHAPES[c][1])
         else:
-            assert got == "tok128_ch128"
+            t256 = -(-M // 128) * -(-N // 256)
+            assert got == ("tok128_ch256" if t256 >= sms else "tok128_ch128")
 
 
 def test_gemm_force_config_hook():
-    for bad in (-2, 7, 100):
+    for bad in (-2, 8, 100):
         with pytest.raises(rn.RmsNormError) as e:
             rn.fp8_gemm_force_config(bad)
         assert e.value.name == "RN_ERR_CONFIG"
@@ -362,7 +364,7 @@ def test_gemm_force_config_hook():
             assert rn.fp8_gemm_config(1, 8, 16) == name
     finally:
         rn.fp8_gemm_force_config(None)
-    assert rn.fp8_gemm_config(8192, 8192, 3840) == "tok128_ch128"
+    assert rn.fp8_gemm_config(8192, 8192, 3840) == "tok128_ch256"
 
 
 def test_status_strings():

@@ -23,13 +23,25 @@ Every rank of a group must make the same sequence of calls.
 from __future__ import annotations
 
 import ctypes
+import itertools
+import weakref
 from typing import Optional, Sequence
 
 import torch
 
 from . import ALLREDUCE_MAX_WORLD, ALLREDUCE_SIGNAL_BYTES, RnAllreduceComm
 
-__all__ = ["AllReduceComm", "buffer_bytes_for", "exchange_records"]
+__all__ = ["AllReduceComm", "buffer_bytes_for", "exchange_records", "lookup"]
+
+# Live communicators by integer handle (the torch custom ops take the handle:
+# their schemas admit tensors and scalars only).
+_LIVE: "weakref.WeakValueDictionary[int, AllReduceComm]" = weakref.WeakValueDictionary()
+_HANDLES = itertools.count(1)
+
+
+def lookup(handle: int) -> "AllReduceComm":
+    """The live AllReduceComm with this handle (KeyError when gone)."""
+    return _LIVE[handle]
 
 
 def buffer_bytes_for(max_rows: int, hidden: int) -> int:
@@ -81,6 +93,8 @@ class AllReduceComm:
         d.timeout_ns = self.timeout_ns
         self._desc = d
         self._ref = ctypes.byref(d)
+        self.handle = next(_HANDLES)
+        _LIVE[self.handle] = self
 
     @property
     def max_elements(self) -> int:

@@ -22,6 +22,12 @@ Ops (namespace ``rmsnorm_b200``; CUDA only, N-D inputs flattened to
   residual := x + residual; q (float8_e4m3fn, shape of x) and scale
   (float32, shape of x with the last dim 1) the per-token dynamic cast of
   rms_norm(residual)
+* ``allreduce_fused_add_rms_norm(x, residual!, weight, epsilon, comm) -> out``
+  and ``allreduce_fused_add_rms_norm_fp8(...) -> (q, scale)``: the
+  tensor-parallel forms, x the local partial sum, all-reduced across the
+  group of the AllReduceComm whose ``handle`` is ``comm`` before the fused op
+  (with a whole group on one device, the operands carry the leading rank
+  dimension)
 
 Each has a fake (meta) implementation, so torch.compile traces through it.
 
@@ -44,6 +50,9 @@ from . import fused_add_rms_norm_fp8 as _fused_fp8
 from . import rms_norm as _rms
 from . import fp8_rowwise_gemm as _gemm
 from . import silu_and_mul_fp8 as _silu_fp8
+from . import allreduce_fused_add_rms_norm as _ar
+from . import allreduce_fused_add_rms_norm_fp8 as _ar_fp8
+from .allreduce import lookup as _comm_lookup
 
 __all__ = [
     "flatten_to_2d_is_free", "rms_no_var_16bit_only", "rms_add_no_var_16bit_only",
@@ -180,6 +189,38 @@ def _fp8_rowwise_gemm_op(a: torch.Tensor, b: torch.Tensor, a_scale: torch.Tensor
 @_fp8_rowwise_gemm_op.register_fake
 def _(a, b, a_scale, b_scale):
     return torch.empty(a.shape[:-1] + (b.shape[0],), dtype=torch.bfloat16, device=a.device)
+
+
+@torch.library.custom_op(f"{LIB}::allreduce_fused_add_rms_norm", mutates_args=("residual",),
+                         device_types="cuda")
+def _allreduce_fused_add_rms_norm_op(x: torch.Tensor, residual: torch.Tensor,
+                                     weight: Optional[torch.Tensor], epsilon: float,
+                                     comm: int) -> torch.Tensor:
+    out = _dense_like(x)
+    _ar(out, x, residual, weight, epsilon, _comm_lookup(comm))
+    return out
+
+
+@_allreduce_fused_add_rms_norm_op.register_fake
+def _(x, residual, weight, epsilon, comm):
+    return _dense_like(x)
+
+
+@torch.library.custom_op(f"{LIB}::allreduce_fused_add_rms_norm_fp8", mutates_args=("residual",),
+                         device_types="cuda")
+def _allreduce_fused_add_rms_norm_fp8_op(x: torch.Tensor, residual: torch.Tensor,
+                                         weight: Optional[torch.Tensor], epsilon: float,
+                                         comm: int) -> tuple[torch.Tensor, torch.Tensor]:
+    q = _dense_like(x, torch.float8_e4m3fn)
+    scale = torch.empty(x.shape[:-1] + (1,), dtype=torch.float32, device=x.device)
+    _ar_fp8(q, scale, x, residual, weight, epsilon, _comm_lookup(comm))
+    return q, scale
+
+
+@_allreduce_fused_add_rms_norm_fp8_op.register_fake
+def _(x, residual, weight, epsilon, comm):
+    return (_dense_like(x, torch.float8_e4m3fn),
+            torch.empty(x.shape[:-1] + (1,), dtype=torch.float32, device=x.device))
 
 
 # --------------------------------------------------------------------------- dispatch

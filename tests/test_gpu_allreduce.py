@@ -237,3 +237,32 @@ def test_allreduce_cuda_graph_replay():
         got = {"residual": res[rep % W], "out": out[rep % W]}
         compare("fused", got, {"residual": r_bits, "out": out_bits}, "bf16")
     del g
+
+
+def test_allreduce_torch_ops_equal_direct_calls():
+    """The torch custom ops (communicator passed by handle) against the
+    direct binding, bit for bit, and through torch.compile."""
+    W, T, H = 2, 16, 3840
+    wl = synth.make_tp_inputs("bf16", W, T, H, seed=77)
+    x, w = wl.x.cuda(), wl.weight.cuda()
+    res = wl.residual.cuda().unsqueeze(0).repeat(W, 1, 1).contiguous()
+    comm = AllReduceComm.single_device(W, T, H, "cuda")
+    ra, rb = res.clone(), res.clone()
+    out_a = torch.ops.rmsnorm_b200.allreduce_fused_add_rms_norm(x, ra, w, wl.eps, comm.handle)
+    out_b = torch.empty_like(x)
+    rn.allreduce_fused_add_rms_norm(out_b, x, rb, w, wl.eps, comm)
+    torch.cuda.synchronize()
+    assert torch.equal(out_a.view(torch.int16), out_b.view(torch.int16))
+    assert torch.equal(ra.view(torch.int16), rb.view(torch.int16))
+
+    def layer(x, r, w):
+        return torch.ops.rmsnorm_b200.allreduce_fused_add_rms_norm_fp8(x, r, w, wl.eps,
+                                                                       comm.handle)
+
+    rc, re_ = res.clone(), res.clone()
+    qc, sc = torch.compile(layer, backend="aot_eager", fullgraph=True)(x, rc, w)
+    qe, se = layer(x, re_, w)
+    torch.cuda.synchronize()
+    assert sc.shape == (W, T, 1)
+    assert torch.equal(qc.view(torch.uint8), qe.view(torch.uint8)) and torch.equal(sc, se)
+    assert torch.equal(rc.view(torch.int16), re_.view(torch.int16))

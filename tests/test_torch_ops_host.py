@@ -72,6 +72,27 @@ def test_fake_implementations_infer_shapes():
         assert q.shape == x.shape and q.dtype == torch.float8_e4m3fn
         assert s.shape == (2, 3, 1) and s.dtype == torch.float32
         assert torch.ops.rmsnorm_b200.fused_add_rms_norm(x, r, w, 1e-6) is None
+        out = torch.ops.rmsnorm_b200.allreduce_fused_add_rms_norm(x, r, w, 1e-6, 7)
+        assert out.shape == x.shape and out.dtype == BF
+        q, s = torch.ops.rmsnorm_b200.allreduce_fused_add_rms_norm_fp8(x, r, w, 1e-6, 7)
+        assert q.shape == x.shape and s.shape == (2, 3, 1)
+
+
+def test_allreduce_ops_schemas_and_comm_handles():
+    import re
+    for name in ("allreduce_fused_add_rms_norm", "allreduce_fused_add_rms_norm_fp8"):
+        schema = str(getattr(torch.ops.rmsnorm_b200, name).default._schema)
+        assert re.search(r"Tensor\(a\d*!\) residual", schema) and "Int comm" in schema, schema
+    from residual_add_rmsnorm_rms_b200.allreduce import AllReduceComm, lookup
+    a = AllReduceComm(2, 0, 2, [16, 32], [48, 64], 4096)
+    b = AllReduceComm(1, 0, 1, [16], [48], 4096)
+    assert a.handle != b.handle and lookup(a.handle) is a and lookup(b.handle) is b
+    h = b.handle
+    del b
+    import gc
+    gc.collect()
+    with pytest.raises(KeyError):
+        lookup(h)
 
 
 def test_dispatch_rejects_ineligible_inputs_loudly():

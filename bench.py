@@ -641,24 +641,38 @@ def time_gemm_cell(rn, M, N, K, iters, device, configs=(None,)):
     return out
 
 
-def tp_bytes(fp8: bool, W: int, T: int, H: int) -> int:
-    """Bytes one single-device group call moves, per rank and row: the
-    partial read (2H), its copy into the exchange buffer (2H), the reads of
-    all W exchange buffers (2WH: every rank reads every buffer; W buffers of
-    a large call do not stay in L2 together), the residual read and write
-    (4H) and the output (2H, or H codes + a 4-byte scale)."""
-    per_row = (9 + 2 * W) * H + 4 if fp8 else (10 + 2 * W) * H
-    return W * T * per_row
+def tp_bytes(fp8: bool, W: int, T: int, H: int, two_shot: bool = False) -> int:
+    """Bytes one single-device group call moves (every rank of the group).
+
+    One-shot, per rank and row: the partial read (2H), its copy into the
+    exchange buffer (2H), the reads of all W exchange buffers (2WH: every rank
+    reads every buffer; W buffers of a large call do not stay in L2
+    together), the residual read and write (4H) and the output (2H, or H
+    codes + a 4-byte scale). Two-shot, per rank: the same copy (4H per row);
+    for its T/W rows the W partial reads, the residual read and write and the
+    output, each finished row also written to its buffer (residual and
+    output); for the other rows, the finished residual and output read from
+    their owner and written out."""
+    if not two_shot:
+        per_row = (9 + 2 * W) * H + 4 if fp8 else (10 + 2 * W) * H
+        return W * T * per_row
+    out = H + 4 if fp8 else 2 * H                     # output bytes of one row
+    own = 2 * W * H + 2 * H + 2 * H + out + 2 * H + out  # a row of the rank's slice
+    other = 2 * (2 * H + out)                         # a row gathered from its owner
+    S = -(-T // W)
+    per_rank = [T * 4 * H + max(0, min(T, (q + 1) * S) - q * S) * (own - other) + T * other
+                for q in range(W)]
+    return sum(per_rank)
 
 
-def time_tp_cell(rn, fp8, W, T, H, iters, device):
+def time_tp_cell(rn, fp8, W, T, H, iters, device, algorithm="one_shot"):
     """A whole tensor-parallel group of W ranks on this device (one launch
     per call): mean time per call over `iters` eager calls rotating over
     operand sets of >= 4x L2 (at most 8), and CUDA-graph replay time of 50
     captured calls for calls under 60 us."""
     from residual_add_rmsnorm_rms_b200.allreduce import AllReduceComm
     wl = synth.make_tp_inputs("bf16", W, T, H, device=device)
-    comm = AllReduceComm.single_device(W, T, H, device)
+    comm = AllReduceComm.single_device(W, T, H, device, algorithm=algorithm)
     per = 2 * W * T * H * 3
     n = min(8, max(1, math.ceil(4 * torch.cuda.get_device_properties(device).L2_cache_size / per)))
     sets = []
@@ -739,21 +753,25 @@ def run_sweep(args, world, rank, local):
                "tpr": plan["threads_per_row"], "vpt": plan["vectors_per_thread"]}
         out.write(json.dumps(rec) + "\n")
         out.flush()
-    tp_cells = [(fp8, W, T, H) for fp8 in (False, True) for W in synth.TP_W
+    tp_cells = [(fp8, W, T, H, algo) for fp8 in (False, True) for W in synth.TP_W
                 for T in synth.TP_T for H in (3840,)
+                for algo in (("one_shot", "two_shot") if W >= 3 else ("one_shot",))
                 if all(w in ("tp", "allreduce", str(W), str(T), str(H),
-                             "fp8" if fp8 else "bf16") for w in want)]
-    for fp8, W, T, H in tp_cells:
-        us, gus = time_tp_cell(rn, fp8, W, T, H, args.sweep_iters, device)
+                             "fp8" if fp8 else "bf16", algo) for w in want)]
+    for fp8, W, T, H, algo in tp_cells:
+        us, gus = time_tp_cell(rn, fp8, W, T, H, args.sweep_iters, device, algo)
         best = gus if gus is not None else us
-        nbytes = tp_bytes(fp8, W, T, H)
+        nbytes = tp_bytes(fp8, W, T, H, algo == "two_shot")
+        S = -(-T // W)
+        remote = ((W - 1) * 2 * T * H if algo == "one_shot"
+                  else S * (W - 1) * 2 * H + (T - S) * (2 * H + (H + 4 if fp8 else 2 * H)))
         rec = {"workload": "tp", "op": "allreduce_fused_add_rms_norm" + ("_fp8" if fp8 else ""),
-               "dtype": "bf16", "W": W, "T": T, "H": H, "us": round(us, 3),
-               "graph_us": None if gus is None else round(gus, 3),
+               "dtype": "bf16", "W": W, "T": T, "H": H, "algorithm": algo,
+               "us": round(us, 3), "graph_us": None if gus is None else round(gus, 3),
                "gbs": round(nbytes / best / 1e3, 1),
                "frac_of_measured": round(nbytes / best / 1e3 / peak, 4), "bytes": nbytes,
                "rows_per_s": round(W * T / (best / 1e6), 1),
-               "remote_bytes_per_rank": (W - 1) * 2 * T * H,
+               "remote_bytes_per_rank": remote,
                "how": "whole group on one device, one cooperative launch per call"}
         out.write(json.dumps(rec) + "\n")
         out.flush()

@@ -242,22 +242,38 @@ RN_API rn_status rn_fp8_gemm_force_config(int32_t config);
  * call counters stay equal) and writes nothing. */
 #define RN_ALLREDUCE_MAX_WORLD 8
 /* Signal pad bytes per rank: a 64-byte header (the rank's call counter and an
- * arrival counter, kept by the kernel) and 2 x 1024 blocks x 8 ranks 32-bit
- * flags. */
-#define RN_ALLREDUCE_SIGNAL_BYTES 65600
+ * arrival counter, kept by the kernel) and 2 parities x 2 stages x 1024
+ * blocks x 8 ranks 32-bit flags. */
+#define RN_ALLREDUCE_SIGNAL_BYTES 131136
+
+/* Exchange algorithms. ONE_SHOT: every rank reads every row of every peer's
+ * partial ((W - 1) * 2 * T * H bytes of peer reads per rank). TWO_SHOT (3 to 8
+ * ranks): rank q reduces and finishes the rows [q * S, (q + 1) * S), S =
+ * ceil(T / W), writes them to its buffer, and every rank copies the other
+ * slices' finished rows ((W - 1) / W * 6 * T * H bytes per rank, a second
+ * exchange barrier, buffers of 12 * T * H + 32 bytes). AUTO takes two-shot
+ * when the buffers hold it, W >= 4 and it saves at least 2.3 MB of peer reads
+ * per rank; both give bit-identical results. */
+typedef enum {
+    RN_ALLREDUCE_AUTO = 0,
+    RN_ALLREDUCE_ONE_SHOT = 1,
+    RN_ALLREDUCE_TWO_SHOT = 2
+} rn_allreduce_algorithm;
 
 typedef struct {
     int32_t world;       /* ranks in the group, 1..RN_ALLREDUCE_MAX_WORLD */
     int32_t rank;        /* group rank of the first (or only) rank this call computes */
     int32_t local_ranks; /* ranks this call computes on this device: 1, or `world`
                           * with rank == 0 (the whole group on one device) */
+    int32_t algorithm;   /* rn_allreduce_algorithm; the same on every rank */
     void* buffers[RN_ALLREDUCE_MAX_WORLD]; /* [world] each rank's exchange buffer, as
                           * addressed from this device; the caller owns them */
     void* signals[RN_ALLREDUCE_MAX_WORLD]; /* [world] each rank's signal pad of
                           * RN_ALLREDUCE_SIGNAL_BYTES: zero-filled before the first
                           * call, then written only by these kernels; one group's */
     int64_t buffer_bytes; /* size of each exchange buffer: two halves, each holding
-                          * T * H 16-bit values: buffer_bytes >= 4 * T * H + 32 */
+                          * T * H 16-bit values (one-shot: buffer_bytes >= 4 * T * H + 32)
+                          * or 3 * T * H (two-shot: >= 12 * T * H + 32) */
     int64_t timeout_ns;  /* bound on each wait for a peer; <= 0 selects 1 second */
 } rn_allreduce_comm;
 
@@ -266,8 +282,9 @@ typedef struct {
  * so calls captured in a CUDA graph stay numbered correctly on replay. */
 
 /* Errors: the fused ops' validation, then RN_ERR_COMM for an invalid `comm`
- * (world, rank, local_ranks, a NULL or misaligned buffer or pad,
- * buffers too small for T and H), RN_ERR_LAYOUT for the alignment rules
+ * (world, rank, local_ranks, algorithm, a NULL or misaligned buffer or pad,
+ * buffers too small for T, H and the algorithm, TWO_SHOT with fewer than 3
+ * ranks), RN_ERR_LAYOUT for the alignment rules
  * above, RN_ERR_SHAPE for H > 32768 or a row count not divisible by
  * local_ranks, RN_ERR_ALIAS when an operand overlaps a local exchange buffer
  * or signal pad, RN_ERR_CUDA when the launch fails. A peer that does not
@@ -296,13 +313,15 @@ RN_API rn_status rn_allreduce_fused_add_rms_norm_fp8(const rn_tensor* q, const r
  * Capacity: world * round_up(4 * T * H + 32, 256) <= RN_LOCAL_EXCHANGE_BYTES
  * (32 MiB of buffers, plus 8 signal pads), else RN_ERR_CAPACITY before any
  * CUDA call; world outside 1..8 is RN_ERR_COMM; otherwise the checks and
- * errors of rn_allreduce_fused_add_rms_norm. The first call on a device
- * looks the array up (the device must be current, as for every call), and
- * the first call with a given `world` after another clears the signal pads
- * with cudaMemsetAsync on `stream`: make those calls outside stream capture
- * (RN_ERR_CONFIG inside); later calls may be captured. The memory is shared
- * by every call on a device: calls that overlap in time (other streams,
- * other threads) race and give undefined results. */
+ * errors of rn_allreduce_fused_add_rms_norm, with the AUTO algorithm (buffers
+ * sized for two-shot when world * round_up(12 * T * H + 32, 256) fits). The
+ * first call on a device looks the array up (the device must be current, as
+ * for every call), and the first call with a given `world` after another
+ * clears the signal pads with cudaMemsetAsync on `stream`: make those calls
+ * outside stream capture (RN_ERR_CONFIG inside); later calls may be
+ * captured. The memory is shared by every call on a device: calls that
+ * overlap in time (other streams, other threads) race and give undefined
+ * results. */
 #define RN_LOCAL_EXCHANGE_BYTES 33554432
 RN_API rn_status rn_allreduce_fused_add_rms_norm_local(const rn_tensor* out, const rn_tensor* x,
                                                        const rn_tensor* residual,
@@ -367,8 +386,11 @@ RN_API rn_status rn_validate(int32_t op, const rn_tensor* out_or_q, const rn_ten
  * and vectors_per_thread one of the compiled widths (see
  * rn_supported_vectors_per_thread); otherwise RN_ERR_CONFIG. A forced shape
  * that cannot cover a row (threads_per_row * vectors_per_thread * 8 < H) or
- * exceeds the kernel's block limit falls back to the scalar kernel. Not
- * thread-safe with concurrent launches; meant for tests and tuning. */
+ * exceeds the kernel's block limit falls back to the scalar kernel. The
+ * all-reduce kernels take a forced (threads_per_row, vectors_per_thread)
+ * too when threads_per_row is a power of two <= 512, vectors_per_thread is
+ * 1, 2, 4 or 8 and together they cover a row. Not thread-safe with
+ * concurrent launches; meant for tests and tuning. */
 RN_API rn_status rn_force_plan(int32_t threads_per_row, int32_t vectors_per_thread,
                                 int32_t rows_per_cta);
 

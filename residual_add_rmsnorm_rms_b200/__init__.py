@@ -27,7 +27,8 @@ __all__ = [
     "silu_and_mul_fp8", "fp8_rowwise_gemm", "fp8_gemm_config", "fp8_gemm_force_config",
     "GEMM_CONFIGS", "allreduce_fused_add_rms_norm", "allreduce_fused_add_rms_norm_fp8",
     "allreduce_fused_add_rms_norm_local",
-    "RnAllreduceComm", "ALLREDUCE_MAX_WORLD", "ALLREDUCE_SIGNAL_BYTES", "plan_launch", "validate", "force_plan", "force_staged",
+    "RnAllreduceComm", "ALLREDUCE_MAX_WORLD", "ALLREDUCE_SIGNAL_BYTES", "ALLREDUCE_ALGORITHMS",
+    "plan_launch", "validate", "force_plan", "force_staged",
     "set_launch_options", "device_errors", "supported_vectors_per_thread", "status_string",
     "LIB_PATH", "lib", "RnTensor", "RnPlan", "STATUS", "OPS",
 ]
@@ -46,7 +47,8 @@ _DTYPES = {torch.float16: 0, torch.bfloat16: 1, torch.float8_e4m3fn: 2, torch.fl
 
 
 ALLREDUCE_MAX_WORLD = 8
-ALLREDUCE_SIGNAL_BYTES = 65600
+ALLREDUCE_SIGNAL_BYTES = 131136
+ALLREDUCE_ALGORITHMS = {"auto": 0, "one_shot": 1, "two_shot": 2}
 
 
 class RnAllreduceComm(ctypes.Structure):
@@ -55,6 +57,7 @@ class RnAllreduceComm(ctypes.Structure):
         ("world", ctypes.c_int32),
         ("rank", ctypes.c_int32),
         ("local_ranks", ctypes.c_int32),
+        ("algorithm", ctypes.c_int32),
         ("buffers", ctypes.c_void_p * ALLREDUCE_MAX_WORLD),
         ("signals", ctypes.c_void_p * ALLREDUCE_MAX_WORLD),
         ("buffer_bytes", ctypes.c_int64),

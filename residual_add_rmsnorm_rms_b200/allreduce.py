@@ -17,8 +17,9 @@ numbered). Two ways to build one:
   (``all_gather_object``), then map their peers' buffers.
 
 Buffers are sized for at most ``max_rows`` rows of ``hidden`` 16-bit values
-per call (two halves, alternated by call parity). Pads start zero-filled.
-Every rank of a group must make the same sequence of calls.
+per call (two halves, alternated by call parity), with room for the two-shot
+algorithm unless ``algorithm="one_shot"``. Pads start zero-filled. Every rank
+of a group must make the same sequence of calls with the same algorithm.
 """
 from __future__ import annotations
 
@@ -29,7 +30,7 @@ from typing import Optional, Sequence
 
 import torch
 
-from . import ALLREDUCE_MAX_WORLD, ALLREDUCE_SIGNAL_BYTES, RnAllreduceComm
+from . import ALLREDUCE_ALGORITHMS, ALLREDUCE_MAX_WORLD, ALLREDUCE_SIGNAL_BYTES, RnAllreduceComm
 
 __all__ = ["AllReduceComm", "buffer_bytes_for", "exchange_records", "lookup"]
 
@@ -44,9 +45,10 @@ def lookup(handle: int) -> "AllReduceComm":
     return _LIVE[handle]
 
 
-def buffer_bytes_for(max_rows: int, hidden: int) -> int:
-    """Exchange-buffer size for calls of up to max_rows x hidden 16-bit values."""
-    return 4 * max_rows * hidden + 32
+def buffer_bytes_for(max_rows: int, hidden: int, two_shot: bool = True) -> int:
+    """Exchange-buffer size for calls of up to max_rows x hidden 16-bit values:
+    two halves of T*H values (one-shot) or of 3*T*H values (two-shot too)."""
+    return (12 if two_shot else 4) * max_rows * hidden + 32
 
 
 def exchange_records(record: dict, group=None) -> list[dict]:
@@ -60,7 +62,7 @@ def exchange_records(record: dict, group=None) -> list[dict]:
     for p, rec in enumerate(gathered):
         if rec.get("rank") != p:
             raise ValueError(f"record {p} comes from rank {rec.get('rank')}")
-        for key in ("buffer_bytes", "max_rows", "hidden", "world"):
+        for key in ("buffer_bytes", "max_rows", "hidden", "world", "algorithm"):
             if rec.get(key) != gathered[0].get(key):
                 raise ValueError(f"ranks disagree on {key}: rank 0 has {gathered[0].get(key)}, "
                                  f"rank {p} has {rec.get(key)}")
@@ -73,7 +75,8 @@ class AllReduceComm:
 
     def __init__(self, world: int, rank: int, local_ranks: int, buffers: Sequence[int],
                  signals: Sequence[int], buffer_bytes: int, timeout_s: float = 1.0,
-                 keepalive: Sequence = (), local_pads: Sequence[torch.Tensor] = ()):
+                 keepalive: Sequence = (), local_pads: Sequence[torch.Tensor] = (),
+                 algorithm: str = "auto"):
         if not 1 <= world <= ALLREDUCE_MAX_WORLD:
             raise ValueError(f"world must be 1..{ALLREDUCE_MAX_WORLD}")
         if len(buffers) != world or len(signals) != world:
@@ -82,10 +85,12 @@ class AllReduceComm:
         self.buffers, self.signals = list(buffers), list(signals)
         self.buffer_bytes = int(buffer_bytes)
         self.timeout_ns = int(timeout_s * 1e9)
+        self.algorithm = algorithm
         self._keepalive = list(keepalive)
         self._local_pads = list(local_pads)
         d = RnAllreduceComm()
         d.world, d.rank, d.local_ranks = world, rank, local_ranks
+        d.algorithm = ALLREDUCE_ALGORITHMS[algorithm]
         for p in range(world):
             d.buffers[p] = self.buffers[p]
             d.signals[p] = self.signals[p]
@@ -98,7 +103,7 @@ class AllReduceComm:
 
     @property
     def max_elements(self) -> int:
-        """Largest T * H one call may carry."""
+        """Largest T * H one one-shot call may carry (a third of it two-shot)."""
         return ((self.buffer_bytes // 2) & ~15) // 2
 
     def descriptor(self) -> RnAllreduceComm:
@@ -115,25 +120,27 @@ class AllReduceComm:
 
     @classmethod
     def single_device(cls, world: int, max_rows: int, hidden: int, device,
-                      timeout_s: float = 1.0) -> "AllReduceComm":
-        nbytes = buffer_bytes_for(max_rows, hidden)
+                      timeout_s: float = 1.0, algorithm: str = "auto") -> "AllReduceComm":
+        nbytes = buffer_bytes_for(max_rows, hidden, algorithm != "one_shot")
         bufs = [torch.zeros(nbytes, dtype=torch.uint8, device=device) for _ in range(world)]
         pads = [torch.zeros(ALLREDUCE_SIGNAL_BYTES, dtype=torch.uint8, device=device)
                 for _ in range(world)]
         return cls(world, 0, world, [b.data_ptr() for b in bufs], [p.data_ptr() for p in pads],
-                   nbytes, timeout_s, keepalive=bufs + pads, local_pads=pads)
+                   nbytes, timeout_s, keepalive=bufs + pads, local_pads=pads,
+                   algorithm=algorithm)
 
     @classmethod
     def from_process_group(cls, max_rows: int, hidden: int, device, group=None,
-                           timeout_s: float = 1.0) -> "AllReduceComm":
+                           timeout_s: float = 1.0, algorithm: str = "auto") -> "AllReduceComm":
         import torch.distributed as dist
         world, rank = dist.get_world_size(group), dist.get_rank(group)
-        nbytes = buffer_bytes_for(max_rows, hidden)
+        nbytes = buffer_bytes_for(max_rows, hidden, algorithm != "one_shot")
         buf = torch.zeros(nbytes, dtype=torch.uint8, device=device)
         pad = torch.zeros(ALLREDUCE_SIGNAL_BYTES, dtype=torch.uint8, device=device)
         torch.cuda.synchronize(device)  # zeros in place before any peer maps them
         mine = {"rank": rank, "world": world, "buffer_bytes": nbytes, "max_rows": max_rows,
-                "hidden": hidden, "buffer": _export(buf), "signal": _export(pad)}
+                "hidden": hidden, "algorithm": algorithm, "buffer": _export(buf),
+                "signal": _export(pad)}
         records = exchange_records(mine, group)
         keep = [buf, pad]
         bufs, pads = [], []
@@ -147,7 +154,8 @@ class AllReduceComm:
             bufs.append(b.data_ptr())
             pads.append(s.data_ptr())
         dist.barrier(group)  # every rank has mapped every buffer
-        return cls(world, rank, 1, bufs, pads, nbytes, timeout_s, keepalive=keep, local_pads=[pad])
+        return cls(world, rank, 1, bufs, pads, nbytes, timeout_s, keepalive=keep, local_pads=[pad],
+                   algorithm=algorithm)
 
 
 def _export(t: torch.Tensor) -> tuple:

@@ -75,11 +75,11 @@ __device__ unsigned int g_rn_ar_error = 0;
 constexpr unsigned kErrPeerTimeout = 2u;
 
 // Signal pad layout, in 32-bit words: the call counter, the arrival counter,
-// padding to 64 bytes, then flags [2][kArMaxBlocks][kArMaxWorld].
+// padding to 64 bytes, then flags [2 parities][2 stages][kArMaxBlocks][kArMaxWorld].
 constexpr int kPadEpoch = 0;
 constexpr int kPadArrived = 1;
 constexpr int kPadFlags = 16;
-static_assert((kPadFlags + 2 * kArMaxBlocks * kArMaxWorld) * 4 == kArSignalBytes,
+static_assert((kPadFlags + 4 * kArMaxBlocks * kArMaxWorld) * 4 == kArSignalBytes,
               "signal pad size");
 
 __device__ __forceinline__ uint4 ld_volatile_v4(const uint4* p) {
@@ -89,6 +89,60 @@ __device__ __forceinline__ uint4 ld_volatile_v4(const uint4* p) {
                  : "l"(p)
                  : "memory");
     return v;
+}
+
+__device__ __forceinline__ uint2 ld_volatile_v2(const uint2* p) {
+    uint2 v;
+    asm volatile("ld.volatile.global.v2.u32 {%0, %1}, [%2];"
+                 : "=r"(v.x), "=r"(v.y)
+                 : "l"(p)
+                 : "memory");
+    return v;
+}
+
+__device__ __forceinline__ uint4 ld_copy(const uint4* p, bool exchange) {
+    return exchange ? ld_volatile_v4(p) : ld_stream(p);
+}
+__device__ __forceinline__ uint2 ld_copy(const uint2* p, bool) { return ld_volatile_v2(p); }
+__device__ __forceinline__ void st_copy(uint4* p, const uint4& v) { st_v4(p, v); }
+__device__ __forceinline__ void st_copy(uint2* p, const uint2& v) { st_v2(p, v); }
+
+// Copies the rows [s0, s1) this block owns (row groups of rpc rows,
+// block-strided: the mapping of the reduce step) from src to dst, as `nvec`
+// vectors per row (16 bytes for 16-bit rows, 8 for e4m3 rows). Thread
+// (row, lr) moves vectors lr, lr + tpr, ... of its row, U row groups at a
+// time, all loads before any store, so a thread keeps U * VPT loads in
+// flight. `exchange` selects volatile loads (memory other ranks write).
+template <int VPT, typename V>
+__device__ __forceinline__ void copy_rows(V* dst, const V* src, const int64_t s0,
+                                          const int64_t s1, const int tpr, const int rpc,
+                                          const int nvec, const bool exchange) {
+    constexpr int U = VPT >= 4 ? 1 : 4 / VPT;
+    const int row_in_cta = threadIdx.x / tpr;
+    const int lr = threadIdx.x - row_in_cta * tpr;
+    const int64_t stride = static_cast<int64_t>(gridDim.x) * rpc;
+    for (int64_t base = s0 + static_cast<int64_t>(blockIdx.x) * rpc; base < s1;
+         base += U * stride) {
+        V v[U][VPT];
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t row = base + u * stride + row_in_cta;
+#pragma unroll
+            for (int k = 0; k < VPT; ++k) {
+                const int j = lr + k * tpr;
+                if (row < s1 && j < nvec) v[u][k] = ld_copy(src + row * nvec + j, exchange);
+            }
+        }
+#pragma unroll
+        for (int u = 0; u < U; ++u) {
+            const int64_t row = base + u * stride + row_in_cta;
+#pragma unroll
+            for (int k = 0; k < VPT; ++k) {
+                const int j = lr + k * tpr;
+                if (row < s1 && j < nvec) st_copy(dst + row * nvec + j, v[u][k]);
+            }
+        }
+    }
 }
 
 __device__ __forceinline__ void st_release_sys(uint32_t* p, uint32_t v) {
@@ -149,28 +203,53 @@ __device__ __forceinline__ uint4 sum8(const uint4 (&pv)[kW], int W) {
     }
 }
 
-// Step 4 for the rows of this block: reduce + residual add + RMSNorm (+ FP8),
-// rows mapped as in the vector kernel.
-template <typename T, int VPT, int kW, bool kFp8, bool kHasW>
+// Byte offsets inside one buffer half (T x H 16-bit values per region): the
+// partial (both algorithms), then, for the two-shot algorithm, the finished
+// residual rows and the finished output rows (16-bit out, or e4m3 codes
+// followed by the T fp32 scales).
+struct SlotLayout {
+    int64_t partial, residual2, out2, scale2;
+    __device__ explicit SlotLayout(const ArArgs& a) {
+        const int64_t th2 = a.T * a.H * 2;
+        partial = 0;
+        residual2 = th2;
+        out2 = 2 * th2;
+        scale2 = 2 * th2 + a.T * a.H;
+    }
+};
+
+__device__ __forceinline__ char* slot_base(const ArArgs& a, int p, uint32_t epoch) {
+    return static_cast<char*>(a.buffers[p]) + static_cast<int64_t>(epoch & 1u) * a.slot_elems * 2;
+}
+
+// Step 4 for the rows [s0, s1) this block owns in that range (row groups of
+// rpc rows, block-strided, as in the vector kernel): reduce + residual add +
+// RMSNorm (+ FP8) into this rank's outputs; with kStage2 (two-shot) the
+// finished rows are also written to this rank's buffer for the other ranks.
+template <typename T, int VPT, int kW, bool kFp8, bool kHasW, bool kStage2>
 __device__ __forceinline__ void reduce_rows(const ArArgs& a, const int tpr, const int rpc,
-                                            float2* red, const int ly, const uint32_t epoch,
-                                            const int nvec, const int64_t local) {
+                                            float2* red, const int ly, const int rank,
+                                            const uint32_t epoch, const int nvec,
+                                            const int64_t local, const int64_t s0,
+                                            const int64_t s1) {
     const int W = a.world;
+    const SlotLayout lay(a);
     const int64_t slot = static_cast<int64_t>(epoch & 1u) * (a.slot_elems >> 3);
     const uint4* __restrict__ wv = static_cast<const uint4*>(a.weight);
     const float hf = static_cast<float>(a.H);
     const uint4* peer[kW];
 #pragma unroll
     for (int p = 0; p < kW; ++p)
-        peer[p] = static_cast<const uint4*>(a.buffers[p < W ? p : 0]) + slot;
+        peer[p] = static_cast<const uint4*>(a.buffers[p < W ? p : 0]) + slot;  // partials at 0
     const int row_in_cta = threadIdx.x / tpr;
     const int lr = threadIdx.x - row_in_cta * tpr;
     const int wpr = tpr >> 5;
+    char* const mine = slot_base(a, rank, epoch);
     int parity = 0;
-    for (int64_t base = static_cast<int64_t>(blockIdx.x) * rpc; base < a.T;
+    for (int64_t base = s0 + static_cast<int64_t>(blockIdx.x) * rpc; base < s1;
          base += static_cast<int64_t>(gridDim.x) * rpc) {
         const int64_t row = base + row_in_cta;
-        const bool active = row < a.T;
+        const bool active = row < s1;
         const int64_t roff = (active ? row : 0) * nvec;
         uint4* rrow = static_cast<uint4*>(a.residual) + local + roff;
 
@@ -200,7 +279,11 @@ __device__ __forceinline__ void reduce_rows(const ArArgs& a, const int tpr, cons
         for (int k = 0; k < VPT; ++k) {
             const int j = lr + k * tpr;
             v[k] = add8<T>(v[k], r[k]);
-            if (active && j < nvec) st_v4(rrow + j, v[k]);
+            if (active && j < nvec) {
+                st_v4(rrow + j, v[k]);
+                if constexpr (kStage2)
+                    st_v4(reinterpret_cast<uint4*>(mine + lay.residual2) + roff + j, v[k]);
+            }
             acc = ssq8<T>(v[k], acc);
             if constexpr (kFp8) {
                 uint4 w = make_uint4(0, 0, 0, 0);
@@ -241,13 +324,18 @@ __device__ __forceinline__ void reduce_rows(const ArArgs& a, const int tpr, cons
                 if (!(active && j < nvec)) continue;
                 uint4 w = make_uint4(0, 0, 0, 0);
                 if constexpr (kHasW) w = __ldg(wv + j);
-                st_v4(orow + j, scale8<T, kHasW>(v[k], w, inv2));
+                const uint4 o = scale8<T, kHasW>(v[k], w, inv2);
+                st_v4(orow + j, o);
+                if constexpr (kStage2) st_v4(reinterpret_cast<uint4*>(mine + lay.out2) + roff + j, o);
             }
         } else {
             const float qmul = pm > 0.f ? 448.0f / pm : 0.f;
             const float2 q2 = make_float2(qmul, qmul);
-            if (active && lr == 0)
-                a.scale[static_cast<int64_t>(ly) * a.T + row] = pm > 0.f ? (pm * inv) / 448.0f : 0.f;
+            if (active && lr == 0) {
+                const float sc = pm > 0.f ? (pm * inv) / 448.0f : 0.f;
+                a.scale[static_cast<int64_t>(ly) * a.T + row] = sc;
+                if constexpr (kStage2) reinterpret_cast<float*>(mine + lay.scale2)[row] = sc;
+            }
             uint2* qrow = reinterpret_cast<uint2*>(a.q) + local + roff;
 #pragma unroll
             for (int k = 0; k < VPT; ++k) {
@@ -258,48 +346,56 @@ __device__ __forceinline__ void reduce_rows(const ArArgs& a, const int tpr, cons
                 uint2 o = quant8<T, kHasW>(v[k], w, q2);
                 if (!(pm > 0.f)) o = make_uint2(0, 0);
                 st_v2(qrow + j, o);
+                if constexpr (kStage2) st_v2(reinterpret_cast<uint2*>(mine + lay.out2) + roff + j, o);
             }
         }
     }
 }
 
-template <typename T, int VPT, int kW, bool kFp8, bool kHasW>
-__device__ __forceinline__ void allreduce_rows(const ArArgs& a, const int tpr, const int rpc,
-                                               float2* red) {
-    const int ly = blockIdx.y;
-    const int rank = a.rank + ly;
-    const int W = a.world;
-    const int nvec = static_cast<int>(a.H >> 3);
-    const int64_t local = static_cast<int64_t>(ly) * a.T * nvec;  // in 16-byte vectors
-    uint32_t* const pad = a.signals[rank];
-    uint32_t epoch = *reinterpret_cast<volatile uint32_t*>(pad + kPadEpoch) + 1u;
-    if (epoch == 0) epoch = 1;
-    const int64_t slot = static_cast<int64_t>(epoch & 1u) * (a.slot_elems >> 3);
-
-    // 1. this block's rows of the local partial into this rank's buffer
-    {
-        const uint4* x = static_cast<const uint4*>(a.x) + local;
-        uint4* mine = static_cast<uint4*>(a.buffers[rank]) + slot;
-        for (int64_t base = static_cast<int64_t>(blockIdx.x) * rpc; base < a.T;
-             base += static_cast<int64_t>(gridDim.x) * rpc) {
-            const int64_t v0 = base * nvec;
-            const int64_t v1 = (base + rpc < a.T ? base + rpc : a.T) * nvec;
-#pragma unroll 4
-            for (int64_t i = v0 + threadIdx.x; i < v1; i += blockDim.x) st_v4(mine + i, ld_stream(x + i));
-        }
+// Two-shot step 6: copy the finished rows [s0, s1) that rank `owner` wrote
+// into its buffer (this block's share of them) into this rank's outputs.
+template <int VPT, bool kFp8>
+__device__ __forceinline__ void gather_rows(const ArArgs& a, const int tpr, const int rpc,
+                                            const int owner, const uint32_t epoch,
+                                            const int nvec, const int64_t local,
+                                            const int64_t s0, const int64_t s1) {
+    const SlotLayout lay(a);
+    const char* src = slot_base(a, owner, epoch);
+    copy_rows<VPT>(static_cast<uint4*>(a.residual) + local,
+                   reinterpret_cast<const uint4*>(src + lay.residual2), s0, s1, tpr, rpc, nvec,
+                   true);
+    if constexpr (!kFp8) {
+        copy_rows<VPT>(static_cast<uint4*>(a.out) + local,
+                       reinterpret_cast<const uint4*>(src + lay.out2), s0, s1, tpr, rpc, nvec,
+                       true);
+    } else {
+        copy_rows<VPT>(reinterpret_cast<uint2*>(a.q) + local,
+                       reinterpret_cast<const uint2*>(src + lay.out2), s0, s1, tpr, rpc, nvec,
+                       true);
+        const volatile float* sc2 = reinterpret_cast<const volatile float*>(src + lay.scale2);
+        const int64_t stride = static_cast<int64_t>(gridDim.x) * rpc;
+        for (int64_t base = s0 + static_cast<int64_t>(blockIdx.x) * rpc; base < s1; base += stride)
+            for (int64_t r = base + threadIdx.x; r < base + rpc && r < s1; r += blockDim.x)
+                a.scale[static_cast<int64_t>(blockIdx.y) * a.T + r] = sc2[r];
     }
-    __syncthreads();
+}
 
-    // 2. publish, 3. wait for every rank's copy of the same rows
-    const int flag0 = kPadFlags + ((epoch & 1u) * kArMaxBlocks + blockIdx.x) * kArMaxWorld;
-    // The barrier above orders every thread's copy before the release
-    // stores, and a system-scope release orders everything that happens
-    // before it: no separate fence is needed. Thread p publishes to rank p,
-    // so the W releases proceed in parallel.
+// Publishes this block's stage `stage` of call `epoch` to every rank, then
+// waits (bounded) for the same block of every rank. The barrier first orders
+// every thread's prior writes before the release stores, and a system-scope
+// release orders everything that happens before it: no separate fence is
+// needed. Thread p publishes to and waits for rank p, so the W releases and
+// polls proceed in parallel. Returns true (on every thread) when a wait ran out.
+__device__ __forceinline__ bool exchange_barrier(const ArArgs& a, const int rank,
+                                                 const uint32_t epoch, const int stage) {
+    const int W = a.world;
+    const int flag0 =
+        kPadFlags + (((epoch & 1u) * 2 + stage) * kArMaxBlocks + blockIdx.x) * kArMaxWorld;
+    __syncthreads();
     if (threadIdx.x < W) st_release_sys(a.signals[threadIdx.x] + flag0 + rank, epoch);
     bool late = false;
     if (threadIdx.x < W) {
-        const uint32_t* f = pad + flag0 + threadIdx.x;
+        const uint32_t* f = a.signals[rank] + flag0 + threadIdx.x;
         if (ld_acquire_sys(f) != epoch) {
             const unsigned long long t0 = global_ns();
             while (ld_acquire_sys(f) != epoch) {
@@ -311,13 +407,61 @@ __device__ __forceinline__ void allreduce_rows(const ArArgs& a, const int tpr, c
             }
         }
     }
-    if (__syncthreads_or(late)) {
-        if (threadIdx.x == 0) atomicOr(&g_rn_ar_error, kErrPeerTimeout);
-    } else {
-        reduce_rows<T, VPT, kW, kFp8, kHasW>(a, tpr, rpc, red, ly, epoch, nvec, local);
+    return __syncthreads_or(late) != 0;
+}
+
+template <typename T, int VPT, int kW, bool kFp8, bool kHasW, bool kTwoShot>
+__device__ __forceinline__ void allreduce_rows(const ArArgs& a, const int tpr, const int rpc,
+                                               float2* red) {
+    const int ly = blockIdx.y;
+    const int rank = a.rank + ly;
+    const int W = a.world;
+    const int nvec = static_cast<int>(a.H >> 3);
+    const int64_t local = static_cast<int64_t>(ly) * a.T * nvec;  // in 16-byte vectors
+    uint32_t* const pad = a.signals[rank];
+    uint32_t epoch = *reinterpret_cast<volatile uint32_t*>(pad + kPadEpoch) + 1u;
+    if (epoch == 0) epoch = 1;
+    // two-shot: rank q owns the rows [q * S, (q + 1) * S)
+    const int64_t S = kTwoShot ? (a.T + W - 1) / W : a.T;
+
+    // 1. this block's rows of the local partial into this rank's buffer: the
+    //    block's share of every slice, so that block b of the slice's owner
+    //    waits only for block b of each rank
+    {
+        const uint4* x = static_cast<const uint4*>(a.x) + local;
+        uint4* mine = reinterpret_cast<uint4*>(slot_base(a, rank, epoch));
+        for (int q = 0; q < (kTwoShot ? W : 1); ++q) {
+            const int64_t s0 = q * S, s1 = s0 + S < a.T ? s0 + S : a.T;
+            copy_rows<VPT>(mine, x, s0 < a.T ? s0 : a.T, s1, tpr, rpc, nvec, false);
+        }
     }
 
-    // 5. arrival; the last block of this rank advances the call counter
+    // 2.-3. publish and wait for every rank's copy of the same rows
+    bool late = exchange_barrier(a, rank, epoch, 0);
+    if (!late) {
+        if constexpr (!kTwoShot) {
+            // 4. reduce + finish every row
+            reduce_rows<T, VPT, kW, kFp8, kHasW, false>(a, tpr, rpc, red, ly, rank, epoch, nvec,
+                                                        local, 0, a.T);
+        } else {
+            // 4. reduce + finish this rank's slice, also into its buffer;
+            // 5. publish and wait; 6. copy every other slice from its owner
+            const int64_t s0 = rank * S, s1 = s0 + S < a.T ? s0 + S : a.T;
+            reduce_rows<T, VPT, kW, kFp8, kHasW, true>(a, tpr, rpc, red, ly, rank, epoch, nvec,
+                                                       local, s0 < a.T ? s0 : a.T, s1);
+            late = exchange_barrier(a, rank, epoch, 1);
+            if (!late) {
+                for (int q = 0; q < W; ++q) {
+                    if (q == rank) continue;
+                    const int64_t g0 = q * S, g1 = g0 + S < a.T ? g0 + S : a.T;
+                    if (g0 < a.T) gather_rows<VPT, kFp8>(a, tpr, rpc, q, epoch, nvec, local, g0, g1);
+                }
+            }
+        }
+    }
+    if (late && threadIdx.x == 0) atomicOr(&g_rn_ar_error, kErrPeerTimeout);
+
+    // 7. arrival; the last block of this rank advances the call counter
     __syncthreads();
     if (threadIdx.x == 0) {
         __threadfence();
@@ -328,44 +472,52 @@ __device__ __forceinline__ void allreduce_rows(const ArArgs& a, const int tpr, c
     }
 }
 
-template <typename T, int VPT, int kW, bool kFp8>
+template <typename T, int VPT, int kW, bool kFp8, bool kTwoShot>
 __global__ void __launch_bounds__(kArMaxBlock)
     rn_allreduce_kernel(const ArArgs a, const int tpr, const int rpc) {
     extern __shared__ float2 red[];  // [2][rpc][warps per row]
     if (a.weight)
-        allreduce_rows<T, VPT, kW, kFp8, true>(a, tpr, rpc, red);
+        allreduce_rows<T, VPT, kW, kFp8, true, kTwoShot>(a, tpr, rpc, red);
     else
-        allreduce_rows<T, VPT, kW, kFp8, false>(a, tpr, rpc, red);
+        allreduce_rows<T, VPT, kW, kFp8, false, kTwoShot>(a, tpr, rpc, red);
 }
 
 using ArKernel = void (*)(const ArArgs, const int, const int);
 
-template <typename T, int kW, bool kFp8>
+template <typename T, int kW, bool kFp8, bool kTwoShot>
 ArKernel pick_vpt(int vpt) {
     switch (vpt) {
-        case 1: return rn_allreduce_kernel<T, 1, kW, kFp8>;
-        case 2: return rn_allreduce_kernel<T, 2, kW, kFp8>;
-        case 4: return rn_allreduce_kernel<T, 4, kW, kFp8>;
-        case 8: return rn_allreduce_kernel<T, 8, kW, kFp8>;
+        case 1: return rn_allreduce_kernel<T, 1, kW, kFp8, kTwoShot>;
+        case 2: return rn_allreduce_kernel<T, 2, kW, kFp8, kTwoShot>;
+        case 4: return rn_allreduce_kernel<T, 4, kW, kFp8, kTwoShot>;
+        case 8: return rn_allreduce_kernel<T, 8, kW, kFp8, kTwoShot>;
         default: return nullptr;
     }
 }
 
+// Two-shot kernels exist for groups of 3 to 8 ranks (it moves more data than
+// one-shot with two ranks).
 template <typename T, bool kFp8>
-ArKernel pick_w(int world, int vpt) {
-    if (world == 1) return pick_vpt<T, 1, kFp8>(vpt);
-    if (world == 2) return pick_vpt<T, 2, kFp8>(vpt);
-    if (world <= 4) return pick_vpt<T, 4, kFp8>(vpt);
-    return pick_vpt<T, 8, kFp8>(vpt);
+ArKernel pick_w(int world, int vpt, bool two_shot) {
+    if (two_shot) {
+        if (world < 3) return nullptr;
+        if (world <= 4) return pick_vpt<T, 4, kFp8, true>(vpt);
+        return pick_vpt<T, 8, kFp8, true>(vpt);
+    }
+    if (world == 1) return pick_vpt<T, 1, kFp8, false>(vpt);
+    if (world == 2) return pick_vpt<T, 2, kFp8, false>(vpt);
+    if (world <= 4) return pick_vpt<T, 4, kFp8, false>(vpt);
+    return pick_vpt<T, 8, kFp8, false>(vpt);
 }
 
-ArKernel pick(int dtype, bool fp8, int world, int vpt) {
+ArKernel pick(int dtype, bool fp8, int world, int vpt, bool two_shot) {
     if (world < 1 || world > kArMaxWorld) return nullptr;
     if (dtype == kBF16)
-        return fp8 ? pick_w<__nv_bfloat16, true>(world, vpt)
-                   : pick_w<__nv_bfloat16, false>(world, vpt);
+        return fp8 ? pick_w<__nv_bfloat16, true>(world, vpt, two_shot)
+                   : pick_w<__nv_bfloat16, false>(world, vpt, two_shot);
     if (dtype == kF16)
-        return fp8 ? pick_w<__half, true>(world, vpt) : pick_w<__half, false>(world, vpt);
+        return fp8 ? pick_w<__half, true>(world, vpt, two_shot)
+                   : pick_w<__half, false>(world, vpt, two_shot);
     return nullptr;
 }
 
@@ -373,7 +525,7 @@ ArKernel pick(int dtype, bool fp8, int world, int vpt) {
 
 cudaError_t allreduce_blocks_per_sm(int dtype, bool fp8, int world, const ArLaunch& l,
                                     int* blocks) {
-    const ArKernel k = pick(dtype, fp8, world, l.vpt);
+    const ArKernel k = pick(dtype, fp8, world, l.vpt, l.two_shot);
     if (!k) return cudaErrorInvalidValue;
     return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks, k, l.block,
                                                          static_cast<size_t>(l.smem));
@@ -381,7 +533,7 @@ cudaError_t allreduce_blocks_per_sm(int dtype, bool fp8, int world, const ArLaun
 
 cudaError_t launch_allreduce(int dtype, bool fp8, const ArArgs& a, const ArLaunch& l,
                              cudaStream_t s) {
-    const ArKernel k = pick(dtype, fp8, a.world, l.vpt);
+    const ArKernel k = pick(dtype, fp8, a.world, l.vpt, l.two_shot);
     if (!k) return cudaErrorInvalidValue;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(l.grid_x), static_cast<unsigned>(l.local_ranks));

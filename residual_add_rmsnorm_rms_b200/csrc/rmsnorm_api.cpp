@@ -635,27 +635,46 @@ bool overlaps_bytes(const Flat& f, const void* p, int64_t bytes) {
 }
 
 // Row mapping of the all-reduce kernel: a power-of-two group of threads per
-// row holding v vectors of 16 bytes each, v chosen so that a thread keeps
-// about 128 bytes of loads in flight (v = 8 / (W + 1) rounded down to a power
-// of two, at least 1: each vector costs W exchange loads and one residual
-// load), up to the 512-thread block (then 2, 4 or 8 vectors each);
-// 256-thread blocks of several rows for narrow rows.
-rn_status ar_shape(int64_t H, int world, rn::ArLaunch* l) {
+// row holding two 16-byte vectors each (up to the 512-thread block, then 4 or
+// 8), 256-thread blocks of several rows for narrow rows. Measured on B200 for
+// H = 3840 and 2, 4 and 8 ranks at T = 8192, two vectors per thread is the
+// fastest of 1, 2, 4 and 8 for both algorithms (by 3 to 35 %): fewer leave too
+// few loads in flight, more cost resident warps.
+rn_status ar_shape(int64_t H, rn::ArLaunch* l) {
     const int64_t nvec = H / 8;
-    int target = 1;
-    while (target * 2 <= 8 / (world + 1)) target *= 2;
-    int tpr = 1;
-    while (static_cast<int64_t>(tpr) * target < nvec && tpr < rn::kArMaxBlock) tpr *= 2;
-    const int64_t need = (nvec + tpr - 1) / tpr;
-    int vpt = 1;
-    while (vpt < need) vpt *= 2;
-    if (vpt > 8) return RN_ERR_SHAPE;
+    int tpr = 1, vpt = 1;
+    const int ftpr = g_force_tpr.load(), fvpt = g_force_vpt.load();
+    if (ftpr > 0 && (ftpr & (ftpr - 1)) == 0 && ftpr <= rn::kArMaxBlock &&
+        (fvpt == 1 || fvpt == 2 || fvpt == 4 || fvpt == 8) &&
+        static_cast<int64_t>(ftpr) * fvpt >= nvec) {
+        tpr = ftpr;  // a forced vector-kernel shape that suits this kernel too
+        vpt = fvpt;
+    } else {
+        const int target = 2;
+        while (static_cast<int64_t>(tpr) * target < nvec && tpr < rn::kArMaxBlock) tpr *= 2;
+        const int64_t need = (nvec + tpr - 1) / tpr;
+        while (vpt < need) vpt *= 2;
+        if (vpt > 8) return RN_ERR_SHAPE;
+    }
     l->tpr = tpr;
     l->vpt = vpt;
     l->rpc = tpr >= 256 ? 1 : 256 / tpr;
     l->block = tpr * l->rpc;
     l->smem = static_cast<int>(2 * l->rpc * (tpr >= 64 ? tpr / 32 : 1) * sizeof(float) * 2);
     return RN_OK;
+}
+
+// Automatic choice of the two-shot algorithm: each rank reads (W - 1) * 2TH
+// bytes from its peers in one-shot and (W - 1) / W * 6TH in two-shot (its
+// slice's partials, then the other slices' finished residual and output rows),
+// at the cost of a second exchange barrier (a few microseconds). Two-shot is
+// taken from four ranks on, once it saves at least 2.3 MB of peer reads per
+// rank: about 3 us at the 770 GB/s a B200 peer copy reaches over NVLink.
+bool ar_two_shot_pays(int W, int64_t T, int64_t H) {
+    if (W < 4) return false;
+    const double th = static_cast<double>(T) * static_cast<double>(H);
+    const double saved = (W - 1) * 2.0 * th - (W - 1) * 6.0 * th / W;
+    return saved >= 2.3e6;
 }
 
 rn_status check_comm(const rn_allreduce_comm* comm) {
@@ -686,8 +705,15 @@ rn_status run_allreduce(bool fp8, const rn_tensor* o, const rn_tensor* sc, const
     if (H > kArMaxH) return RN_ERR_SHAPE;
     const int64_t slot_bytes = (comm->buffer_bytes / 2) & ~static_cast<int64_t>(15);
     if (comm->buffer_bytes < 0 || slot_bytes < 2 * T * H) return RN_ERR_COMM;
+    if (comm->algorithm < RN_ALLREDUCE_AUTO || comm->algorithm > RN_ALLREDUCE_TWO_SHOT)
+        return RN_ERR_COMM;
+    const bool two_shot_fits = comm->world >= 3 && slot_bytes >= 6 * T * H;
+    if (comm->algorithm == RN_ALLREDUCE_TWO_SHOT && !two_shot_fits) return RN_ERR_COMM;
     rn::ArLaunch l;
-    if ((st = ar_shape(H, comm->world, &l)) != RN_OK) return st;
+    if ((st = ar_shape(H, &l)) != RN_OK) return st;
+    l.two_shot = comm->algorithm == RN_ALLREDUCE_TWO_SHOT ||
+                 (comm->algorithm == RN_ALLREDUCE_AUTO && two_shot_fits &&
+                  ar_two_shot_pays(comm->world, T, H));
     if (T > 0) {
         rn_plan unused;
         if ((st = check_pointers_and_plan(op, c, device_sms(), &unused)) != RN_OK) return st;
@@ -772,7 +798,11 @@ rn_status rn_allreduce_fused_add_rms_norm_local(const rn_tensor* out, const rn_t
     if (st != RN_OK) return st;
     if (c.x.T % world != 0) return RN_ERR_SHAPE;
     const int64_t T = c.x.T / world, H = c.x.H;
-    const int64_t buffer_bytes = ((4 * T * H + 32 + 255) / 256) * 256;
+    // two buffer halves of 3TH values (room for two-shot) when the static
+    // memory holds them, else of TH values (one-shot only)
+    int64_t buffer_bytes = ((12 * T * H + 32 + 255) / 256) * 256;
+    if (buffer_bytes * world > rn::kLocalBufferBytes)
+        buffer_bytes = ((4 * T * H + 32 + 255) / 256) * 256;
     if (buffer_bytes * world > rn::kLocalBufferBytes) return RN_ERR_CAPACITY;
 
     int dev = 0;
@@ -813,6 +843,7 @@ rn_status rn_allreduce_fused_add_rms_norm_local(const rn_tensor* out, const rn_t
         }
         comm.buffer_bytes = buffer_bytes;
         comm.timeout_ns = 0;
+        comm.algorithm = RN_ALLREDUCE_AUTO;
     }
     return run_allreduce(false, out, nullptr, x, residual, weight, eps, &comm, stream);
 }

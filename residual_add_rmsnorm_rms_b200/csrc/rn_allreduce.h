@@ -13,14 +13,15 @@ namespace rn {
 constexpr int kArMaxWorld = 8;      // ranks in one group (one NVSwitch domain)
 constexpr int kArMaxBlocks = 1024;  // signal-pad capacity, in blocks per rank
 constexpr int kArMaxBlock = 512;    // threads per block (the kernel's launch bound)
-constexpr int kArSignalBytes = 64 + 2 * kArMaxBlocks * kArMaxWorld * 4;  // per rank
+constexpr int kArSignalBytes = 64 + 4 * kArMaxBlocks * kArMaxWorld * 4;  // per rank
 
 struct ArArgs {
     int world;                        // ranks in the group
     int rank;                         // rank driven by blockIdx.y == 0
     void* buffers[kArMaxWorld];       // every rank's exchange buffer (this process's address)
     uint32_t* signals[kArMaxWorld];   // every rank's signal pad (kArSignalBytes)
-    int64_t slot_elems;               // 16-bit elements per buffer half (call parity picks one)
+    int64_t slot_elems;               // 16-bit elements per buffer half (call parity picks one):
+                                      // >= T*H (one-shot) or 3*T*H (two-shot)
     long long timeout_ns;             // bound on each wait for a peer
     const void* x;                    // partial sums [local ranks][T][H]
     void* residual;                   // [local ranks][T][H], in place
@@ -40,6 +41,7 @@ struct ArLaunch {
     int smem;         // dynamic shared memory bytes
     int grid_x;       // blocks per rank (the same on every rank)
     int local_ranks;  // gridDim.y
+    bool two_shot;    // reduce-scatter of row slices + gather of finished rows
 };
 
 // Resident blocks per SM of the all-reduce kernel for this shape.

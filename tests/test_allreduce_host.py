@@ -22,7 +22,7 @@ def _comm(world=2, rank=0, local=2, nbytes=None, T=8, H=512, bufs=None, pads=Non
     if bufs is None:
         bufs = []
         for _ in range(world):
-            b = torch.zeros(buffer_bytes_for(T, H) // 8 + 8, dtype=torch.int64)
+            b = torch.zeros(buffer_bytes_for(T, H, False) // 8 + 8, dtype=torch.int64)
             keep.append(b)
             bufs.append(b.data_ptr())
     if pads is None:
@@ -35,7 +35,7 @@ def _comm(world=2, rank=0, local=2, nbytes=None, T=8, H=512, bufs=None, pads=Non
     c.world, c.rank, c.local_ranks = world, rank, local
     for i in range(world):
         c.buffers[i], c.signals[i] = bufs[i], pads[i]
-    c.buffer_bytes = buffer_bytes_for(T, H) if nbytes is None else nbytes
+    c.buffer_bytes = buffer_bytes_for(T, H, False) if nbytes is None else nbytes
     c.timeout_ns = 0
     return c, keep
 
@@ -62,12 +62,17 @@ def test_comm_validation():
     out, x, r, w = _ops()
     assert _call(out, x, r, w, None) == "RN_ERR_NULL"
     bad = [("world", 0), ("world", 9), ("rank", 2), ("rank", -1), ("rank", 1),  # rank 1 with 2 local
-           ("local_ranks", 3), ("local_ranks", 0),
-           ("buffer_bytes", buffer_bytes_for(8, 512) - 64), ("buffer_bytes", -1)]
+           ("local_ranks", 3), ("local_ranks", 0), ("algorithm", 3), ("algorithm", -1),
+           ("algorithm", 2),  # two-shot needs 3 ranks and buffers of 12*T*H + 32
+           ("buffer_bytes", buffer_bytes_for(8, 512, False) - 64), ("buffer_bytes", -1)]
     for field, value in bad:
         c, keep = _comm()
         setattr(c, field, value)
         assert _call(out, x, r, w, c) == "RN_ERR_COMM", (field, value)
+    o4, x4, r4, _ = _ops(L=4, T=8, H=512)
+    c4, keep4 = _comm(world=4, local=4)  # buffers sized for one-shot only
+    c4.algorithm = 2
+    assert _call(o4, x4, r4, w, c4) == "RN_ERR_COMM"
     c, keep = _comm()
     c.buffers[1] = None
     assert _call(out, x, r, w, c) == "RN_ERR_COMM"
@@ -99,7 +104,7 @@ def test_operand_validation():
     assert _call(out, xm, r, w, c) == "RN_ERR_LAYOUT"
     # residual aliasing x, and an operand inside a local exchange buffer
     assert _call(out, x, x, w, c) == "RN_ERR_ALIAS"
-    buf = torch.zeros(buffer_bytes_for(8, 512) // 2, dtype=torch.bfloat16)
+    buf = torch.zeros(buffer_bytes_for(8, 512, False) // 2, dtype=torch.bfloat16)
     cb, keepb = _comm(bufs=[buf.data_ptr(), keep[1].data_ptr()])
     inside = buf[: 2 * 8 * 512].view(2, 8, 512)
     assert _call(inside, x, r, w, cb) == "RN_ERR_ALIAS"
@@ -115,7 +120,10 @@ def test_operand_validation():
 def test_comm_descriptor():
     comm = AllReduceComm(2, 0, 2, [16, 32], [48, 64], 4096, timeout_s=0.25)
     d = comm.descriptor()
-    assert (d.world, d.rank, d.local_ranks) == (2, 0, 2)
+    assert (d.world, d.rank, d.local_ranks, d.algorithm) == (2, 0, 2, 0)
+    assert AllReduceComm(3, 0, 3, [0] * 3, [0] * 3, 64, algorithm="two_shot").descriptor().algorithm == 2
+    assert buffer_bytes_for(8, 512) == 12 * 8 * 512 + 32
+    assert buffer_bytes_for(8, 512, two_shot=False) == 4 * 8 * 512 + 32
     assert [d.buffers[0], d.buffers[1], d.signals[0], d.signals[1]] == [16, 32, 48, 64]
     assert (d.buffer_bytes, d.timeout_ns) == (4096, 250_000_000)
     assert comm.max_elements == 1024

@@ -21,6 +21,7 @@ import torch
 import oracle
 import residual_add_rmsnorm_rms_b200 as rn
 import synth
+from residual_add_rmsnorm_rms_b200 import torch_ops  # noqa: F401  (registers the ops)
 from residual_add_rmsnorm_rms_b200.allreduce import AllReduceComm
 from tests.cmp_util import bits16
 from tests.gpu_util import CORES, compare, sample_rows
@@ -97,33 +98,39 @@ CASES = [(1, 1, 512), (2, 7, 512), (2, 300, 3840), (4, 64, 4096), (8, 1, 3840),
 @pytest.mark.parametrize("W,T,H", CASES)
 @pytest.mark.parametrize("dtype", ["bf16", "fp16"])
 @pytest.mark.parametrize("fp8", [False, True], ids=["bf16out", "fp8"])
-def test_allreduce_parity(fp8, dtype, W, T, H):
+@pytest.mark.parametrize("algorithm", ["one_shot", "two_shot"])
+def test_allreduce_parity(algorithm, fp8, dtype, W, T, H):
+    if algorithm == "two_shot" and W < 3:
+        pytest.skip("two-shot needs three or more ranks")
     wl = synth.make_tp_inputs(dtype, W, T, H)
-    comm = AllReduceComm.single_device(W, T, H, "cuda")
+    comm = AllReduceComm.single_device(W, T, H, "cuda", algorithm=algorithm)
     got = _run(fp8, comm, wl.x.cuda(), wl.residual.cuda(), wl.weight.cuda(), wl.eps)
     print(_check(fp8, got, wl, dtype))
 
 
 @pytest.mark.parametrize("W", synth.TP_W)
 @pytest.mark.parametrize("fp8", [False, True], ids=["bf16out", "fp8"])
-def test_allreduce_prefill_size(fp8, W):
-    """Full prefill size [8192 x 3840] bf16, sampled rows against the oracle."""
+@pytest.mark.parametrize("algorithm", ["one_shot", "auto"])
+def test_allreduce_prefill_size(algorithm, fp8, W):
+    """Full prefill size [8192 x 3840] bf16, sampled rows against the oracle
+    (the automatic choice is two-shot here from four ranks on)."""
     T, H = 8192, 3840
     wl = synth.make_tp_inputs("bf16", W, T, H, device="cuda")
-    comm = AllReduceComm.single_device(W, T, H, "cuda")
+    comm = AllReduceComm.single_device(W, T, H, "cuda", algorithm=algorithm)
     got = _run(fp8, comm, wl.x, wl.residual, wl.weight, wl.eps)
     rows = sample_rows(T, k=96)
     wl.x, wl.residual, wl.weight = wl.x.cpu(), wl.residual.cpu(), wl.weight.cpu()
     print(_check(fp8, got, wl, "bf16", rows=rows))
 
 
-def test_allreduce_consecutive_calls():
+@pytest.mark.parametrize("algorithm", ["one_shot", "two_shot"])
+def test_allreduce_consecutive_calls(algorithm):
     """Calls 1..8 on the same buffers with changing row counts (both buffer
     halves and both flag parities, grids of different sizes, a call with no
     rows in between), each call checked in full; the device call counters
     advance once per call."""
     W, H = 4, 3840
-    comm = AllReduceComm.single_device(W, 300, H, "cuda")
+    comm = AllReduceComm.single_device(W, 300, H, "cuda", algorithm=algorithm)
     for i, T in enumerate([5, 300, 1, 0, 64, 300, 2, 17]):
         wl = synth.make_tp_inputs("bf16", W, T, H, seed=100 + i)
         fp8 = i % 2 == 1
@@ -165,7 +172,7 @@ def test_allreduce_exact_sum_edge_values():
 def test_allreduce_capacity_and_comm_checks():
     W, T, H = 2, 16, 512
     wl = synth.make_tp_inputs("bf16", W, T, H, device="cuda")
-    comm = AllReduceComm.single_device(W, T // 2, H, "cuda")  # room for 8 rows only
+    comm = AllReduceComm.single_device(W, T // 2, H, "cuda", algorithm="one_shot")  # 8 rows
     with pytest.raises(rn.RmsNormError) as e:
         _run(False, comm, wl.x, wl.residual, wl.weight, wl.eps)
     assert e.value.name == "RN_ERR_COMM"
@@ -176,6 +183,18 @@ def test_allreduce_capacity_and_comm_checks():
                                         torch.empty(3, 5, H, dtype=torch.bfloat16, device="cuda"),
                                         None, 1e-6, AllReduceComm.single_device(2, 8, H, "cuda"))
     assert e.value.name == "RN_ERR_SHAPE"
+    # two-shot forced on buffers sized for one-shot, and with two ranks
+    wl4 = synth.make_tp_inputs("bf16", 4, 8, H, device="cuda")
+    small = AllReduceComm.single_device(4, 8, H, "cuda", algorithm="one_shot")
+    forced = AllReduceComm(4, 0, 4, small.buffers, small.signals, small.buffer_bytes,
+                           keepalive=[small], algorithm="two_shot")
+    with pytest.raises(rn.RmsNormError) as e:
+        _run(False, forced, wl4.x, wl4.residual, wl4.weight, wl4.eps)
+    assert e.value.name == "RN_ERR_COMM"
+    with pytest.raises(rn.RmsNormError) as e:
+        _run(False, AllReduceComm.single_device(2, T, H, "cuda", algorithm="two_shot"), wl.x,
+             wl.residual, wl.weight, wl.eps)
+    assert e.value.name == "RN_ERR_COMM"
 
 
 def test_allreduce_peer_timeout_is_reported():
@@ -203,12 +222,13 @@ def test_allreduce_peer_timeout_is_reported():
            wl, "bf16")
 
 
-def test_allreduce_cuda_graph_replay():
+@pytest.mark.parametrize("algorithm", ["one_shot", "two_shot"])
+def test_allreduce_cuda_graph_replay(algorithm):
     """Calls captured in a CUDA graph take fresh call numbers on every replay
     (the counter lives in the signal pads), so replays with new data in the
     captured tensors stay correct."""
     W, T, H = 4, 48, 3840
-    comm = AllReduceComm.single_device(W, T, H, "cuda")
+    comm = AllReduceComm.single_device(W, T, H, "cuda", algorithm=algorithm)
     parts = torch.empty(W, T, H, dtype=torch.bfloat16, device="cuda")
     res = torch.empty(W, T, H, dtype=torch.bfloat16, device="cuda")
     out = torch.empty(W, T, H, dtype=torch.bfloat16, device="cuda")
@@ -266,3 +286,14 @@ def test_allreduce_torch_ops_equal_direct_calls():
     assert sc.shape == (W, T, 1)
     assert torch.equal(qc.view(torch.uint8), qe.view(torch.uint8)) and torch.equal(sc, se)
     assert torch.equal(rc.view(torch.int16), re_.view(torch.int16))
+
+
+@pytest.mark.parametrize("W,T", [(3, 1), (4, 2), (8, 5), (8, 7), (5, 3)])
+def test_allreduce_two_shot_fewer_rows_than_ranks(W, T):
+    """Two-shot slices of ceil(T / W) rows leave some ranks without rows."""
+    H = 512
+    for fp8 in (False, True):
+        wl = synth.make_tp_inputs("bf16", W, T, H, seed=W * 10 + T)
+        comm = AllReduceComm.single_device(W, T, H, "cuda", algorithm="two_shot")
+        got = _run(fp8, comm, wl.x.cuda(), wl.residual.cuda(), wl.weight.cuda(), wl.eps)
+        _check(fp8, got, wl, "bf16")

@@ -253,11 +253,16 @@ __device__ __forceinline__ void reduce_rows(const ArArgs& a, const int tpr, cons
         const int64_t roff = (active ? row : 0) * nvec;
         uint4* rrow = static_cast<uint4*>(a.residual) + local + roff;
 
-        uint4 r[VPT];  // residual loads first: in flight during the exchange reads
+        uint4 r[VPT];  // residual (and weight) loads first: in flight during the exchange reads
+        uint4 wk[VPT];
 #pragma unroll
         for (int k = 0; k < VPT; ++k) {
             const int j = lr + k * tpr;
             r[k] = (active && j < nvec) ? ld_stream(rrow + j) : make_uint4(0, 0, 0, 0);
+            wk[k] = make_uint4(0, 0, 0, 0);
+            if constexpr (kHasW) {
+                if (j < nvec) wk[k] = __ldg(wv + j);
+            }
         }
         uint4 v[VPT];
 #pragma unroll
@@ -285,13 +290,7 @@ __device__ __forceinline__ void reduce_rows(const ArArgs& a, const int tpr, cons
                     st_v4(reinterpret_cast<uint4*>(mine + lay.residual2) + roff + j, v[k]);
             }
             acc = ssq8<T>(v[k], acc);
-            if constexpr (kFp8) {
-                uint4 w = make_uint4(0, 0, 0, 0);
-                if constexpr (kHasW) {
-                    if (j < nvec) w = __ldg(wv + j);
-                }
-                pm = amax8<T, kHasW>(v[k], w, pm);
-            }
+            if constexpr (kFp8) pm = amax8<T, kHasW>(v[k], wk[k], pm);
         }
         float ss = acc.x + acc.y;
         const int width = tpr < 32 ? tpr : 32;
@@ -322,9 +321,7 @@ __device__ __forceinline__ void reduce_rows(const ArArgs& a, const int tpr, cons
             for (int k = 0; k < VPT; ++k) {
                 const int j = lr + k * tpr;
                 if (!(active && j < nvec)) continue;
-                uint4 w = make_uint4(0, 0, 0, 0);
-                if constexpr (kHasW) w = __ldg(wv + j);
-                const uint4 o = scale8<T, kHasW>(v[k], w, inv2);
+                const uint4 o = scale8<T, kHasW>(v[k], wk[k], inv2);
                 st_v4(orow + j, o);
                 if constexpr (kStage2) st_v4(reinterpret_cast<uint4*>(mine + lay.out2) + roff + j, o);
             }
@@ -341,9 +338,7 @@ __device__ __forceinline__ void reduce_rows(const ArArgs& a, const int tpr, cons
             for (int k = 0; k < VPT; ++k) {
                 const int j = lr + k * tpr;
                 if (!(active && j < nvec)) continue;
-                uint4 w = make_uint4(0, 0, 0, 0);
-                if constexpr (kHasW) w = __ldg(wv + j);
-                uint2 o = quant8<T, kHasW>(v[k], w, q2);
+                uint2 o = quant8<T, kHasW>(v[k], wk[k], q2);
                 if (!(pm > 0.f)) o = make_uint2(0, 0);
                 st_v2(qrow + j, o);
                 if constexpr (kStage2) st_v2(reinterpret_cast<uint2*>(mine + lay.out2) + roff + j, o);
@@ -461,14 +456,13 @@ __device__ __forceinline__ void allreduce_rows(const ArArgs& a, const int tpr, c
     }
     if (late && threadIdx.x == 0) atomicOr(&g_rn_ar_error, kErrPeerTimeout);
 
-    // 7. arrival; the last block of this rank advances the call counter
+    // 7. arrival; the last block of this rank advances the call counter. Every
+    //    block read the counter before arriving, and the next launch reads it
+    //    only after this grid has completed, so no fence is needed.
     __syncthreads();
-    if (threadIdx.x == 0) {
-        __threadfence();
-        if (atomicAdd(pad + kPadArrived, 1u) == gridDim.x - 1) {
-            atomicExch(pad + kPadArrived, 0u);
-            atomicExch(pad + kPadEpoch, epoch);
-        }
+    if (threadIdx.x == 0 && atomicAdd(pad + kPadArrived, 1u) == gridDim.x - 1) {
+        pad[kPadArrived] = 0u;
+        pad[kPadEpoch] = epoch;
     }
 }
 

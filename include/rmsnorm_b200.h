@@ -166,8 +166,9 @@ RN_API rn_status rn_silu_and_mul_fp8(const rn_tensor* q, const rn_tensor* scale,
  * Requirements: dense views (flattening rule of the norm ops), K % 16 == 0,
  * N % 8 == 0, 16-byte-aligned A, B and D, K, N and M below 2^31; D must not
  * overlap any input. M == 0 is a no-op. Needs no workspace. Asynchronous on
- * `stream`; validation errors return before any CUDA call. The tile shape is
- * chosen per call (rn_fp8_gemm_config). */
+ * `stream`, with programmatic dependent launch as the other kernels
+ * (rn_set_launch_options); validation errors return before any CUDA call.
+ * The tile shape is chosen per call (rn_fp8_gemm_config). */
 RN_API rn_status rn_fp8_rowwise_gemm(const rn_tensor* d, const rn_tensor* a,
                                      const rn_tensor* b, const rn_tensor* a_scale,
                                      const rn_tensor* b_scale, void* stream);

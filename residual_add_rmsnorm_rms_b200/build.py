@@ -34,7 +34,11 @@ NVCC_FLAGS = [
 ]
 # Sources that instantiate CUTLASS templates.
 CUTLASS_SOURCES = {"fp8_gemm.cu", "fp8_gemm_ch128.cu", "fp8_gemm_ch64.cu"}
-CUTLASS_FLAGS = ["--expt-relaxed-constexpr", "-diag-suppress", "20012"]
+# CUTLASS_ENABLE_GDC_FOR_SM100: the GEMM kernels wait for the previous kernel
+# in the stream (griddepcontrol) before touching memory, so they can be
+# launched with programmatic dependent launch like the other kernels.
+CUTLASS_FLAGS = ["--expt-relaxed-constexpr", "-diag-suppress", "20012",
+                 "-DCUTLASS_ENABLE_GDC_FOR_SM100=1"]
 
 
 def sources() -> list[str]:

@@ -15,7 +15,9 @@
 // with the accumulator in tensor memory, TMA loads of both operand tiles into
 // a multi-stage shared-memory pipeline, warp-specialised (load / MMA /
 // epilogue warps), persistent tile scheduler, cluster 1 x 1 x 1 (no
-// multicast), K step 128. The epilogue is an epilogue-visitor tree: fp32
+// multicast), K step 128, launched with programmatic dependent launch (the
+// kernel waits for the previous kernel in the stream before its first global
+// memory access, so its launch and prologue overlap that kernel's tail). The epilogue is an epilogue-visitor tree: fp32
 // accumulator x a_scale[m], then x b_scale[n], rounded once to bf16, stored
 // by TMA.
 //
@@ -127,7 +129,8 @@ struct RowwiseGemm {
         if (Gemm::get_workspace_size(args) != 0) return cudaErrorInvalidValue;  // none by design
         if (gemm.initialize(args, nullptr, stream) != cutlass::Status::kSuccess)
             return cudaErrorInvalidConfiguration;
-        if (gemm.run(stream) != cutlass::Status::kSuccess) return cudaErrorLaunchFailure;
+        if (gemm.run(stream, nullptr, g.pdl) != cutlass::Status::kSuccess)
+            return cudaErrorLaunchFailure;
         return cudaGetLastError();
     }
 };

@@ -604,8 +604,9 @@ rn_status rn_fp8_rowwise_gemm(const rn_tensor* d, const rn_tensor* a, const rn_t
     if (e == cudaSuccess) {
         rn::GemmArgs g{fa.ptr, fb.ptr, reinterpret_cast<const float*>(fsa.ptr),
                        reinterpret_cast<const float*>(fsb.ptr), fd.ptr, M, N, K, dev,
-                       device_sms(), 0};
+                       device_sms(), 0, false};
         g.config = gemm_config(M, N, g.num_sms);
+        g.pdl = g_pdl.load() < 0 ? kPdlDefault : g_pdl.load() == 1;
         e = rn::launch_fp8_rowwise_gemm(g, static_cast<cudaStream_t>(stream));
     }
     if (e != cudaSuccess) {

@@ -19,6 +19,7 @@ struct GemmArgs {
     int device;
     int num_sms;
     int config;           // GemmConfig: tile shape and orientation
+    bool pdl;             // launch with programmatic dependent launch
 };
 
 // Tile configurations of the fp8 GEMM (values of rn_gemm_config in the public

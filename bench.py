@@ -729,6 +729,49 @@ def time_tp_cell(rn, fp8, W, T, H, iters, device, algorithm="one_shot"):
     return us, gus
 
 
+def time_chain_cell(rn, T, iters, device, pdl):
+    """The decode chain of one layer input: fused_add_rms_norm_fp8 on [T x
+    3840] bf16, then the row-wise fp8 GEMM of its codes and per-token scales
+    with the 8192 x 3840 Gemma 4 12B weight. Mean time per chain over `iters`
+    chains under CUDA-graph replay (device time), with or without
+    programmatic dependent launch between the kernels."""
+    H, N = 3840, 8192
+    wl = synth.make_inputs("decode", "fused_add_rms_norm_fp8", "bf16", T, H, device=device)
+    g = torch.Generator(device=device).manual_seed(T)
+    b = (torch.randn(N, H, generator=g, device=device) * 40).clamp_(-448, 448).to(torch.float8_e4m3fn)
+    sb = torch.rand(N, generator=g, device=device) * 0.01
+    q = torch.empty(T, H, dtype=torch.float8_e4m3fn, device=device)
+    sc = torch.empty(T, dtype=torch.float32, device=device)
+    d = torch.empty(T, N, dtype=torch.bfloat16, device=device)
+    r = wl.residual.clone()
+    rn.set_launch_options(pdl=1 if pdl else 0)
+    try:
+        def chain():
+            rn.fused_add_rms_norm_fp8(q, sc, wl.x, r, wl.weight, wl.eps)
+            rn.fp8_rowwise_gemm(d, q, b, sc, sb)
+        st = torch.cuda.Stream(device)
+        with torch.cuda.stream(st):
+            chain()
+            torch.cuda.synchronize(device)
+            gr = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(gr, stream=st):
+                for _ in range(iters):
+                    chain()
+        gr.replay()
+        torch.cuda.synchronize(device)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record()
+        for _ in range(3):
+            gr.replay()
+        e1.record()
+        torch.cuda.synchronize(device)
+        us = e0.elapsed_time(e1) / (3 * iters) * 1e3
+        del gr
+    finally:
+        rn.set_launch_options(pdl=-1)
+    return us
+
+
 def run_sweep(args, world, rank, local):
     import residual_add_rmsnorm_rms_b200 as rn
     device = torch.device("cuda", local)
@@ -775,6 +818,17 @@ def run_sweep(args, world, rank, local):
                "how": "whole group on one device, one cooperative launch per call"}
         out.write(json.dumps(rec) + "\n")
         out.flush()
+    chain_cells = [T for T in synth.DECODE_T
+                   if all(w in ("chain", "decode", str(T)) for w in want)]
+    for T in chain_cells:
+        us_pdl = time_chain_cell(rn, T, 50, device, True)
+        us_plain = time_chain_cell(rn, T, 50, device, False)
+        rec = {"workload": "chain", "op": "fused_add_rms_norm_fp8 -> fp8_rowwise_gemm",
+               "dtype": "bf16/e4m3", "T": T, "H": 3840, "N": 8192,
+               "graph_us_pdl": round(us_pdl, 3), "graph_us_no_pdl": round(us_plain, 3),
+               "how": "CUDA-graph replay of 50 chains; device time per chain"}
+        out.write(json.dumps(rec) + "\n")
+        out.flush()
     gemm_cells = [(M, N, K) for (N, K) in GEMMA_NK for M in GEMM_M
                   if all(w in ("gemm", "fp8_rowwise_gemm", str(M), f"{N}x{K}") for w in want)]
     fp8_peak, fp8_src = measured_fp8_peak()
@@ -798,7 +852,7 @@ def run_sweep(args, world, rank, local):
     out.close()
     assert rn.device_errors() == 0
     print(json.dumps({"sweep": args.sweep_out,
-                      "cells": len(cells) + len(tp_cells) + len(gemm_cells)}))
+                      "cells": len(cells) + len(tp_cells) + len(chain_cells) + len(gemm_cells)}))
 
 
 def main():

@@ -244,6 +244,17 @@ def cpu_baseline(target_cpu_s: float = 15.0):
                       f"fp64 C oracle on {cores} host threads, {dt:.2f} s wall"}
 
 
+def step_config(eps: float) -> dict:
+    """The workload both arms report: the prefill step on [8192 x 3840] bf16."""
+    return {
+        "workload": f"prefill: fused_add_rms_norm (bf16 out) + fused_add_rms_norm_fp8 "
+                    f"(e4m3 + per-token scale), bf16 [{T_PREFILL} x {H_PREFILL}]",
+        "T": T_PREFILL, "H": H_PREFILL, "eps": eps,
+        "inputs": "x ~ Student-t(3) clipped +-1e3, residual ~ N(0,16), weight 1+N(0,0.1)",
+        "bytes_per_step": step_bytes(T_PREFILL, H_PREFILL),
+    }
+
+
 def run_reference(args, world, rank):
     """The reference arm: the fp64 CPU oracle timed on the host cores."""
     if rank != 0:
@@ -269,9 +280,7 @@ def run_reference(args, world, rank):
         "ms_per_step": round(total / args.steps * 1e3, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "rows_per_s": round(rows * args.steps / total, 2),
-        "config": {"workload": f"prefill fused_add_rms_norm + fused_add_rms_norm_fp8, bf16, "
-                               f"{T_PREFILL}x{H_PREFILL} (row sample of {rows})",
-                   "T": rows, "H": H_PREFILL},
+        "config": dict(step_config(wl.eps), sample_rows_per_step=rows),
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores,
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
@@ -392,16 +401,11 @@ def run_ours(args, world, rank, local):
         "rows_per_s": round(T * K * world / (total_ms / 1e3), 1),
         "frac_of_nominal_8tbs": round(value / world / NOMINAL_HBM_GBS, 4),
         "frac_of_measured_peak": round(value / world / peak, 4),
-        "config": {
-            "workload": f"prefill: fused_add_rms_norm (bf16 out) + fused_add_rms_norm_fp8 "
-                        f"(e4m3 + per-token scale), bf16 [{T} x {H}]",
-            "T": T, "H": H, "eps": eps,
-            "inputs": "x ~ Student-t(3) clipped +-1e3, residual ~ N(0,16), weight 1+N(0,0.1)",
-            "l2": f"rotating {n_sets} buffer sets ({n_sets * set_bytes(T, H) / 1e6:.0f} MB, "
-                  f">= 4x L2 of {l2 / 1e6:.0f} MB); no L2 flush",
-            "bytes_per_step": b_step,
-            "plans": {op: rn.plan_launch(op, torch.bfloat16, T, H) for op in STEP_OPS},
-        },
+        "config": dict(
+            step_config(eps),
+            l2=f"rotating {n_sets} buffer sets ({n_sets * set_bytes(T, H) / 1e6:.0f} MB, "
+               f">= 4x L2 of {l2 / 1e6:.0f} MB); no L2 flush",
+            plans={op: rn.plan_launch(op, torch.bfloat16, T, H) for op in STEP_OPS}),
         "per_kernel_how": f"each op alone, {K} launches back to back, events at the ends",
         "per_kernel_ms": {"fused_add_rms_norm": round(dom_ms, 5),
                           "fused_add_rms_norm_fp8": round(fp8_ms, 5)},

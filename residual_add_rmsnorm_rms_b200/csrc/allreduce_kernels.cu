@@ -111,13 +111,14 @@ __device__ __forceinline__ void st_copy(uint2* p, const uint2& v) { st_v2(p, v);
 // block-strided: the mapping of the reduce step) from src to dst, as `nvec`
 // vectors per row (16 bytes for 16-bit rows, 8 for e4m3 rows). Thread
 // (row, lr) moves vectors lr, lr + tpr, ... of its row, U row groups at a
-// time, all loads before any store, so a thread keeps U * VPT loads in
-// flight. `exchange` selects volatile loads (memory other ranks write).
+// time, all loads before any store, so a thread keeps U * VPT loads (at
+// least 64 bytes) in flight. `exchange` selects volatile loads (memory other ranks write).
 template <int VPT, typename V>
 __device__ __forceinline__ void copy_rows(V* dst, const V* src, const int64_t s0,
                                           const int64_t s1, const int tpr, const int rpc,
                                           const int nvec, const bool exchange) {
-    constexpr int U = VPT >= 4 ? 1 : 4 / VPT;
+    // at least 64 bytes of loads in flight per thread, 16- or 8-byte vectors
+    constexpr int U = (VPT >= 4 ? 1 : 4 / VPT) * (sizeof(V) == 8 ? 2 : 1);
     const int row_in_cta = threadIdx.x / tpr;
     const int lr = threadIdx.x - row_in_cta * tpr;
     const int64_t stride = static_cast<int64_t>(gridDim.x) * rpc;

@@ -13,7 +13,7 @@ import torch
 import synth
 import residual_add_rmsnorm_rms_b200 as rn
 from tests.cmp_util import bits16
-from tests.gpu_util import DT, compare, gpu_run, oracle_run
+from tests.gpu_util import compare, gpu_run, oracle_run
 
 pytestmark = pytest.mark.gpu
 OPS = ["rms_norm", "fused_add_rms_norm", "fused_add_rms_norm_fp8"]

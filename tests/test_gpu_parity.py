@@ -7,7 +7,6 @@ cells, the inputs are drawn on the GPU and a row sample (first, last, evenly
 spaced and random rows) is compared, in the same launch configuration the
 benchmark uses (the automatic plan).
 """
-import numpy as np
 import pytest
 import torch
 

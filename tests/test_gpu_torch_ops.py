@@ -1,14 +1,12 @@
 """torch custom ops on the GPU: same bits as the direct C-ABI calls and the
 oracle on N-D inputs, opcheck of schemas and fake implementations, and a
 torch.compile trace (aot_eager, fullgraph) through the mutating ops."""
-import numpy as np
 import pytest
 import torch
 
 import residual_add_rmsnorm_rms_b200 as rn
 import synth
 from residual_add_rmsnorm_rms_b200 import torch_ops as ops
-from tests.cmp_util import bits16
 from tests.gpu_util import compare, oracle_run
 
 pytestmark = pytest.mark.gpu

@@ -2,7 +2,6 @@
 (rn_validate) accepts exactly the views the eligibility predicate
 flatten_to_2d_is_free accepts, and never accepts a view whose flattening to
 2-D would copy or leave gaps."""
-import pytest
 import torch
 from hypothesis import HealthCheck, given, settings
 from hypothesis import strategies as st

@@ -207,7 +207,7 @@ int rows_per_block(int tpr, int64_t T) {
     return 1;
 }
 
-bool auto_vector_plan(int64_t T, int64_t H, int num_sms, rn_plan* p) {
+bool auto_vector_plan(int op, int64_t T, int64_t H, int num_sms, rn_plan* p) {
     const int64_t nvec = H / 8;
     auto idle_of = [&](int tpr, int vpt) {
         const int64_t slots = static_cast<int64_t>(tpr) * vpt;
@@ -217,6 +217,15 @@ bool auto_vector_plan(int64_t T, int64_t H, int num_sms, rn_plan* p) {
     const bool many_rows = tpr4 <= rn::max_block_for_vpt(4) &&
                            static_cast<double>(T) * tpr4 >= 1.0 * num_sms * 1024;
     if (many_rows) {
+        // fused_add_rms_norm: three vectors per thread when they tile the row
+        // exactly and four would leave lanes idle (H = 3840: 160 x 3 against
+        // 128 x 4 = 512 slots for 480 vectors), measured 1.9 % faster on B200
+        if (op == rn::kFusedAdd && idle_of(tpr_for(nvec, 3), 3) == 0.0 && idle_of(tpr4, 4) > 0.0 &&
+            tpr_for(nvec, 3) <= rn::max_block_for_vpt(3)) {
+            const int tpr = tpr_for(nvec, 3);
+            fill_vector_plan(tpr, 3, T, p, rows_per_block(tpr, T));
+            return true;
+        }
         for (int vpt : {4, 5, 3, 6, 8, 2}) {
             const int tpr = tpr_for(nvec, vpt);
             if (tpr > rn::max_block_for_vpt(vpt) || idle_of(tpr, vpt) > 1.0 / 8) continue;
@@ -292,7 +301,7 @@ rn_status plan_shape(int op, int64_t T, int64_t H, bool vector_ok, int num_sms, 
     }
     // The STAGED kernel is chosen only when forced: measured on B200 it trails
     // the VECTOR kernel at every shape tried (T up to 65536, H 2048..16384).
-    if (!auto_vector_plan(T, H, num_sms, p)) fill_scalar_plan(T, p);
+    if (!auto_vector_plan(op, T, H, num_sms, p)) fill_scalar_plan(T, p);
     return RN_OK;
 }
 

@@ -23,8 +23,10 @@
  * Common conventions for every entry point:
  *
  *  - Memory. Every data pointer is a DEVICE pointer on the current CUDA
- *    device. The caller owns and allocates all memory; the library allocates
- *    nothing and keeps no pointer after returning. Its only global state:
+ *    device, except the activations of the rn_host_* entry points, which
+ *    live in host memory. The caller owns and allocates all memory; the
+ *    library allocates nothing and keeps no pointer after returning. Its
+ *    only global state:
  *    the test and tuning overrides (rn_force_plan, rn_force_staged,
  *    rn_set_launch_options, rn_fp8_gemm_force_config), the thread-local
  *    error text, the device error flags (rn_device_errors) and the static
@@ -90,9 +92,9 @@ typedef enum {
     RN_ERR_VARIANCE_SIZE = 7, /* variance_size != -1 */
     RN_ERR_EPS = 8,           /* eps negative, NaN or infinite */
     RN_ERR_CUDA = 9,          /* a CUDA runtime call failed */
-    RN_ERR_CONFIG = 10,       /* rn_force_plan / rn_plan_launch: unsupported request */
+    RN_ERR_CONFIG = 10,       /* unsupported tuning request, op, or host-pipeline stream count */
     RN_ERR_COMM = 11,         /* all-reduce: bad group description or exchange buffers too small */
-    RN_ERR_CAPACITY = 12      /* rn_allreduce_fused_add_rms_norm_local: beyond its static memory */
+    RN_ERR_CAPACITY = 12      /* beyond the static exchange memory, or host-pipeline scratch too small */
 } rn_status;
 
 typedef enum {
@@ -331,6 +333,82 @@ RN_API rn_status rn_allreduce_fused_add_rms_norm_local(const rn_tensor* out, con
                                                        const rn_tensor* residual,
                                                        const rn_tensor* weight, float eps,
                                                        int32_t world, void* stream);
+
+/* ---- operands in host memory: chunked copy-in / compute / copy-out ------
+ *
+ * No counterpart on the pages, which time device-resident tensors only. These
+ * entry points run rn_rms_norm, rn_fused_add_rms_norm and
+ * rn_fused_add_rms_norm_fp8 on activations that live in HOST memory: out, x,
+ * residual, q and scale are host pointers (any memory a cudaMemcpyDefault
+ * copy reaches; only page-locked host memory lets the copies run
+ * asynchronously and overlap), while the weight is a device pointer as for
+ * the device entry points. The T rows are cut into chunks of chunk_rows rows.
+ * Chunk c runs on streams[c % n_streams] in slot (c % n_streams) of the
+ * scratch: its rows of x (and residual) are copied in, the kernel of the
+ * device entry point runs on the slot (16-bit output in place over the
+ * slot's x), and residual and out (or residual, q and scale) are copied back
+ * over the host rows. Chunks on different streams overlap, so the copy in of
+ * one chunk, the kernel of another and the copy out of a third proceed at
+ * once over the full-duplex host link. The results are those of the device
+ * entry point bit for bit: rows are independent and each chunk is one
+ * launch of the same kernels.
+ *
+ * Everything is enqueued and the call returns; the host buffers must stay
+ * untouched until every stream has finished. Work of earlier calls on the
+ * same streams orders before a chunk as usual; the scratch must not be used
+ * by anything else until then. Validation follows the device entry point
+ * (aliasing rules applied to the host buffers, out == x allowed), then the
+ * pipeline: NULL pipeline, streams or scratch -> RN_ERR_NULL; n_streams
+ * outside 1..RN_HOST_MAX_STREAMS or reserved != 0 -> RN_ERR_CONFIG; scratch
+ * not 256-byte aligned -> RN_ERR_LAYOUT; the slots (see rn_host_plan_chunks)
+ * not fitting in scratch_bytes -> RN_ERR_CAPACITY; scratch overlapping the
+ * weight or a host operand -> RN_ERR_ALIAS. All of these return before any
+ * CUDA call. A failed copy or launch returns RN_ERR_CUDA; chunks enqueued
+ * before it still run. T == 0 is a no-op. */
+#define RN_HOST_MAX_STREAMS 8
+
+typedef struct {
+    void* scratch;          /* caller-owned device memory, 256-byte aligned */
+    int64_t scratch_bytes;
+    void* const* streams;   /* n_streams caller-owned cudaStream_t of the current device */
+    int32_t n_streams;      /* 1 .. RN_HOST_MAX_STREAMS */
+    int32_t reserved;       /* must be 0 */
+    int64_t chunk_rows;     /* rows per chunk; <= 0: the library's choice */
+} rn_host_pipeline;
+
+typedef struct {
+    int64_t chunk_rows;  /* rows per chunk (the last chunk may hold fewer) */
+    int64_t chunks;      /* ceil(T / chunk_rows); 0 when T == 0 */
+    int64_t slot_bytes;  /* scratch bytes of one slot */
+    int32_t slots;       /* slots in use: min(n_streams, chunks) */
+    int32_t reserved;
+} rn_host_plan;
+
+/* The chunking of a host-memory call: op (rn_op, not SILU_AND_MUL_FP8), a
+ * [T x H] 16-bit problem, scratch_bytes of scratch, n_streams streams and the
+ * requested chunk_rows (<= 0: automatic). A slot holds, for chunk_rows rows,
+ * the x rows (2 * H bytes each), the residual rows (fused ops, 2 * H), the
+ * codes (fp8 op, H) and the scales (fp8 op, 4), each region rounded up to 256
+ * bytes. Automatic: chunks of ceil(T / (4 * n_streams)) rows, but at least
+ * enough rows for 8 MiB of x per copy, at most T, and no more than
+ * n_streams slots can hold in scratch_bytes. RN_ERR_CAPACITY when the slots
+ * in use do not fit, RN_ERR_SHAPE for T < 0 or H < 1, RN_ERR_CONFIG for a bad
+ * op or n_streams. Pure host logic. */
+RN_API rn_status rn_host_plan_chunks(int32_t op, int64_t T, int64_t H, int64_t scratch_bytes,
+                                     int32_t n_streams, int64_t chunk_rows, rn_host_plan* plan);
+
+RN_API rn_status rn_host_rms_norm(const rn_tensor* out, const rn_tensor* x,
+                                  const rn_tensor* weight, float eps, int64_t variance_size,
+                                  const rn_host_pipeline* pipeline);
+RN_API rn_status rn_host_fused_add_rms_norm(const rn_tensor* out, const rn_tensor* x,
+                                            const rn_tensor* residual, const rn_tensor* weight,
+                                            float eps, int64_t variance_size,
+                                            const rn_host_pipeline* pipeline);
+RN_API rn_status rn_host_fused_add_rms_norm_fp8(const rn_tensor* q, const rn_tensor* scale,
+                                                const rn_tensor* x, const rn_tensor* residual,
+                                                const rn_tensor* weight, float eps,
+                                                int64_t variance_size,
+                                                const rn_host_pipeline* pipeline);
 
 /* Static text for a status code (never NULL). */
 RN_API const char* rn_status_string(rn_status status);

@@ -27,6 +27,8 @@ __all__ = [
     "silu_and_mul_fp8", "fp8_rowwise_gemm", "fp8_gemm_config", "fp8_gemm_force_config",
     "GEMM_CONFIGS", "allreduce_fused_add_rms_norm", "allreduce_fused_add_rms_norm_fp8",
     "allreduce_fused_add_rms_norm_local",
+    "host_rms_norm", "host_fused_add_rms_norm", "host_fused_add_rms_norm_fp8",
+    "host_plan_chunks", "RnHostPipeline", "RnHostPlan", "HOST_MAX_STREAMS",
     "RnAllreduceComm", "ALLREDUCE_MAX_WORLD", "ALLREDUCE_SIGNAL_BYTES", "ALLREDUCE_ALGORITHMS",
     "plan_launch", "validate", "force_plan", "force_staged",
     "set_launch_options", "device_errors", "supported_vectors_per_thread", "status_string",
@@ -40,6 +42,7 @@ STATUS = {
     5: "RN_ERR_LAYOUT", 6: "RN_ERR_ALIAS", 7: "RN_ERR_VARIANCE_SIZE", 8: "RN_ERR_EPS",
     9: "RN_ERR_CUDA", 10: "RN_ERR_CONFIG", 11: "RN_ERR_COMM", 12: "RN_ERR_CAPACITY",
 }
+HOST_MAX_STREAMS = 8
 OPS = {"rms_norm": 0, "fused_add_rms_norm": 1, "fused_add_rms_norm_fp8": 2}
 PLAN_OPS = dict(OPS, silu_and_mul_fp8=3)
 _DTYPES = {torch.float16: 0, torch.bfloat16: 1, torch.float8_e4m3fn: 2, torch.float32: 3,
@@ -63,6 +66,32 @@ class RnAllreduceComm(ctypes.Structure):
         ("buffer_bytes", ctypes.c_int64),
         ("timeout_ns", ctypes.c_int64),
     ]
+
+
+class RnHostPipeline(ctypes.Structure):
+    """rn_host_pipeline (include/rmsnorm_b200.h)."""
+    _fields_ = [
+        ("scratch", ctypes.c_void_p),
+        ("scratch_bytes", ctypes.c_int64),
+        ("streams", ctypes.POINTER(ctypes.c_void_p)),
+        ("n_streams", ctypes.c_int32),
+        ("reserved", ctypes.c_int32),
+        ("chunk_rows", ctypes.c_int64),
+    ]
+
+
+class RnHostPlan(ctypes.Structure):
+    """rn_host_plan (include/rmsnorm_b200.h)."""
+    _fields_ = [
+        ("chunk_rows", ctypes.c_int64),
+        ("chunks", ctypes.c_int64),
+        ("slot_bytes", ctypes.c_int64),
+        ("slots", ctypes.c_int32),
+        ("reserved", ctypes.c_int32),
+    ]
+
+    def as_dict(self):
+        return {k: getattr(self, k) for k, _ in self._fields_ if k != "reserved"}
 
 
 class RnTensor(ctypes.Structure):
@@ -123,6 +152,15 @@ def _load():
     L.rn_allreduce_fused_add_rms_norm_local.argtypes = [P, P, P, P, F, ctypes.c_int32, VP]
     L.rn_allreduce_fused_add_rms_norm_local.restype = ctypes.c_int
     L.rn_allreduce_fused_add_rms_norm_fp8.restype = ctypes.c_int
+    HP = ctypes.POINTER(RnHostPipeline)
+    L.rn_host_rms_norm.argtypes = [P, P, P, F, I64, HP]
+    L.rn_host_fused_add_rms_norm.argtypes = [P, P, P, P, F, I64, HP]
+    L.rn_host_fused_add_rms_norm_fp8.argtypes = [P, P, P, P, P, F, I64, HP]
+    for f in (L.rn_host_rms_norm, L.rn_host_fused_add_rms_norm, L.rn_host_fused_add_rms_norm_fp8):
+        f.restype = ctypes.c_int
+    L.rn_host_plan_chunks.argtypes = [ctypes.c_int32, I64, I64, I64, ctypes.c_int32, I64,
+                                      ctypes.POINTER(RnHostPlan)]
+    L.rn_host_plan_chunks.restype = ctypes.c_int
     L.rn_fp8_gemm_config.argtypes = [I64, I64, I64, ctypes.c_int32, ctypes.POINTER(ctypes.c_int32)]
     L.rn_fp8_gemm_config.restype = ctypes.c_int
     L.rn_fp8_gemm_force_config.argtypes = [ctypes.c_int32]
@@ -322,6 +360,65 @@ def allreduce_fused_add_rms_norm_local(out: torch.Tensor, x: torch.Tensor,
                _desc(residual, 2), None if weight is None else _desc(weight, 3), eps,
                int(world), s)
     _check(st, "rn_allreduce_fused_add_rms_norm_local")
+
+
+def host_plan_chunks(op: str, T: int, H: int, scratch_bytes: int, n_streams: int,
+                     chunk_rows: int = 0) -> dict:
+    """The chunking of a host-memory call (C ABI rn_host_plan_chunks; host logic)."""
+    p = RnHostPlan()
+    _check(lib.rn_host_plan_chunks(OPS[op], T, H, scratch_bytes, n_streams, chunk_rows,
+                                   ctypes.byref(p)), "rn_host_plan_chunks")
+    return p.as_dict()
+
+
+def _host_call(fn, name, pipeline, tensors, weight, args, join):
+    """Validates that the activations are CPU tensors and the weight lives on
+    the pipeline's device, then enqueues through the pipeline's streams."""
+    for t in tensors:
+        if t.is_cuda:
+            raise ValueError(f"{name}: activations must be host (CPU) tensors")
+    if weight is not None and weight.get_device() != pipeline.device:
+        raise ValueError(f"{name}: the weight must be on the pipeline's device")
+    with torch.cuda.device(pipeline.device):
+        pipeline.begin(args[0], join)
+        st = fn(*args[1:], pipeline.descriptor_ref())
+        pipeline.end(join)
+    _check(st, name)
+
+
+def host_rms_norm(out: torch.Tensor, x: torch.Tensor, weight: torch.Tensor | None, eps: float,
+                  pipeline, variance_size=None, join: bool = True) -> None:
+    """rms_norm on host-memory activations through `pipeline` (a
+    ``host.HostPipeline``): chunked copy in, kernel, copy out (C ABI
+    rn_host_rms_norm). With join, the pipeline's streams start after the
+    current stream's work and the current stream waits for them."""
+    _host_call(lib.rn_host_rms_norm, "rn_host_rms_norm", pipeline, (out, x), weight,
+               (("rms_norm", x.shape[-1] if x.dim() else 0), _desc(out, 0), _desc(x, 1),
+                None if weight is None else _desc(weight, 2), eps, _vs(variance_size)), join)
+
+
+def host_fused_add_rms_norm(out: torch.Tensor, x: torch.Tensor, residual: torch.Tensor,
+                            weight: torch.Tensor | None, eps: float, pipeline,
+                            variance_size=None, join: bool = True) -> None:
+    """fused_add_rms_norm on host-memory activations (C ABI
+    rn_host_fused_add_rms_norm); residual is updated in host memory."""
+    _host_call(lib.rn_host_fused_add_rms_norm, "rn_host_fused_add_rms_norm", pipeline,
+               (out, x, residual), weight,
+               (("fused_add_rms_norm", x.shape[-1] if x.dim() else 0), _desc(out, 0),
+                _desc(x, 1), _desc(residual, 2), None if weight is None else _desc(weight, 3),
+                eps, _vs(variance_size)), join)
+
+
+def host_fused_add_rms_norm_fp8(q: torch.Tensor, scale: torch.Tensor, x: torch.Tensor,
+                                residual: torch.Tensor, weight: torch.Tensor | None, eps: float,
+                                pipeline, variance_size=None, join: bool = True) -> None:
+    """fused_add_rms_norm_fp8 on host-memory activations (C ABI
+    rn_host_fused_add_rms_norm_fp8); q and scale are written in host memory."""
+    _host_call(lib.rn_host_fused_add_rms_norm_fp8, "rn_host_fused_add_rms_norm_fp8", pipeline,
+               (q, scale, x, residual), weight,
+               (("fused_add_rms_norm_fp8", x.shape[-1] if x.dim() else 0), _desc(q, 0),
+                _desc(scale, 1), _desc(x, 2), _desc(residual, 3),
+                None if weight is None else _desc(weight, 4), eps, _vs(variance_size)), join)
 
 
 # rn_gemm_config values: TOK = token-major (tokens x channels) tiles, CH =

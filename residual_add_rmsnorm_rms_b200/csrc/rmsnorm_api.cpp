@@ -477,6 +477,26 @@ rn_status prepare(int op, const rn_tensor* o, const rn_tensor* sc, const rn_tens
     return RN_OK;
 }
 
+// Enqueues the norm kernel `plan` describes.
+rn_status launch_plan(int op, int dt, const rn::Args& a, const rn_plan& plan, bool pdl,
+                      void* stream) {
+    const rn::Launch l{plan.kernel,
+                       plan.threads_per_row,
+                       plan.kernel == RN_KERNEL_STAGED ? plan.stages : plan.vectors_per_thread,
+                       plan.rows_per_cta,
+                       plan.block_threads,
+                       plan.smem_bytes,
+                       plan.grid,
+                       pdl};
+    const cudaError_t e = rn::launch(op, dt, a, l, static_cast<cudaStream_t>(stream));
+    if (e != cudaSuccess) {
+        std::snprintf(g_cuda_error, sizeof g_cuda_error, "%s: %s", cudaGetErrorName(e),
+                      cudaGetErrorString(e));
+        return RN_ERR_CUDA;
+    }
+    return RN_OK;
+}
+
 rn_status run(int op, const rn_tensor* o, const rn_tensor* sc, const rn_tensor* x,
               const rn_tensor* r, const rn_tensor* w, float eps, int64_t variance_size,
               void* stream) {
@@ -498,21 +518,8 @@ rn_status run(int op, const rn_tensor* o, const rn_tensor* sc, const rn_tensor* 
     a.T = c.x.T;
     a.H = c.x.H;
     a.eps = eps;
-    const rn::Launch l{plan.kernel,
-                       plan.threads_per_row,
-                       plan.kernel == RN_KERNEL_STAGED ? plan.stages : plan.vectors_per_thread,
-                       plan.rows_per_cta,
-                       plan.block_threads,
-                       plan.smem_bytes,
-                       plan.grid,
-                       g_pdl.load() < 0 ? kPdlDefault : g_pdl.load() == 1};
-    const cudaError_t e = rn::launch(op, c.dt, a, l, static_cast<cudaStream_t>(stream));
-    if (e != cudaSuccess) {
-        std::snprintf(g_cuda_error, sizeof g_cuda_error, "%s: %s", cudaGetErrorName(e),
-                      cudaGetErrorString(e));
-        return RN_ERR_CUDA;
-    }
-    return RN_OK;
+    return launch_plan(op, c.dt, a, plan, g_pdl.load() < 0 ? kPdlDefault : g_pdl.load() == 1,
+                       stream);
 }
 
 }  // namespace
@@ -794,6 +801,157 @@ rn_status local_cuda_error(cudaError_t e) {
     return RN_ERR_CUDA;
 }
 
+// ---- activations in host memory (rn_host_*) ------------------------------
+//
+// Chunk c of the rows goes to stream c % n and to slot c % n of the scratch:
+// copy in, one launch of the device kernel on the slot, copy out, all on
+// that stream. A slot is reused only by a later chunk of the same stream, so
+// stream order alone keeps a slot's copy out before the next chunk's copy in.
+
+constexpr int64_t kHostAlign = 256;
+// x bytes per chunk copy, at least: on B200 over PCIe 5, 5 MB chunks ran the
+// prefill step 7 % slower than 8-10 MB chunks, 2 MB chunks 16 % slower
+constexpr int64_t kHostMinCopyBytes = int64_t{8} << 20;
+
+// Byte offsets of the regions of one slot of `rows` rows.
+struct HostSlot {
+    int64_t x = 0, r = 0, q = 0, s = 0, bytes = 0;
+};
+
+HostSlot host_slot(int op, int64_t rows, int64_t H) {
+    HostSlot l;
+    int64_t off = round_up(rows * H * 2, kHostAlign);  // x, and the 16-bit out in place
+    if (op != rn::kRmsNorm) {
+        l.r = off;
+        off += round_up(rows * H * 2, kHostAlign);
+    }
+    if (op == rn::kFusedAddFp8) {
+        l.q = off;
+        off += round_up(rows * H, kHostAlign);
+        l.s = off;
+        off += round_up(rows * 4, kHostAlign);
+    }
+    l.bytes = off;
+    return l;
+}
+
+// The most rows of which `slots` slots fit in `bytes` (0 if not one).
+int64_t host_rows_fitting(int op, int64_t H, int64_t bytes, int64_t slots) {
+    const int64_t per_slot = bytes / slots;
+    const int64_t per_row = 2 * H + (op != rn::kRmsNorm ? 2 * H : 0) +
+                            (op == rn::kFusedAddFp8 ? H + 4 : 0);
+    int64_t rows = per_slot / per_row;
+    while (rows > 0 && host_slot(op, rows, H).bytes > per_slot) --rows;
+    return rows;
+}
+
+rn_status host_plan(int op, int64_t T, int64_t H, int64_t scratch_bytes, int n_streams,
+                    int64_t want_rows, rn_host_plan* p) {
+    std::memset(p, 0, sizeof *p);
+    if (op < rn::kRmsNorm || op > rn::kFusedAddFp8) return RN_ERR_CONFIG;
+    if (n_streams < 1 || n_streams > RN_HOST_MAX_STREAMS) return RN_ERR_CONFIG;
+    if (T < 0 || H < 1) return RN_ERR_SHAPE;
+    // keeps every byte count below 2^62
+    if (H > (int64_t{1} << 40) || static_cast<double>(T) * static_cast<double>(H) > 1e17)
+        return RN_ERR_SHAPE;
+    if (T == 0) return RN_OK;
+    if (scratch_bytes < 0) scratch_bytes = 0;
+    int64_t rows;
+    if (want_rows > 0) {
+        rows = want_rows < T ? want_rows : T;
+    } else {
+        const int64_t n = n_streams;
+        rows = (T + 4 * n - 1) / (4 * n);
+        const int64_t min_rows = (kHostMinCopyBytes + 2 * H - 1) / (2 * H);
+        if (rows < min_rows) rows = min_rows;
+        if (rows > T) rows = T;
+        const int64_t fit = host_rows_fitting(op, H, scratch_bytes, n);
+        if (fit < 1) return RN_ERR_CAPACITY;
+        if (rows > fit) rows = fit;
+    }
+    const int64_t chunks = (T + rows - 1) / rows;
+    const int64_t slots = chunks < n_streams ? chunks : n_streams;
+    const int64_t slot_bytes = host_slot(op, rows, H).bytes;
+    if (slot_bytes > scratch_bytes / slots) return RN_ERR_CAPACITY;
+    p->chunk_rows = rows;
+    p->chunks = chunks;
+    p->slot_bytes = slot_bytes;
+    p->slots = static_cast<int32_t>(slots);
+    return RN_OK;
+}
+
+rn_status run_host(int op, const rn_tensor* o, const rn_tensor* sc, const rn_tensor* x,
+                   const rn_tensor* r, const rn_tensor* w, float eps, int64_t variance_size,
+                   const rn_host_pipeline* hp) {
+    Common c;
+    rn_status st = check_descriptors(op, o, sc, x, r, w, eps, variance_size, &c);
+    if (st != RN_OK) return st;
+    if (!hp) return RN_ERR_NULL;
+    if (hp->n_streams < 1 || hp->n_streams > RN_HOST_MAX_STREAMS || hp->reserved != 0)
+        return RN_ERR_CONFIG;
+    if (!hp->streams) return RN_ERR_NULL;
+    if (c.x.T == 0) return RN_OK;
+    rn_plan whole;  // the whole-problem plan is not used: each chunk is planned
+    st = check_pointers_and_plan(op, c, kDefaultSms, &whole);
+    if (st != RN_OK) return st;
+    if (!hp->scratch) return RN_ERR_NULL;
+    if (!aligned(hp->scratch, kHostAlign)) return RN_ERR_LAYOUT;
+    rn_host_plan hpl;
+    st = host_plan(op, c.x.T, c.x.H, hp->scratch_bytes, hp->n_streams, hp->chunk_rows, &hpl);
+    if (st != RN_OK) return st;
+    Flat used;
+    used.ptr = static_cast<char*>(hp->scratch);
+    used.numel = hpl.slots * hpl.slot_bytes;
+    used.esize = 1;
+    for (const Flat* f : {&c.x, &c.out, &c.res, &c.q, &c.scale, &c.w})
+        if (f->ptr && overlap(used, *f)) return RN_ERR_ALIAS;
+
+    const int64_t T = c.x.T, H = c.x.H;
+    const bool fused = op != rn::kRmsNorm, fp8 = op == rn::kFusedAddFp8;
+    const bool vector_ok = H % 8 == 0 && (!c.has_w || aligned(c.w.ptr, 16));
+    const int num_sms = device_sms();
+    const HostSlot L = host_slot(op, hpl.chunk_rows, H);
+    for (int64_t k = 0; k < hpl.chunks; ++k) {
+        const int64_t t0 = k * hpl.chunk_rows;
+        const int64_t rows = T - t0 < hpl.chunk_rows ? T - t0 : hpl.chunk_rows;
+        const int slot = static_cast<int>(k % hpl.slots);
+        char* base = static_cast<char*>(hp->scratch) + slot * hpl.slot_bytes;
+        cudaStream_t s = static_cast<cudaStream_t>(hp->streams[slot]);
+        const int64_t b16 = rows * H * 2, off16 = t0 * H * 2;
+        cudaError_t e = cudaMemcpyAsync(base + L.x, c.x.ptr + off16, b16, cudaMemcpyDefault, s);
+        if (e == cudaSuccess && fused)
+            e = cudaMemcpyAsync(base + L.r, c.res.ptr + off16, b16, cudaMemcpyDefault, s);
+        if (e != cudaSuccess) return local_cuda_error(e);
+
+        rn::Args a;
+        a.x = base + L.x;
+        a.residual = fused ? base + L.r : nullptr;
+        a.weight = c.has_w ? c.w.ptr : nullptr;
+        a.out = fp8 ? nullptr : base + L.x;  // in place over the slot's x
+        a.q = fp8 ? reinterpret_cast<uint8_t*>(base + L.q) : nullptr;
+        a.scale = fp8 ? reinterpret_cast<float*>(base + L.s) : nullptr;
+        a.T = rows;
+        a.H = H;
+        a.eps = eps;
+        rn_plan plan;
+        st = plan_impl(op, rows, H, vector_ok, num_sms, &plan);
+        if (st != RN_OK) return st;
+        // no programmatic dependent launch: the kernel follows copies
+        st = launch_plan(op, c.dt, a, plan, false, s);
+        if (st != RN_OK) return st;
+
+        if (fused) e = cudaMemcpyAsync(c.res.ptr + off16, base + L.r, b16, cudaMemcpyDefault, s);
+        if (e == cudaSuccess && !fp8)
+            e = cudaMemcpyAsync(c.out.ptr + off16, base + L.x, b16, cudaMemcpyDefault, s);
+        if (e == cudaSuccess && fp8)
+            e = cudaMemcpyAsync(c.q.ptr + t0 * H, base + L.q, rows * H, cudaMemcpyDefault, s);
+        if (e == cudaSuccess && fp8)
+            e = cudaMemcpyAsync(c.scale.ptr + t0 * 4, base + L.s, rows * 4, cudaMemcpyDefault, s);
+        if (e != cudaSuccess) return local_cuda_error(e);
+    }
+    return RN_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -896,9 +1054,9 @@ const char* rn_status_string(rn_status s) {
         case RN_ERR_VARIANCE_SIZE: return "variance_size override is not supported";
         case RN_ERR_EPS: return "eps must be finite and >= 0";
         case RN_ERR_CUDA: return "CUDA error (see rn_last_cuda_error)";
-        case RN_ERR_CONFIG: return "unsupported launch configuration";
+        case RN_ERR_CONFIG: return "unsupported configuration (tuning request, op or stream count)";
         case RN_ERR_COMM: return "bad all-reduce group description or exchange buffers too small";
-        case RN_ERR_CAPACITY: return "problem larger than the library's static exchange memory";
+        case RN_ERR_CAPACITY: return "problem larger than the static exchange memory or the scratch";
     }
     return "unknown status";
 }
@@ -989,6 +1147,35 @@ rn_status rn_fp8_gemm_force_config(int32_t config) {
     return RN_OK;
 }
 
-const char* rn_version(void) { return "0.3.0"; }
+rn_status rn_host_plan_chunks(int32_t op, int64_t T, int64_t H, int64_t scratch_bytes,
+                              int32_t n_streams, int64_t chunk_rows, rn_host_plan* plan) {
+    if (!plan) return RN_ERR_NULL;
+    return host_plan(op, T, H, scratch_bytes, n_streams, chunk_rows, plan);
+}
+
+rn_status rn_host_rms_norm(const rn_tensor* out, const rn_tensor* x, const rn_tensor* weight,
+                           float eps, int64_t variance_size, const rn_host_pipeline* pipeline) {
+    return run_host(rn::kRmsNorm, out, nullptr, x, nullptr, weight, eps, variance_size,
+                    pipeline);
+}
+
+rn_status rn_host_fused_add_rms_norm(const rn_tensor* out, const rn_tensor* x,
+                                     const rn_tensor* residual, const rn_tensor* weight,
+                                     float eps, int64_t variance_size,
+                                     const rn_host_pipeline* pipeline) {
+    return run_host(rn::kFusedAdd, out, nullptr, x, residual, weight, eps, variance_size,
+                    pipeline);
+}
+
+rn_status rn_host_fused_add_rms_norm_fp8(const rn_tensor* q, const rn_tensor* scale,
+                                         const rn_tensor* x, const rn_tensor* residual,
+                                         const rn_tensor* weight, float eps,
+                                         int64_t variance_size,
+                                         const rn_host_pipeline* pipeline) {
+    return run_host(rn::kFusedAddFp8, q, scale, x, residual, weight, eps, variance_size,
+                    pipeline);
+}
+
+const char* rn_version(void) { return "0.4.0"; }
 
 }  // extern "C"

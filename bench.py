@@ -237,11 +237,18 @@ def cpu_baseline(target_cpu_s: float = 15.0):
     rows = int(max(probe_rows, min(T_PREFILL, target_cpu_s / per_row)))
     sample = (wl.x[:rows], wl.residual[:rows], wl.weight, wl.eps)
     dt, rows, nbytes = oracle_step_sample(rows, cores, sample)
+    # one core: about 2 s of work on the first rows of the same batch
+    rows1 = int(max(probe_rows, min(T_PREFILL, 2.0 / per_row)))
+    dt1, rows1, nbytes1 = oracle_step_sample(
+        rows1, 1, (wl.x[:rows1], wl.residual[:rows1], wl.weight, wl.eps))
     return {"value": round(nbytes / dt / 1e9, 4), "unit": "GB/s", "cores": cores,
             "kind": "oracle",
             "rows_per_s": round(rows / dt, 2),
             "sample": f"first {rows} of {T_PREFILL} rows of the prefill batch, both ops of a step, "
-                      f"fp64 C oracle on {cores} host threads, {dt:.2f} s wall"}
+                      f"fp64 C oracle on {cores} host threads, {dt:.2f} s wall",
+            "one_core": {"value": round(nbytes1 / dt1 / 1e9, 4), "unit": "GB/s",
+                         "rows_per_s": round(rows1 / dt1, 2),
+                         "sample": f"first {rows1} rows, one thread, {dt1:.2f} s wall"}}
 
 
 def step_config(eps: float) -> dict:

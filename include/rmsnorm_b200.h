@@ -362,9 +362,11 @@ RN_API rn_status rn_allreduce_fused_add_rms_norm_local(const rn_tensor* out, con
  * outside 1..RN_HOST_MAX_STREAMS or reserved != 0 -> RN_ERR_CONFIG; scratch
  * not 256-byte aligned -> RN_ERR_LAYOUT; the slots (see rn_host_plan_chunks)
  * not fitting in scratch_bytes -> RN_ERR_CAPACITY; scratch overlapping the
- * weight or a host operand -> RN_ERR_ALIAS. All of these return before any
- * CUDA call. A failed copy or launch returns RN_ERR_CUDA; chunks enqueued
- * before it still run. T == 0 is a no-op. */
+ * weight or a host operand -> RN_ERR_ALIAS; all of these before any CUDA
+ * call. Last, the scratch and the weight must be device (or managed)
+ * memory: cudaPointerGetAttributes is asked, RN_ERR_LAYOUT otherwise. A
+ * failed copy or launch returns RN_ERR_CUDA; chunks enqueued before it
+ * still run. T == 0 is a no-op. */
 #define RN_HOST_MAX_STREAMS 8
 
 typedef struct {

@@ -905,6 +905,17 @@ rn_status run_host(int op, const rn_tensor* o, const rn_tensor* sc, const rn_ten
     used.esize = 1;
     for (const Flat* f : {&c.x, &c.out, &c.res, &c.q, &c.scale, &c.w})
         if (f->ptr && overlap(used, *f)) return RN_ERR_ALIAS;
+    // The kernels dereference the scratch and the weight: both must be device
+    // memory (a host weight is the likely mistake with these entry points).
+    for (const void* d : {static_cast<const void*>(hp->scratch),
+                          static_cast<const void*>(c.has_w ? c.w.ptr : nullptr)}) {
+        if (!d) continue;
+        cudaPointerAttributes attr;
+        const cudaError_t e = cudaPointerGetAttributes(&attr, d);
+        if (e != cudaSuccess) return local_cuda_error(e);
+        if (attr.type != cudaMemoryTypeDevice && attr.type != cudaMemoryTypeManaged)
+            return RN_ERR_LAYOUT;
+    }
 
     const int64_t T = c.x.T, H = c.x.H;
     const bool fused = op != rn::kRmsNorm, fp8 = op == rn::kFusedAddFp8;

@@ -147,3 +147,22 @@ def test_host_pipeline_empty_and_plan():
     with pytest.raises(rn.RmsNormError) as e:
         _run_host("fused_add_rms_norm", wl.x, wl.residual, wl.weight, wl.eps, small)
     assert e.value.name == "RN_ERR_CAPACITY"
+
+
+def test_host_pipeline_refuses_host_weight():
+    """The weight must be device memory: a page-locked host weight is refused
+    before any copy or launch (page-locked, so that even a launch could only
+    read mapped host memory), by the binding and by the C ABI itself."""
+    T, H = 64, 512
+    wl = synth.make_inputs("small", "fused_add_rms_norm", "bf16", T, H)
+    pipe = _pipeline("fused_add_rms_norm", T, H, 2, 16)
+    hx, hr, out = wl.x.clone(), wl.residual.clone(), torch.empty_like(wl.x)
+    w_host = wl.weight.clone().pin_memory()
+    with pytest.raises(ValueError):
+        rn.host_fused_add_rms_norm(out, hx, hr, w_host, wl.eps, pipe)
+    st = rn.lib.rn_host_fused_add_rms_norm(rn._desc(out, 0), rn._desc(hx, 1), rn._desc(hr, 2),
+                                           rn._desc(w_host, 3), wl.eps, -1,
+                                           pipe.descriptor_ref())
+    torch.cuda.synchronize()
+    assert rn.STATUS[st] == "RN_ERR_LAYOUT"
+    assert torch.equal(hr.view(torch.int16), wl.residual.view(torch.int16))

@@ -386,7 +386,7 @@ def run_ours(args, world, rank, local):
 
     # end to end through the public API with host buffers: pinned H2D of each
     # launch's inputs, the two launches, D2H of every output, all timed.
-    e2e = run_e2e(args, rn, wl, S, device, stream)
+    e2e = run_e2e(args, rn, wl, S, device, stream, world)
     del S
     torch.cuda.empty_cache()
 
@@ -439,12 +439,14 @@ def run_ours(args, world, rank, local):
 E2E_STREAMS = 2
 
 
-def run_e2e(args, rn, wl, S, device, stream):
+def run_e2e(args, rn, wl, S, device, stream, world=1):
     """The step end to end through the host-memory entry points (C ABI
     rn_host_fused_add_rms_norm / rn_host_fused_add_rms_norm_fp8): inputs and
     outputs in page-locked host memory, every byte crossing the host link
     inside the timed region, each op chunked over its own two streams so
-    that copies in, kernels and copies out overlap."""
+    that copies in, kernels and copies out overlap. With several ranks each
+    streams its own copy of the step over its own host link; the time is the
+    slowest rank's and the value counts every rank's bytes."""
     from residual_add_rmsnorm_rms_b200.host import HostPipeline
     T, H = wl.T, wl.H
     pin = lambda t: t.cpu().clone().pin_memory()  # noqa: E731
@@ -477,6 +479,7 @@ def run_e2e(args, rn, wl, S, device, stream):
     join()
     torch.cuda.synchronize(device)
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
     e0.record(stream)
     pa.wait_for(stream)
     pb.wait_for(stream)
@@ -485,12 +488,13 @@ def run_e2e(args, rn, wl, S, device, stream):
     join()
     e1.record(stream)
     torch.cuda.synchronize(device)
-    ms = e0.elapsed_time(e1) / n
+    barrier(world)
+    ms = max_over_ranks(e0.elapsed_time(e1), world, device) / n
     plan = rn.host_plan_chunks("fused_add_rms_norm", T, H, 1 << 50, E2E_STREAMS)
-    return {"value": round(step_bytes(T, H) / (ms / 1e3) / 1e9, 3), "unit": "GB/s",
+    return {"value": round(step_bytes(T, H) * world / (ms / 1e3) / 1e9, 3), "unit": "GB/s",
             "ms_per_step": round(ms, 4), "steps": n,
-            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
-            "link_gbs": round((h2d + d2h) / (ms / 1e3) / 1e9, 2),
+            "h2d_bytes_per_step": h2d * world, "d2h_bytes_per_step": d2h * world,
+            "link_gbs_per_gpu": round((h2d + d2h) / (ms / 1e3) / 1e9, 2),
             "how": "C ABI rn_host_fused_add_rms_norm + rn_host_fused_add_rms_norm_fp8 on "
                    "page-locked host buffers: per op and step, x and residual copied in, "
                    "residual and out (or q and scale) copied back, in "

@@ -4,8 +4,9 @@ that are copied in, normalised on the device and copied back over one to
 four streams. Every result is checked against the CPU oracle on the same
 input bits: ragged last chunks, one-row chunks, one chunk, the scalar
 kernel's rows (H % 8 != 0), pageable and page-locked host memory, in-place
-output, the prefill batch with the automatic chunking, and calls of
-different ops queued back to back through one pipeline."""
+output, the prefill batch with the automatic chunking, calls of different
+ops queued back to back through one pipeline, and a call captured in a CUDA
+graph and replayed."""
 import pytest
 import torch
 
@@ -166,3 +167,35 @@ def test_host_pipeline_refuses_host_weight():
     torch.cuda.synchronize()
     assert rn.STATUS[st] == "RN_ERR_LAYOUT"
     assert torch.equal(hr.view(torch.int16), wl.residual.view(torch.int16))
+
+
+def test_host_pipeline_in_a_cuda_graph():
+    """A host-memory call captured in a CUDA graph (the pipeline's streams fork
+    from and join back into the capturing stream): each replay copies the
+    page-locked rows in, normalises them and copies them back, so two replays
+    apply the fused op twice."""
+    T, H = 600, 4096
+    wl = synth.make_inputs("small", "fused_add_rms_norm", "bf16", T, H)
+    pipe = _pipeline("fused_add_rms_norm", T, H, 2, 128)
+    hx = wl.x.clone().pin_memory()
+    hr = wl.residual.clone().pin_memory()
+    out = torch.empty_like(wl.x).pin_memory()
+    w = wl.weight.cuda()
+    graph = torch.cuda.CUDAGraph()
+    side = torch.cuda.Stream()
+    side.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(side):
+        with torch.cuda.graph(graph, stream=side, capture_error_mode="relaxed"):
+            rn.host_fused_add_rms_norm(out, hx, hr, w, wl.eps, pipe)
+    torch.cuda.synchronize()
+    assert torch.equal(hr.view(torch.int16), wl.residual.view(torch.int16))  # nothing ran yet
+    graph.replay()
+    torch.cuda.synchronize()
+    want = oracle_run("fused_add_rms_norm", wl.x, wl.residual, wl.weight, wl.eps, "bf16")
+    compare("fused_add_rms_norm", {"out": out.clone(), "residual": hr.clone()}, want, "bf16")
+    r1 = torch.from_numpy(want["residual"].view("int16").copy()).view(torch.bfloat16).view(T, H)
+    graph.replay()
+    torch.cuda.synchronize()
+    want2 = oracle_run("fused_add_rms_norm", wl.x, r1, wl.weight, wl.eps, "bf16")
+    compare("fused_add_rms_norm", {"out": out, "residual": hr}, want2, "bf16")
+    del graph

@@ -3,6 +3,7 @@
 // "vllm.kernels.aiter_ops": 16-bit activations, matching weight dtype or
 // None, no variance-size override, free flattening to dense 2-D), aliasing
 // rules, launch planning and the launch itself. Pure host code.
+#include <algorithm>
 #include <cmath>
 #include <cstdlib>
 #include <cstdint>
@@ -837,7 +838,8 @@ HostSlot host_slot(int op, int64_t rows, int64_t H) {
 
 // The most rows of which `slots` slots fit in `bytes` (0 if not one).
 int64_t host_rows_fitting(int op, int64_t H, int64_t bytes, int64_t slots) {
-    const int64_t per_slot = bytes / slots;
+    // capped so that the byte counts below cannot overflow
+    const int64_t per_slot = std::min<int64_t>(bytes / slots, int64_t{1} << 60);
     const int64_t per_row = 2 * H + (op != rn::kRmsNorm ? 2 * H : 0) +
                             (op == rn::kFusedAddFp8 ? H + 4 : 0);
     int64_t rows = per_slot / per_row;

@@ -79,6 +79,10 @@ def test_plan_chunks_errors():
     st, p = status(1, 0, 512, 0, 2, 0)
     assert st == "RN_OK" and (p.chunk_rows, p.chunks, p.slots) == (0, 0, 0)
     assert rn.lib.rn_host_plan_chunks(0, 10, 512, BIG, 2, 0, None) == 1  # RN_ERR_NULL
+    # the largest scratch size plans like any ample one (no overflow)
+    for op in OPS:
+        assert rn.host_plan_chunks(op, 8192, 3840, (1 << 63) - 1, 8) == \
+            rn.host_plan_chunks(op, 8192, 3840, BIG, 8)
     assert ctypes.sizeof(rn.RnHostPipeline) == 8 + 8 + 8 + 4 + 4 + 8  # C layout
     assert ctypes.sizeof(rn.RnHostPlan) == 8 * 3 + 4 + 4
 

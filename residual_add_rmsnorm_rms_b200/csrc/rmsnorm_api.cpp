@@ -218,15 +218,9 @@ bool auto_vector_plan(int op, int64_t T, int64_t H, int num_sms, rn_plan* p) {
     const bool many_rows = tpr4 <= rn::max_block_for_vpt(4) &&
                            static_cast<double>(T) * tpr4 >= 1.0 * num_sms * 1024;
     if (many_rows) {
-        // fused_add_rms_norm: three vectors per thread when they tile the row
-        // exactly and four would leave lanes idle (H = 3840: 160 x 3 against
-        // 128 x 4 = 512 slots for 480 vectors), measured 1.9 % faster on B200
-        if (op == rn::kFusedAdd && idle_of(tpr_for(nvec, 3), 3) == 0.0 && idle_of(tpr4, 4) > 0.0 &&
-            tpr_for(nvec, 3) <= rn::max_block_for_vpt(3)) {
-            const int tpr = tpr_for(nvec, 3);
-            fill_vector_plan(tpr, 3, T, p, rows_per_block(tpr, T));
-            return true;
-        }
+        // Four vectors per thread first. (Three that tile the row exactly beat
+        // four with idle lanes, H = 3840, by 1.9 % for fused_add_rms_norm
+        // with 16-byte accesses; with 32-byte pairs four win by 0.6 %.)
         for (int vpt : {4, 5, 3, 6, 8, 2}) {
             const int tpr = tpr_for(nvec, vpt);
             if (tpr > rn::max_block_for_vpt(vpt) || idle_of(tpr, vpt) > 1.0 / 8) continue;
@@ -478,17 +472,31 @@ rn_status prepare(int op, const rn_tensor* o, const rn_tensor* sc, const rn_tens
     return RN_OK;
 }
 
-// Enqueues the norm kernel `plan` describes.
+// Whether the vector kernel may move its vectors in adjacent pairs with
+// 32-byte accesses: an even vector count per row (H % 16 == 0) and 32-byte
+// aligned 16-bit rows (x, and out or residual where written; the weight is
+// read 16 bytes at a time), 16-byte aligned code rows for the fp8 op.
+bool pair_ok(int op, int64_t H, const void* x, const void* res, const void* out,
+             const void* q) {
+    if (H % 16 != 0 || !aligned(x, 32)) return false;
+    if (op != rn::kRmsNorm && !aligned(res, 32)) return false;
+    if (op != rn::kFusedAddFp8) return aligned(out, 32);
+    return aligned(q, 16);
+}
+
+// Enqueues the norm kernel `plan` describes; `pair` as pair_ok (used by the
+// vector kernel when its vector count per thread is even).
 rn_status launch_plan(int op, int dt, const rn::Args& a, const rn_plan& plan, bool pdl,
-                      void* stream) {
-    const rn::Launch l{plan.kernel,
-                       plan.threads_per_row,
-                       plan.kernel == RN_KERNEL_STAGED ? plan.stages : plan.vectors_per_thread,
-                       plan.rows_per_cta,
-                       plan.block_threads,
-                       plan.smem_bytes,
-                       plan.grid,
-                       pdl};
+                      bool pair, void* stream) {
+    rn::Launch l{plan.kernel,
+                 plan.threads_per_row,
+                 plan.kernel == RN_KERNEL_STAGED ? plan.stages : plan.vectors_per_thread,
+                 plan.rows_per_cta,
+                 plan.block_threads,
+                 plan.smem_bytes,
+                 plan.grid,
+                 pdl};
+    l.pair = pair && plan.kernel == RN_KERNEL_VECTOR && plan.vectors_per_thread % 2 == 0;
     const cudaError_t e = rn::launch(op, dt, a, l, static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) {
         std::snprintf(g_cuda_error, sizeof g_cuda_error, "%s: %s", cudaGetErrorName(e),
@@ -520,7 +528,7 @@ rn_status run(int op, const rn_tensor* o, const rn_tensor* sc, const rn_tensor* 
     a.H = c.x.H;
     a.eps = eps;
     return launch_plan(op, c.dt, a, plan, g_pdl.load() < 0 ? kPdlDefault : g_pdl.load() == 1,
-                       stream);
+                       pair_ok(op, a.H, a.x, a.residual, a.out, a.q), stream);
 }
 
 }  // namespace
@@ -950,7 +958,8 @@ rn_status run_host(int op, const rn_tensor* o, const rn_tensor* sc, const rn_ten
         st = plan_impl(op, rows, H, vector_ok, num_sms, &plan);
         if (st != RN_OK) return st;
         // no programmatic dependent launch: the kernel follows copies
-        st = launch_plan(op, c.dt, a, plan, false, s);
+        st = launch_plan(op, c.dt, a, plan, false, pair_ok(op, H, a.x, a.residual, a.out, a.q),
+                         s);
         if (st != RN_OK) return st;
 
         if (fused) e = cudaMemcpyAsync(c.res.ptr + off16, base + L.r, b16, cudaMemcpyDefault, s);

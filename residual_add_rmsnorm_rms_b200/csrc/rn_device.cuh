@@ -106,6 +106,21 @@ __device__ __forceinline__ void st_v2(uint2* p, const uint2& v) {
     asm volatile("st.global.v2.u32 [%0], {%1, %2};" ::"l"(p), "r"(v.x), "r"(v.y) : "memory");
 }
 
+// 32-byte (256-bit) global accesses, new with sm_100: two adjacent 16-byte
+// vectors in one instruction. The address must be 32-byte aligned.
+__device__ __forceinline__ void ld_stream2(const uint4* p, uint4& a, uint4& b) {
+    asm volatile("ld.global.L1::no_allocate.v8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+                 : "=r"(a.x), "=r"(a.y), "=r"(a.z), "=r"(a.w), "=r"(b.x), "=r"(b.y), "=r"(b.z),
+                   "=r"(b.w)
+                 : "l"(p));
+}
+
+__device__ __forceinline__ void st_v8(uint4* p, const uint4& a, const uint4& b) {
+    asm volatile("st.global.v8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"l"(p), "r"(a.x),
+                 "r"(a.y), "r"(a.z), "r"(a.w), "r"(b.x), "r"(b.y), "r"(b.z), "r"(b.w)
+                 : "memory");
+}
+
 // Barrier over the `nthreads` threads of one row group (ids 1..15; 0 is
 // __syncthreads).
 __device__ __forceinline__ void group_barrier(int id, int nthreads) {

@@ -39,6 +39,7 @@ struct Launch {
     int smem;    // dynamic shared memory bytes
     int64_t grid;
     bool pdl;    // launch with programmatic stream serialization (PDL)
+    bool pair = false;  // vector kernel, even VPT: 32-byte accesses (see rmsnorm_kernels.cu)
 };
 
 enum Op { kRmsNorm = 0, kFusedAdd = 1, kFusedAddFp8 = 2 };

@@ -2,6 +2,7 @@
 
 Ragged hidden sizes (scalar kernel), idle vector slots, every compiled
 vectors-per-thread width and threads-per-row shape (forced), misaligned bases,
+rows aligned for 16-byte but not 32-byte accesses,
 T == 0, in-place out == x, no weight, N-D views, zero rows, fp16 subnormal
 inputs, determinism, the structural identity fused(x, r).out ==
 rms_norm(r'), non-default streams and validation errors on real tensors.
@@ -163,6 +164,51 @@ def test_misaligned_base_uses_scalar_kernel(op):
     torch.cuda.synchronize()
     want = oracle_run(op, x, r, w, 1e-6, "bf16")
     compare(op, got, want, "bf16")
+
+
+def _offset_view(t, elems):
+    """A copy of `t` on the device whose data starts `elems` elements past a
+    fresh allocation (which is at least 256-byte aligned)."""
+    buf = torch.empty(t.numel() + elems, dtype=t.dtype, device="cuda")
+    v = buf[elems:].view(t.shape)
+    v.copy_(t.cuda() if not t.is_cuda else t)
+    return v
+
+
+@pytest.mark.parametrize("op", OPS)
+@pytest.mark.parametrize("offset", [8, 16])
+def test_16_byte_but_not_32_byte_aligned_rows(op, offset):
+    """Rows 16-byte but not 32-byte aligned (offset 8 elements: x, residual,
+    out; offset 16 keeps them 32-byte aligned) with an even vector count per
+    thread: the vector kernel with single 16-byte accesses, or with 32-byte
+    pairs, both checked in full against the oracle."""
+    T, H = 67, 3840
+    x, r, w = _inputs(T, H, "bf16", seed=31 + offset)
+    assert rn.plan_launch(op, torch.bfloat16, T, H)["vectors_per_thread"] % 2 == 0
+    xs = _offset_view(x, offset)
+    rs = None if op == "rms_norm" else _offset_view(r, offset)
+    out = None
+    if op != "fused_add_rms_norm_fp8":
+        out = _offset_view(torch.zeros(T, H, dtype=torch.bfloat16), offset)
+    got = gpu_run(op, xs, rs, w.cuda(), 1e-6, out=out)
+    torch.cuda.synchronize()
+    compare(op, got, oracle_run(op, x, r, w, 1e-6, "bf16"), "bf16")
+
+
+@pytest.mark.parametrize("op", ["fused_add_rms_norm_fp8"])
+def test_fp8_codes_8_byte_aligned(op):
+    """Codes 8-byte but not 16-byte aligned: the fp8 op stores them 8 bytes
+    at a time even when x and the residual allow 32-byte pairs."""
+    T, H = 40, 4096
+    x, r, w = _inputs(T, H, "bf16", seed=41)
+    qb = torch.empty(T * H + 8, dtype=torch.float8_e4m3fn, device="cuda")
+    q = qb[8:].view(T, H)
+    scale = torch.empty(T, dtype=torch.float32, device="cuda")
+    rr = r.cuda().clone()
+    rn.fused_add_rms_norm_fp8(q, scale, x.cuda(), rr, w.cuda(), 1e-6)
+    torch.cuda.synchronize()
+    compare(op, {"q": q, "scale": scale, "residual": rr}, oracle_run(op, x, r, w, 1e-6, "bf16"),
+            "bf16")
 
 
 @pytest.mark.parametrize("op", OPS)

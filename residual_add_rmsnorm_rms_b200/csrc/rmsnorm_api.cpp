@@ -587,6 +587,10 @@ rn_status rn_silu_and_mul_fp8(const rn_tensor* q, const rn_tensor* scale, const 
                  plan.smem_bytes,
                  plan.grid,
                  g_pdl.load() < 0 ? kPdlDefault : g_pdl.load() == 1};
+    // 32-byte pairs: an even vector count per thread, I % 16 == 0 (gate and up
+    // rows then start 32-byte aligned), 32-byte aligned x and 16-byte aligned q
+    l.pair = plan.kernel == RN_KERNEL_VECTOR && plan.vectors_per_thread % 2 == 0 && I % 16 == 0 &&
+             aligned(fx.ptr, 32) && aligned(fq.ptr, 16);
     const cudaError_t e = rn::launch_swiglu_fp8(x->dtype == RN_BF16 ? rn::kBF16 : rn::kF16, a, l,
                                                 static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) {

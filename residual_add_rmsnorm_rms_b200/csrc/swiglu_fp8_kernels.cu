@@ -11,7 +11,10 @@
 // output element), so the same register-resident mapping is used: `tpr`
 // threads per row, VPT 16-byte vectors of gate and of up per thread, all
 // loads issued before use, one max-reduction per row (warp butterfly, then a
-// named barrier across the row's warps), one pass writing the codes. silu
+// named barrier across the row's warps), one pass writing the codes. With an
+// even VPT, I % 16 == 0, 32-byte aligned x rows and 16-byte aligned code rows
+// (kPair), a thread's vectors come in adjacent pairs moved by sm_100's 32-byte
+// loads (codes: 16-byte stores), as in the norm kernels' vector kernel. silu
 // uses the fast exponential and division intrinsics (two multi-function-unit
 // operations per element): at ~1.3e12 elements/s the accurate forms would
 // make the kernel issue-bound.
@@ -33,9 +36,19 @@ __device__ __forceinline__ float2 swiglu2(float2 g, float2 u) {
     return __fmul2_rn(make_float2(sx, sy), u);
 }
 
-template <typename T, int VPT>
+// Index (in 16-byte vectors) of a thread's vector k: strided by tpr, or with
+// kPair, pair k / 2 strided by tpr and its two vectors adjacent.
+template <bool kPair>
+__device__ __forceinline__ int swiglu_vec_index(int lr, int k, int tpr) {
+    if constexpr (kPair) return 2 * (lr + (k >> 1) * tpr) + (k & 1);
+    return lr + k * tpr;
+}
+
+template <typename T, int VPT, bool kPair>
 __global__ void __launch_bounds__(max_block_for_vpt(VPT))
     rn_swiglu_fp8_kernel(const SwigluArgs a, const int tpr, const int rpc) {
+    static_assert(!kPair || VPT % 2 == 0, "pairs need an even vector count");
+    constexpr int kStep = kPair ? 2 : 1;
     using F = Fmt<T>;
     extern __shared__ float red[];  // [2][rpc][warps per row]
     pdl_allow_dependents();
@@ -56,12 +69,22 @@ __global__ void __launch_bounds__(max_block_for_vpt(VPT))
         const uint4* urow = grow + ivec;
 
         uint4 g[VPT], u[VPT];
+        const uint4 z4 = make_uint4(0, 0, 0, 0);
 #pragma unroll
-        for (int k = 0; k < VPT; ++k) {
-            const int j = lr + k * tpr;
+        for (int k = 0; k < VPT; k += kStep) {
+            const int j = swiglu_vec_index<kPair>(lr, k, tpr);
             const bool ok = active && j < ivec;
-            g[k] = ok ? ld_stream(grow + j) : make_uint4(0, 0, 0, 0);
-            u[k] = ok ? ld_stream(urow + j) : make_uint4(0, 0, 0, 0);
+            if constexpr (kPair) {
+                if (ok) {
+                    ld_stream2(grow + j, g[k], g[k + 1]);
+                    ld_stream2(urow + j, u[k], u[k + 1]);
+                } else {
+                    g[k] = g[k + 1] = u[k] = u[k + 1] = z4;
+                }
+            } else {
+                g[k] = ok ? ld_stream(grow + j) : z4;
+                u[k] = ok ? ld_stream(urow + j) : z4;
+            }
         }
         float2 y[VPT][4];
         float pm = 0.f;
@@ -92,10 +115,7 @@ __global__ void __launch_bounds__(max_block_for_vpt(VPT))
         const float2 q2 = make_float2(qmul, qmul);
         if (active && lr == 0) a.scale[row] = pm > 0.f ? pm / 448.0f : 0.f;
         uint2* qrow = reinterpret_cast<uint2*>(a.q) + r0 * ivec;
-#pragma unroll
-        for (int k = 0; k < VPT; ++k) {
-            const int j = lr + k * tpr;
-            if (!(active && j < ivec)) continue;
+        auto codes = [&](int k) {
             uint32_t e[4];
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
@@ -104,7 +124,19 @@ __global__ void __launch_bounds__(max_block_for_vpt(VPT))
             }
             uint2 o = make_uint2(e[0] | (e[1] << 16), e[2] | (e[3] << 16));
             if (!(pm > 0.f)) o = make_uint2(0, 0);
-            st_v2(qrow + j, o);
+            return o;
+        };
+#pragma unroll
+        for (int k = 0; k < VPT; k += kStep) {
+            const int j = swiglu_vec_index<kPair>(lr, k, tpr);
+            if (!(active && j < ivec)) continue;
+            const uint2 o = codes(k);
+            if constexpr (kPair) {
+                const uint2 o1 = codes(k + 1);
+                st_v4(reinterpret_cast<uint4*>(qrow + j), make_uint4(o.x, o.y, o1.x, o1.y));
+            } else {
+                st_v2(qrow + j, o);
+            }
         }
     }
 }
@@ -148,8 +180,15 @@ __global__ void __launch_bounds__(kSwigluScalarBlock) rn_swiglu_fp8_scalar_kerne
 template <typename T, int I = 0>
 cudaError_t swiglu_dispatch_vpt(const SwigluArgs& a, const Launch& l, cudaStream_t s) {
     if constexpr (I < kNumVpt) {
-        if (l.vpt == kVptList[I])
-            return launch_kernel(rn_swiglu_fp8_kernel<T, kVptList[I]>, l, s, a, l.tpr, l.rpc);
+        if (l.vpt == kVptList[I]) {
+            if constexpr (kVptList[I] % 2 == 0) {
+                if (l.pair)
+                    return launch_kernel(rn_swiglu_fp8_kernel<T, kVptList[I], true>, l, s, a,
+                                         l.tpr, l.rpc);
+            }
+            return launch_kernel(rn_swiglu_fp8_kernel<T, kVptList[I], false>, l, s, a, l.tpr,
+                                 l.rpc);
+        }
         return swiglu_dispatch_vpt<T, I + 1>(a, l, s);
     } else {
         return cudaErrorInvalidValue;

@@ -193,17 +193,23 @@ __device__ __forceinline__ void vector_rows(const Args& a, const int tpr, const 
             for (int k = 0; k < VPT; k += kStep) {
                 const int j = vec_index<kPair>(lr, k, tpr);
                 if (!(active && j < nvec)) continue;
-                uint4 w = make_uint4(0, 0, 0, 0);
-                if constexpr (kHasW) w = __ldg(wv + j);
-                uint2 o = quant8<T, kHasW>(v[k], w, q2);
-                if (!(pm > 0.f)) o = make_uint2(0, 0);
+                // (both codes computed before the zero-row test: the other
+                // order put a 16-byte temporary in local memory)
                 if constexpr (kPair) {
-                    uint4 w1 = make_uint4(0, 0, 0, 0);
-                    if constexpr (kHasW) w1 = __ldg(wv + j + 1);
+                    uint4 w0 = make_uint4(0, 0, 0, 0), w1 = w0;
+                    if constexpr (kHasW) {
+                        w0 = __ldg(wv + j);
+                        w1 = __ldg(wv + j + 1);
+                    }
+                    uint2 o0 = quant8<T, kHasW>(v[k], w0, q2);
                     uint2 o1 = quant8<T, kHasW>(v[k + 1], w1, q2);
-                    if (!(pm > 0.f)) o1 = make_uint2(0, 0);
-                    st_v4(reinterpret_cast<uint4*>(qrow + j), make_uint4(o.x, o.y, o1.x, o1.y));
+                    if (!(pm > 0.f)) o0 = o1 = make_uint2(0, 0);
+                    st_v4(reinterpret_cast<uint4*>(qrow + j), make_uint4(o0.x, o0.y, o1.x, o1.y));
                 } else {
+                    uint4 w = make_uint4(0, 0, 0, 0);
+                    if constexpr (kHasW) w = __ldg(wv + j);
+                    uint2 o = quant8<T, kHasW>(v[k], w, q2);
+                    if (!(pm > 0.f)) o = make_uint2(0, 0);
                     st_v2(qrow + j, o);
                 }
             }

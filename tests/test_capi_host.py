@@ -262,6 +262,26 @@ def test_planner_invariants(op):
     assert rn.plan_launch(op, BF, 4, 1 << 17)["kernel"] == 1
 
 
+def test_planner_measured_choices():
+    """The launch shapes the forced-shape sweeps on B200 chose: four vectors
+    per thread at H = 3840 (they move as two 32-byte pairs), blocks of about
+    256 threads for rms_norm and 256/512 for the fused ops."""
+    def shape(op, T, H):
+        p = rn.plan_launch(op, BF, T, H)
+        return p["threads_per_row"], p["vectors_per_thread"], p["rows_per_cta"]
+    for op in ("fused_add_rms_norm", "fused_add_rms_norm_fp8"):
+        assert shape(op, 8192, 3840) == (128, 4, 2)
+        assert shape(op, 32768, 4096) == (128, 4, 4)
+        assert shape(op, 32768, 8192) == (256, 4, 2)
+        assert shape(op, 4096, 5120) == (160, 4, 2)
+    assert shape("rms_norm", 8192, 3840) == (128, 4, 2)
+    assert shape("rms_norm", 32768, 4096) == (128, 4, 2)
+    assert shape("rms_norm", 32768, 2048) == (64, 4, 4)
+    assert shape("rms_norm", 4096, 5120) == (160, 4, 2)  # 160-thread rows: two per block
+    assert shape("rms_norm", 4096, 7168) == (224, 4, 1)
+    assert shape("rms_norm", 32768, 8192) == (256, 4, 1)
+
+
 def test_force_plan_hook():
     with pytest.raises(rn.RmsNormError):
         rn.force_plan(48, 4)  # not a power of two <= 32 nor a multiple of 32

@@ -313,8 +313,13 @@ RN_API rn_status rn_allreduce_fused_add_rms_norm_fp8(const rn_tensor* q, const r
 
 /* ---- the whole group on one device, with the library's own exchange memory
  *
- * No counterpart on the pages: they describe no such entry point. This is
- * rn_allreduce_fused_add_rms_norm for a group of `world` ranks all held on
+ * No counterpart on the pages: they describe no such entry point. It is for
+ * callers that cannot allocate device memory: a plugin or kernel library
+ * running inside a host framework that owns every allocation (its caching
+ * allocator, or a fixed arena handed out at start-up) and gives the plugin
+ * no way to ask for more, or code that may run while a stream is being
+ * captured, where an allocation would be recorded into the graph or refused.
+ * This is rn_allreduce_fused_add_rms_norm for a group of `world` ranks all held on
  * the current device (operands stacked [world, T, H], as with local_ranks ==
  * world; one launch computes every rank), whose exchange buffers and signal
  * pads live in a static device array of the library instead of caller
@@ -322,15 +327,19 @@ RN_API rn_status rn_allreduce_fused_add_rms_norm_fp8(const rn_tensor* q, const r
  * Capacity: world * round_up(4 * T * H + 32, 256) <= RN_LOCAL_EXCHANGE_BYTES
  * (32 MiB of buffers, plus 8 signal pads), else RN_ERR_CAPACITY before any
  * CUDA call; world outside 1..8 is RN_ERR_COMM; otherwise the checks and
- * errors of rn_allreduce_fused_add_rms_norm, with the AUTO algorithm (buffers
- * sized for two-shot when world * round_up(12 * T * H + 32, 256) fits). The
- * first call on a device looks the array up (the device must be current, as
- * for every call), and the first call with a given `world` after another
- * clears the signal pads with cudaMemsetAsync on `stream`: make those calls
- * outside stream capture (RN_ERR_CONFIG inside); later calls may be
- * captured. The memory is shared by every call on a device: calls that
- * overlap in time (other streams, other threads) race and give undefined
- * results. */
+ * errors of rn_allreduce_fused_add_rms_norm, with the AUTO algorithm (from
+ * three ranks on, buffers sized for two-shot when
+ * world * round_up(12 * T * H + 32, 256) fits; successive calls may then
+ * alternate between one-shot and two-shot on the same signal pads, which is
+ * safe because a flag is compared with the call number for equality). The
+ * first call in a device's context looks the array up (the device must be
+ * current, as for every call; a context re-created after a device reset
+ * counts as new), and that call and the first call with a given `world`
+ * after another clear the signal pads with cudaMemsetAsync on `stream`: make
+ * those calls outside stream capture (RN_ERR_CONFIG inside). The memory is
+ * shared by every call on a device and keeps what the last call left in it:
+ * calls that overlap in time (other streams, other threads) race and give
+ * undefined results. */
 #define RN_LOCAL_EXCHANGE_BYTES 33554432
 RN_API rn_status rn_allreduce_fused_add_rms_norm_local(const rn_tensor* out, const rn_tensor* x,
                                                        const rn_tensor* residual,
@@ -499,12 +508,27 @@ RN_API rn_status rn_force_staged(int32_t ctas_per_sm, int32_t stages, int32_t th
  * values. Not thread-safe with concurrent launches. */
 RN_API rn_status rn_set_launch_options(int32_t pdl, int64_t max_grid);
 
+/* L2 prefetch across the kernel boundary for every later call in the
+ * process (tuning hook): with mode = 1, a norm vector-kernel launch made with
+ * programmatic dependent launch asks L2 for its blocks' first rows of x (and
+ * the residual) before it waits for the previous kernel in the stream, so
+ * HBM keeps streaming while that kernel drains. A prefetch is a hint: the
+ * values every load returns are unchanged. 0 turns it off, -1 restores the
+ * library default (on); RN_ERR_CONFIG for other values. Not thread-safe with
+ * concurrent launches. */
+RN_API rn_status rn_set_prefetch(int32_t mode);
+
 /* Reads and clears the device-side error flags of the current device:
  * bit 0 = a bounded wait inside the STAGED kernel timed out (some rows of
  * that call were not written); bit 1 = an all-reduce call waited longer than
  * its timeout for a peer (some rows of that call were not written).
  * Synchronises with the device. */
 RN_API rn_status rn_device_errors(uint32_t* flags);
+
+/* The compute capability (major * 10 + minor: 100 for sm_100a) that the
+ * library's device code loaded on the current device was compiled for.
+ * Loads the code if needed; RN_ERR_CUDA without a usable device. */
+RN_API rn_status rn_kernel_binary_version(int32_t* version);
 
 /* Writes up to `cap` compiled vectors_per_thread values into `out` and
  * returns how many exist. */

@@ -31,7 +31,8 @@ __all__ = [
     "host_plan_chunks", "RnHostPipeline", "RnHostPlan", "HOST_MAX_STREAMS",
     "RnAllreduceComm", "ALLREDUCE_MAX_WORLD", "ALLREDUCE_SIGNAL_BYTES", "ALLREDUCE_ALGORITHMS",
     "plan_launch", "validate", "force_plan", "force_staged",
-    "set_launch_options", "device_errors", "supported_vectors_per_thread", "status_string",
+    "set_launch_options", "set_prefetch", "device_errors", "supported_vectors_per_thread",
+    "status_string", "kernel_binary_version", "MAX_DIMS", "LOCAL_EXCHANGE_BYTES",
     "LIB_PATH", "lib", "RnTensor", "RnPlan", "STATUS", "OPS",
 ]
 
@@ -49,6 +50,9 @@ _DTYPES = {torch.float16: 0, torch.bfloat16: 1, torch.float8_e4m3fn: 2, torch.fl
            torch.uint8: 2}
 
 
+# Restated from include/rmsnorm_b200.h (a CPU test checks they agree).
+MAX_DIMS = 8
+LOCAL_EXCHANGE_BYTES = 33554432
 ALLREDUCE_MAX_WORLD = 8
 ALLREDUCE_SIGNAL_BYTES = 131136
 ALLREDUCE_ALGORITHMS = {"auto": 0, "one_shot": 1, "two_shot": 2}
@@ -180,6 +184,10 @@ def _load():
     L.rn_force_staged.restype = ctypes.c_int
     L.rn_set_launch_options.argtypes = [ctypes.c_int32, ctypes.c_int64]
     L.rn_set_launch_options.restype = ctypes.c_int
+    L.rn_kernel_binary_version.argtypes = [ctypes.POINTER(ctypes.c_int32)]
+    L.rn_kernel_binary_version.restype = ctypes.c_int
+    L.rn_set_prefetch.argtypes = [ctypes.c_int32]
+    L.rn_set_prefetch.restype = ctypes.c_int
     L.rn_device_errors.argtypes = [ctypes.POINTER(ctypes.c_uint32)]
     L.rn_device_errors.restype = ctypes.c_int
     L.rn_supported_vectors_per_thread.argtypes = [ctypes.POINTER(ctypes.c_int32), ctypes.c_int32]
@@ -478,6 +486,19 @@ def force_staged(ctas_per_sm: int, stages: int, threads: int) -> None:
 def set_launch_options(pdl: int = -1, max_grid: int = 0) -> None:
     """Tuning hook: pdl 1/0/-1 (on/off/default) and a cap on blocks launched (0 = none)."""
     _check(lib.rn_set_launch_options(pdl, max_grid), "rn_set_launch_options")
+
+
+def set_prefetch(mode: int = -1) -> None:
+    """Tuning hook: L2 prefetch of the first rows before waiting for the
+    previous kernel (1 on, 0 off, -1 library default)."""
+    _check(lib.rn_set_prefetch(mode), "rn_set_prefetch")
+
+
+def kernel_binary_version() -> int:
+    """Compute capability the loaded device code was built for (100 = sm_100a)."""
+    v = ctypes.c_int32(0)
+    _check(lib.rn_kernel_binary_version(ctypes.byref(v)), "rn_kernel_binary_version")
+    return int(v.value)
 
 
 def device_errors() -> int:

@@ -65,6 +65,33 @@ def cutlass_include() -> list[str]:
     raise RuntimeError("no CUTLASS 4 header tree with sm100 support found on the Python path")
 
 
+def _deps(path: str, seen: set | None = None) -> set:
+    """`path` and every repository header it includes, transitively."""
+    seen = set() if seen is None else seen
+    if path in seen or not os.path.exists(path):
+        return seen
+    seen.add(path)
+    with open(path, errors="replace") as f:
+        for line in f:
+            line = line.strip()
+            if line.startswith("#include") and '"' in line:
+                inc = line.split('"')[1]
+                _deps(os.path.normpath(os.path.join(os.path.dirname(path), inc)), seen)
+    return seen
+
+
+def _obj(src: str) -> str:
+    return os.path.join(OBJDIR, os.path.basename(src) + ".o")
+
+
+def _obj_stale(src: str) -> bool:
+    obj = _obj(src)
+    if not os.path.exists(obj):
+        return True
+    t = os.path.getmtime(obj)
+    return any(os.path.getmtime(p) > t for p in _deps(src) | {__file__})
+
+
 def _stale() -> bool:
     if not os.path.exists(LIB):
         return True
@@ -79,9 +106,11 @@ def nvcc() -> str:
     raise RuntimeError("nvcc not found: the CUDA toolkit is required to build the library")
 
 
-def _compile(src: str, verbose_ptxas: bool) -> str:
+def _compile(src: str, verbose_ptxas: bool, force: bool = True) -> str:
     name = os.path.basename(src)
-    obj = os.path.join(OBJDIR, name + ".o")
+    obj = _obj(src)
+    if not force and not _obj_stale(src):
+        return obj
     cmd = [nvcc(), *NVCC_FLAGS]
     if name in CUTLASS_SOURCES:
         cmd += CUTLASS_FLAGS + cutlass_include()
@@ -97,8 +126,11 @@ def build(force: bool = False, verbose_ptxas: bool = False) -> str:
         return LIB
     os.makedirs(OBJDIR, exist_ok=True)
     srcs = sources()
+    # Objects are rebuilt when their source or an included header changed
+    # (all of them with force or verbose_ptxas).
+    every = force or verbose_ptxas
     with ThreadPoolExecutor(max(1, min(len(srcs), os.cpu_count() or 1))) as ex:
-        objs = list(ex.map(lambda s: _compile(s, verbose_ptxas), srcs))
+        objs = list(ex.map(lambda s: _compile(s, verbose_ptxas, every), srcs))
     tmp = LIB + f".tmp{os.getpid()}"
     subprocess.check_call([nvcc(), *ARCH, "-shared", *objs, "-o", tmp, "-lcuda"])
     os.replace(tmp, LIB)

@@ -217,11 +217,40 @@ __device__ __forceinline__ void vector_rows(const Args& a, const int tpr, const 
     }
 }
 
+// Bytes of a row one L2 prefetch covers.
+constexpr uint32_t kPrefetchChunk = 4096;
+
+// L2 prefetch of the rows of the block's first row group (x, and the
+// residual for the fused ops), spread over the row group's threads in
+// 4 KB pieces. Rows are 16-byte aligned and 2H is a multiple of 16 here.
+template <int OP>
+__device__ __forceinline__ void prefetch_first_rows(const Args& a, const int tpr, const int rpc) {
+    const int row_in_cta = threadIdx.x / tpr;
+    const int lr = threadIdx.x - row_in_cta * tpr;
+    const int64_t row = static_cast<int64_t>(blockIdx.x) * rpc + row_in_cta;
+    if (row >= a.T) return;
+    const uint32_t row_bytes = static_cast<uint32_t>(a.H) * 2u;
+    const char* xr = static_cast<const char*>(a.x) + row * row_bytes;
+    const char* rr = static_cast<const char*>(a.residual) + row * row_bytes;
+    for (uint32_t off = static_cast<uint32_t>(lr) * kPrefetchChunk; off < row_bytes;
+         off += static_cast<uint32_t>(tpr) * kPrefetchChunk) {
+        const uint32_t n = row_bytes - off < kPrefetchChunk ? row_bytes - off : kPrefetchChunk;
+        prefetch_l2(xr + off, n);
+        if constexpr (OP != kRmsNorm) prefetch_l2(rr + off, n);
+    }
+}
+
+// `prefetch` (set only under programmatic dependent launch): before waiting
+// for the previous kernel in the stream, the block asks L2 for its first
+// rows. Blocks become resident while the previous kernel drains, so HBM
+// keeps streaming across the kernel boundary instead of idling for one load
+// latency, and the first loads after the wait hit L2.
 template <typename T, int VPT, int OP, bool kPair>
 __global__ void __launch_bounds__(max_block_for_vpt(VPT))
-    rn_vector_kernel(const Args a, const int tpr, const int rpc) {
+    rn_vector_kernel(const Args a, const int tpr, const int rpc, const int prefetch) {
     extern __shared__ float2 red[];  // [2][rpc][warps per row]
     pdl_allow_dependents();
+    if (prefetch) prefetch_first_rows<OP>(a, tpr, rpc);
     pdl_wait_for_prior_grid();
     if (a.weight)
         vector_rows<T, VPT, OP, true, kPair>(a, tpr, rpc, red);
@@ -517,10 +546,12 @@ __global__ void __launch_bounds__(kScalarBlock) rn_scalar_kernel(const Args a) {
 
 template <typename T, int OP, int VPT>
 cudaError_t launch_vector(const Args& a, const Launch& l, cudaStream_t s) {
+    const int pf = l.prefetch && l.pdl ? 1 : 0;
     if constexpr (VPT % 2 == 0) {
-        if (l.pair) return launch_kernel(rn_vector_kernel<T, VPT, OP, true>, l, s, a, l.tpr, l.rpc);
+        if (l.pair)
+            return launch_kernel(rn_vector_kernel<T, VPT, OP, true>, l, s, a, l.tpr, l.rpc, pf);
     }
-    return launch_kernel(rn_vector_kernel<T, VPT, OP, false>, l, s, a, l.tpr, l.rpc);
+    return launch_kernel(rn_vector_kernel<T, VPT, OP, false>, l, s, a, l.tpr, l.rpc, pf);
 }
 
 template <typename T, int OP, int I = 0>
@@ -586,6 +617,13 @@ cudaError_t read_and_clear_device_errors(unsigned* flags) {
         const unsigned zero = 0;
         e = cudaMemcpyToSymbol(g_rn_device_error, &zero, sizeof zero);
     }
+    return e;
+}
+
+cudaError_t kernel_binary_version(int* version) {
+    cudaFuncAttributes attr;
+    const cudaError_t e = cudaFuncGetAttributes(&attr, rn_scalar_kernel<__nv_bfloat16, kRmsNorm>);
+    if (e == cudaSuccess) *version = attr.binaryVersion;
     return e;
 }
 

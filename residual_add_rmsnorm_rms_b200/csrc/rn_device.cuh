@@ -147,6 +147,15 @@ __device__ __forceinline__ void pdl_wait_for_prior_grid() {
     asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
+// Asks the bulk-copy unit to bring `bytes` (a multiple of 16) from 16-byte
+// aligned global address `p` into L2. Nothing reaches the SM and nothing
+// waits for it; it is a hint without effect on what later loads return (L2
+// is the device's point of coherence, so a line that another kernel writes
+// after the prefetch is read back with that write).
+__device__ __forceinline__ void prefetch_l2(const void* p, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(p), "r"(bytes) : "memory");
+}
+
 
 // Launches `kernel` with the plan's shape, with the PDL attribute when asked.
 template <typename... KArgs, typename... Args2>

@@ -40,6 +40,7 @@ struct Launch {
     int64_t grid;
     bool pdl;    // launch with programmatic stream serialization (PDL)
     bool pair = false;  // vector kernel, even VPT: 32-byte accesses (see rmsnorm_kernels.cu)
+    bool prefetch = false;  // vector kernel under PDL: L2 prefetch of the first rows (ibid.)
 };
 
 enum Op { kRmsNorm = 0, kFusedAdd = 1, kFusedAddFp8 = 2 };
@@ -63,6 +64,10 @@ cudaError_t launch(int op, int dtype, const Args& a, const Launch& l, cudaStream
 
 // Enqueues the fused SwiGLU + FP8 cast (vector plan: kernel 0; scalar: 1).
 cudaError_t launch_swiglu_fp8(int dtype, const SwigluArgs& a, const Launch& l, cudaStream_t s);
+
+// The compute capability (major * 10 + minor) the library's device code
+// loaded on the current device was compiled for.
+cudaError_t kernel_binary_version(int* version);
 
 // Reads, and clears when set, the device-side error flags of the current
 // device (bit 0: an mbarrier wait timed out). Synchronous.

@@ -335,3 +335,9 @@ def test_errors_on_real_tensors_launch_nothing():
     assert e.value.name == "RN_ERR_WEIGHT_DTYPE"
     torch.cuda.synchronize()
     assert torch.equal(r, r0)  # nothing ran
+
+
+def test_loaded_device_code_is_sm100a():
+    """The device code the library loaded was compiled for compute
+    capability 10.0 (sm_100a is the only target the build emits)."""
+    assert rn.kernel_binary_version() == 100

@@ -65,6 +65,21 @@ def test_no_alloc_group_size_changes():
         assert torch.equal(rb.view(torch.int16), ra.view(torch.int16)), (W, T)
 
 
+def test_no_alloc_two_shot_then_one_shot_then_two_shot():
+    """Calls the automatic choice runs two-shot in the static memory (eight
+    ranks of [40 x 8192]: two-shot saves 8.75 * 40 * 8192 = 2.87 MB of peer
+    reads per rank, above the 2.3 MB threshold, and eight buffers of
+    round_up(12 * 40 * 8192 + 32, 256) bytes, 31.5 MB, fit the 32 MiB), with a
+    one-shot call of the same group size ([2 x 8192] per rank) in between,
+    each bit for bit against the entry point with caller memory."""
+    W, H = 8, 8192
+    for T in (40, 2, 40):
+        comm = AllReduceComm.single_device(W, T, H, "cuda")
+        _, (oa, ra), (ob, rb) = _both(W, T, H, 970 + T, comm)
+        assert torch.equal(ob.view(torch.int16), oa.view(torch.int16)), T
+        assert torch.equal(rb.view(torch.int16), ra.view(torch.int16)), T
+
+
 def test_no_alloc_capacity_and_arguments():
     W, H = 8, 4096
     T = (32 << 20) // (W * 4 * H) + 1  # one row per rank too many

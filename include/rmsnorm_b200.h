@@ -151,9 +151,10 @@ RN_API rn_status rn_fused_add_rms_norm_fp8(const rn_tensor* q, const rn_tensor* 
  * skipping Nvidia lock-in" ("the SwiGLU activation function, again merging
  * it with an FP8 cast"). Per row of x = [gate | up] ([T x 2I], fp16/bf16,
  * gate in the first half): y_i = silu(gate_i) * up_i with silu(a) =
- * a / (1 + e^-a) in fp32 (fast exponential and division; relative error of y
- * below 1e-6 for |gate| <= 6; silu(a) = 0 for a < -87.3, where its true
- * magnitude is below 1e-36), scale[t] = max|y| / 448, q = e4m3fn(RNE, satfinite)
+ * a / (1 + e^-a) in fp32 (a base-2 exponential of an argument carried in two
+ * floats and a reciprocal: relative error of y a few ulp, below 1e-6, for
+ * any finite gate; silu(a) = 0 for a < -87.3, where its true magnitude is
+ * below 1e-36), scale[t] = max|y| / 448, q = e4m3fn(RNE, satfinite)
  * (y / scale); a row with max|y| = 0 gets scale 0 and zero codes.
  * q: [T x I] RN_E4M3 dense; scale: T RN_F32 dense; x: any view whose flattening
  * to [T x 2I] is free (the rules of the norm ops). 2I must be even.
@@ -509,9 +510,10 @@ RN_API rn_status rn_force_staged(int32_t ctas_per_sm, int32_t stages, int32_t th
 RN_API rn_status rn_set_launch_options(int32_t pdl, int64_t max_grid);
 
 /* L2 prefetch across the kernel boundary for every later call in the
- * process (tuning hook): with mode = 1, a norm vector-kernel launch made with
- * programmatic dependent launch asks L2 for its blocks' first rows of x (and
- * the residual) before it waits for the previous kernel in the stream, so
+ * process (tuning hook): with mode = 1, a vector-kernel launch of the norm ops
+ * or of silu_and_mul_fp8 made with programmatic dependent launch asks L2 for
+ * its blocks' first rows of x (and the residual) before it waits for the
+ * previous kernel in the stream, so
  * HBM keeps streaming while that kernel drains. A prefetch is a hint: the
  * values every load returns are unchanged. 0 turns it off, -1 restores the
  * library default (on); RN_ERR_CONFIG for other values. Not thread-safe with

@@ -45,8 +45,9 @@ std::atomic<int> g_prefetch{-1};         // -1 default, 0 off, 1 on
 std::atomic<int> g_force_gemm{-1};       // fp8 GEMM tile configuration; -1: automatic
 // Launch defaults, measured on B200 (prefill [8192 x 3840], two ops
 // alternating in one stream): programmatic dependent launch lets the next
-// kernel's blocks start as this one drains (+4-5 %), and capping the vector
-// kernel's grid at 16 blocks per SM (blocks then stride over rows) adds ~1 %.
+// kernel's blocks start as this one drains (+4-5 %); rms_norm and the fused
+// ops on fewer rows cap the vector kernel's grid at 16 blocks per SM (blocks
+// then stride over rows; see default_grid_cap).
 // The L2 prefetch of each block's first rows before it waits for the
 // previous kernel keeps HBM busy across the kernel boundary: the prefill
 // step 73.84 -> 71.33 us, [4096 x H] cells of the sweep 2-10 % faster,
@@ -233,6 +234,39 @@ int rows_per_block(int op, int tpr, int64_t T) {
     return 1;
 }
 
+// Row count from which the fused ops run an uncapped grid (one row group per
+// block), and the one from which the fp8 op's blocks grow to ~512 threads.
+constexpr int64_t kFusedManyRows = 8192;
+constexpr int64_t kFp8WideBlockRows = 16384;
+
+// Rows per block of the fused ops when the rows fill at least a wave, from a
+// grid of forced shapes on B200 with the first-row prefetch (T = 4096-65536,
+// H = 2048-16384; each rule within 1 % of the best shape on average):
+// fused_add_rms_norm, about 512 threads; fused_add_rms_norm_fp8 and the
+// SwiGLU kernel, about 256 threads below kFp8WideBlockRows rows (two rows of
+// 129-256 threads), about 512 from there on.
+int many_rows_per_block(int op, int tpr, int64_t T) {
+    if (op == rn::kRmsNorm) return rows_per_block(op, tpr, T);
+    if (op != rn::kFusedAdd && T < kFp8WideBlockRows) {
+        if (tpr <= 128) return 256 / tpr;
+        return tpr <= 256 ? 2 : 1;
+    }
+    const int r = (512 + tpr / 2) / tpr;
+    return r < 1 ? 1 : r;
+}
+
+// Cap on the vector kernel's grid, in blocks (0: none). With the first-row
+// prefetch, the fused ops on kFusedManyRows rows or more run fastest with one
+// row group per block (2-7 % faster than 16 blocks per SM striding over the
+// rows at T = 16384-65536), and so does the SwiGLU kernel from 4096 rows
+// ([8192 x 15360] 6 % faster, [4096 x 15360] 3 %; [32768 x 15360] 1.8 %
+// slower); otherwise 16 blocks per SM.
+long long default_grid_cap(int op, int64_t T, int num_sms) {
+    if ((op == rn::kFusedAdd || op == rn::kFusedAddFp8) && T >= kFusedManyRows) return 0;
+    if (op == rn::kSwigluFp8 && T >= 4096) return 0;
+    return static_cast<long long>(kVectorBlocksPerSmCap) * num_sms;
+}
+
 bool auto_vector_plan(int op, int64_t T, int64_t H, int num_sms, rn_plan* p) {
     const int64_t nvec = H / 8;
     auto idle_of = [&](int tpr, int vpt) {
@@ -243,13 +277,27 @@ bool auto_vector_plan(int op, int64_t T, int64_t H, int num_sms, rn_plan* p) {
     const bool many_rows = tpr4 <= rn::max_block_for_vpt(4) &&
                            static_cast<double>(T) * tpr4 >= 1.0 * num_sms * 1024;
     if (many_rows) {
+        // Eight vectors per thread, one row per block of 128-256 threads:
+        // half the warps per row of the four-vector plan, so half the
+        // cross-warp reduction. Taken by rms_norm and the fp8 op on rows
+        // that would need 512 threads at four vectors (H = 16384: 2-5 %
+        // faster at T = 4096-65536), and by the fp8 op below kFusedManyRows
+        // rows on rows of 128 or more threads at eight vectors (T = 4096:
+        // H = 7168 4.4 % faster, 8192 2 %; from T = 8192 on, 5-10 % slower).
+        const int tpr8 = tpr_for(nvec, 8);
+        const bool wide = tpr4 >= 512 && (op == rn::kRmsNorm || op == rn::kFusedAddFp8);
+        const bool fp8_few = op == rn::kFusedAddFp8 && T < kFusedManyRows && tpr8 >= 128;
+        if ((wide || fp8_few) && tpr8 <= rn::max_block_for_vpt(8) && idle_of(tpr8, 8) <= 1.0 / 8) {
+            fill_vector_plan(tpr8, 8, T, p, 1);
+            return true;
+        }
         // Four vectors per thread first. (Three that tile the row exactly beat
         // four with idle lanes, H = 3840, by 1.9 % for fused_add_rms_norm
         // with 16-byte accesses; with 32-byte pairs four win by 0.6 %.)
         for (int vpt : {4, 5, 3, 6, 8, 2}) {
             const int tpr = tpr_for(nvec, vpt);
             if (tpr > rn::max_block_for_vpt(vpt) || idle_of(tpr, vpt) > 1.0 / 8) continue;
-            fill_vector_plan(tpr, vpt, T, p, rows_per_block(op, tpr, T));
+            fill_vector_plan(tpr, vpt, T, p, many_rows_per_block(op, tpr, T));
             return true;
         }
     }
@@ -289,8 +337,7 @@ rn_status plan_impl(int op, int64_t T, int64_t H, bool vector_ok, int num_sms, r
     const rn_status st = plan_shape(op, T, H, vector_ok, num_sms, p, allow_staged);
     if (st != RN_OK) return st;
     long long cap = g_max_grid.load();
-    if (cap == 0 && p->kernel == RN_KERNEL_VECTOR)
-        cap = static_cast<long long>(kVectorBlocksPerSmCap) * num_sms;
+    if (cap == 0 && p->kernel == RN_KERNEL_VECTOR) cap = default_grid_cap(op, T, num_sms);
     if (cap > 0 && p->grid > cap) p->grid = cap;
     if (p->grid > 0x7fffffffLL) p->grid = 0x7fffffffLL;
     return RN_OK;
@@ -599,9 +646,10 @@ rn_status rn_silu_and_mul_fp8(const rn_tensor* q, const rn_tensor* scale, const 
     if (overlap(fq, fx) || overlap(fs, fx) || overlap(fq, fs)) return RN_ERR_ALIAS;
     const bool vector_ok = I % 8 == 0 && aligned(fx.ptr, 16) && aligned(fq.ptr, 8);
     rn_plan plan;
-    // The row mapping of the fused norm op on I-wide rows: per output element
-    // it moves 2 x 2 bytes in and 1 byte out, within a few bytes of that op.
-    if ((st = plan_impl(rn::kFusedAddFp8, fx.T, I, vector_ok, device_sms(), &plan, false)) != RN_OK)
+    // The row mapping of the fused norm ops on I-wide rows (rows per block as
+    // for the fp8 op): per output element it moves 2 x 2 bytes in and 1 byte
+    // out, within a few bytes of that op.
+    if ((st = plan_impl(rn::kSwigluFp8, fx.T, I, vector_ok, device_sms(), &plan, false)) != RN_OK)
         return st;
     rn::SwigluArgs a{fx.ptr, reinterpret_cast<uint8_t*>(fq.ptr), reinterpret_cast<float*>(fs.ptr),
                      fx.T, I};
@@ -617,6 +665,7 @@ rn_status rn_silu_and_mul_fp8(const rn_tensor* q, const rn_tensor* scale, const 
     // rows then start 32-byte aligned), 32-byte aligned x and 16-byte aligned q
     l.pair = plan.kernel == RN_KERNEL_VECTOR && plan.vectors_per_thread % 2 == 0 && I % 16 == 0 &&
              aligned(fx.ptr, 32) && aligned(fq.ptr, 16);
+    l.prefetch = g_prefetch.load() < 0 ? kPrefetchDefault : g_prefetch.load() == 1;
     const cudaError_t e = rn::launch_swiglu_fp8(x->dtype == RN_BF16 ? rn::kBF16 : rn::kF16, a, l,
                                                 static_cast<cudaStream_t>(stream));
     if (e != cudaSuccess) {
@@ -1162,7 +1211,7 @@ rn_status rn_plan_launch(int32_t op, int32_t dtype, int64_t T, int64_t H, int32_
     if (op < 0 || op > 3) return RN_ERR_CONFIG;
     if (!is16(dtype)) return RN_ERR_DTYPE;
     if (op == RN_OP_SILU_AND_MUL_FP8)
-        return plan_impl(rn::kFusedAddFp8, T, H, vector_ok != 0, kDefaultSms, plan, false);
+        return plan_impl(rn::kSwigluFp8, T, H, vector_ok != 0, kDefaultSms, plan, false);
     return plan_impl(op, T, H, vector_ok != 0, kDefaultSms, plan);
 }
 

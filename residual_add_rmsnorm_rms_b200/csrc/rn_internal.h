@@ -43,7 +43,8 @@ struct Launch {
     bool prefetch = false;  // vector kernel under PDL: L2 prefetch of the first rows (ibid.)
 };
 
-enum Op { kRmsNorm = 0, kFusedAdd = 1, kFusedAddFp8 = 2 };
+// kSwigluFp8 names the SwiGLU + FP8 kernel to the launch planner only.
+enum Op { kRmsNorm = 0, kFusedAdd = 1, kFusedAddFp8 = 2, kSwigluFp8 = 3 };
 enum Dt { kF16 = 0, kBF16 = 1 };
 
 // Compiled vectors-per-thread widths of the vector kernel, ascending.

@@ -15,9 +15,12 @@
 // even VPT, I % 16 == 0, 32-byte aligned x rows and 16-byte aligned code rows
 // (kPair), a thread's vectors come in adjacent pairs moved by sm_100's 32-byte
 // loads (codes: 16-byte stores), as in the norm kernels' vector kernel. silu
-// uses the fast exponential and division intrinsics (two multi-function-unit
-// operations per element): at ~1.3e12 elements/s the accurate forms would
-// make the kernel issue-bound.
+// takes two multi-function-unit operations per element (a base-2 exponential
+// of an argument carried in two floats, and a reciprocal) and packed
+// two-lane fp32 arithmetic for the rest: at ~1.3e12 elements/s the library's
+// accurate exponential and IEEE division would make the kernel issue-bound. Under programmatic dependent launch a block
+// prefetches its first row into L2 before waiting for the previous kernel,
+// as the norm kernels do.
 #include <cstdint>
 
 #include "rn_device.cuh"
@@ -26,14 +29,53 @@
 namespace rn {
 namespace {
 
-// silu(g) * u for a pair, in fp32: fast exponential and fast division
-// intrinsics (documented errors: 2 + 1.173|g| ulp and 2 ulp), one rounding for
-// the up product. For g < -87.3 the divisor exceeds 2^126 and the fast
-// division returns 0: silu(g) is then below 1e-36 in magnitude.
+// log2(e) split into a float and the float nearest to the remainder
+// (Cody and Waite's argument reduction, "Software Manual for the Elementary
+// Functions", 1980), and ln(2).
+constexpr float kLog2eHi = 1.44269502162933349609375f;
+constexpr float kLog2eLo = 1.925963033500e-8f;
+constexpr float kLn2 = 0.693147180559945309f;
+
+// 2^x for an fp32 x on the multi-function unit (ex2.approx: the integer
+// part of x is exact, the relative error is a few ulp whatever |x|).
+__device__ __forceinline__ float exp2_mufu(float x) {
+    float y;
+    asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+    return y;
+}
+
+// 1 / d on the multi-function unit (rcp.approx: within an ulp; with .ftz a
+// divisor past 2^126 gives 0, and +inf gives 0).
+__device__ __forceinline__ float rcp_mufu(float d) {
+    float r;
+    asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(d));
+    return r;
+}
+
+// silu(g) * u for a pair, in fp32, with packed two-lane arithmetic:
+//   silu(g) = g * 1 / (1 + e^-g),  e^-g = 2^p,  p = -g log2(e).
+// Forming p as one float would round it by up to half an ulp of |g| * 1.44,
+// an error e^-g inherits multiplied by |g| * 1.44 (tens of ulp at |g| = 20).
+// Here p = p_hi + p_lo to about 2^-40 relative: p_lo is the exact rounding
+// error of -g * kLog2eHi (an fma) plus -g * kLog2eLo, and
+// 2^p = 2^p_hi * (1 + p_lo ln 2) to within (p_lo ln 2)^2 < 2^-32. With the
+// base-2 exponential and the reciprocal of the multi-function unit and four
+// more roundings, y is within a few ulp of its exact value for any finite
+// gate, so the row maximum, hence the per-token scale, is within 1e-6. An
+// exponent past 128 gives e^-g = +inf and silu = 0; for g < -87.3 the
+// divisor exceeds 2^126 and silu (then below 1e-36 in magnitude) is 0 too.
 __device__ __forceinline__ float2 swiglu2(float2 g, float2 u) {
-    const float sx = __fdividef(g.x, 1.0f + __expf(-g.x));
-    const float sy = __fdividef(g.y, 1.0f + __expf(-g.y));
-    return __fmul2_rn(make_float2(sx, sy), u);
+    const float2 ng = make_float2(-g.x, -g.y);
+    const float2 lhi = make_float2(kLog2eHi, kLog2eHi);
+    const float2 one = make_float2(1.0f, 1.0f);
+    const float2 p_hi = __fmul2_rn(ng, lhi);
+    float2 p_lo = __ffma2_rn(ng, lhi, make_float2(-p_hi.x, -p_hi.y));
+    p_lo = __ffma2_rn(ng, make_float2(kLog2eLo, kLog2eLo), p_lo);
+    const float2 e_hi = make_float2(exp2_mufu(p_hi.x), exp2_mufu(p_hi.y));
+    const float2 e = __fmul2_rn(e_hi, __ffma2_rn(p_lo, make_float2(kLn2, kLn2), one));
+    const float2 d = __fadd2_rn(e, one);
+    const float2 silu = __fmul2_rn(g, make_float2(rcp_mufu(d.x), rcp_mufu(d.y)));
+    return __fmul2_rn(silu, u);
 }
 
 // Index (in 16-byte vectors) of a thread's vector k: strided by tpr, or with
@@ -44,14 +86,32 @@ __device__ __forceinline__ int swiglu_vec_index(int lr, int k, int tpr) {
     return lr + k * tpr;
 }
 
+// L2 prefetch of the block's first rows ([gate | up], 4I bytes each) in 4 KB
+// pieces spread over the row group's threads. Rows are 16-byte aligned and
+// 4I is a multiple of 16 on the vector path.
+__device__ __forceinline__ void swiglu_prefetch_first_rows(const SwigluArgs& a, const int tpr,
+                                                           const int rpc) {
+    constexpr uint32_t kChunk = 4096;
+    const int row_in_cta = threadIdx.x / tpr;
+    const int lr = threadIdx.x - row_in_cta * tpr;
+    const int64_t row = static_cast<int64_t>(blockIdx.x) * rpc + row_in_cta;
+    if (row >= a.T) return;
+    const uint32_t row_bytes = static_cast<uint32_t>(a.I) * 4u;
+    const char* xr = static_cast<const char*>(a.x) + row * row_bytes;
+    for (uint32_t off = static_cast<uint32_t>(lr) * kChunk; off < row_bytes;
+         off += static_cast<uint32_t>(tpr) * kChunk)
+        prefetch_l2(xr + off, row_bytes - off < kChunk ? row_bytes - off : kChunk);
+}
+
 template <typename T, int VPT, bool kPair>
 __global__ void __launch_bounds__(max_block_for_vpt(VPT))
-    rn_swiglu_fp8_kernel(const SwigluArgs a, const int tpr, const int rpc) {
+    rn_swiglu_fp8_kernel(const SwigluArgs a, const int tpr, const int rpc, const int prefetch) {
     static_assert(!kPair || VPT % 2 == 0, "pairs need an even vector count");
     constexpr int kStep = kPair ? 2 : 1;
     using F = Fmt<T>;
     extern __shared__ float red[];  // [2][rpc][warps per row]
     pdl_allow_dependents();
+    if (prefetch) swiglu_prefetch_first_rows(a, tpr, rpc);
     pdl_wait_for_prior_grid();
 
     const int row_in_cta = threadIdx.x / tpr;
@@ -181,13 +241,14 @@ template <typename T, int I = 0>
 cudaError_t swiglu_dispatch_vpt(const SwigluArgs& a, const Launch& l, cudaStream_t s) {
     if constexpr (I < kNumVpt) {
         if (l.vpt == kVptList[I]) {
+            const int pf = l.pdl && l.prefetch ? 1 : 0;
             if constexpr (kVptList[I] % 2 == 0) {
                 if (l.pair)
                     return launch_kernel(rn_swiglu_fp8_kernel<T, kVptList[I], true>, l, s, a,
-                                         l.tpr, l.rpc);
+                                         l.tpr, l.rpc, pf);
             }
             return launch_kernel(rn_swiglu_fp8_kernel<T, kVptList[I], false>, l, s, a, l.tpr,
-                                 l.rpc);
+                                 l.rpc, pf);
         }
         return swiglu_dispatch_vpt<T, I + 1>(a, l, s);
     } else {

@@ -273,25 +273,49 @@ def test_planner_invariants(op):
                 assert tpr % 32 == 0 and rpc <= 15
             else:
                 assert 32 % tpr == 0
-            # grid: one block per rpc rows, capped at 16 blocks per SM (148 SMs)
-            assert p["grid"] == min(-(-T // rpc), 16 * 148)
+            # grid: one block per rpc rows, capped at 16 blocks per SM (148
+            # SMs) except for the fused ops on 8192 rows or more
+            blocks = -(-T // rpc)
+            uncapped = op != "rms_norm" and T >= 8192
+            assert p["grid"] == (blocks if uncapped else min(blocks, 16 * 148))
             assert vpt in rn.supported_vectors_per_thread()
     # the scalar kernel beyond the vector kernel's reach
     assert rn.plan_launch(op, BF, 4, 1 << 17)["kernel"] == 1
 
 
 def test_planner_measured_choices():
-    """The launch shapes the forced-shape sweeps on B200 chose: four vectors
-    per thread at H = 3840 (they move as two 32-byte pairs), blocks of about
-    256 threads for rms_norm and 256/512 for the fused ops."""
+    """The launch shapes the forced-shape grids on B200 chose: four vectors
+    per thread at H = 3840 (they move as two 32-byte pairs); blocks of about
+    256 threads for rms_norm, about 512 for fused_add_rms_norm, about 256
+    then 512 (from 16384 rows) for the fp8 op, which takes eight vectors per
+    thread on wide rows below 8192 rows; no grid cap for the fused ops from
+    8192 rows on."""
     def shape(op, T, H):
         p = rn.plan_launch(op, BF, T, H)
         return p["threads_per_row"], p["vectors_per_thread"], p["rows_per_cta"]
-    for op in ("fused_add_rms_norm", "fused_add_rms_norm_fp8"):
-        assert shape(op, 8192, 3840) == (128, 4, 2)
+    fused, fp8 = "fused_add_rms_norm", "fused_add_rms_norm_fp8"
+    assert shape(fused, 8192, 3840) == (128, 4, 4)
+    assert shape(fused, 4096, 2048) == (64, 4, 8)
+    assert shape(fused, 4096, 5120) == (160, 4, 3)
+    assert shape(fused, 32768, 8192) == (256, 4, 2)
+    assert shape(fp8, 8192, 3840) == (128, 4, 2)
+    assert shape(fp8, 16384, 3840) == (128, 4, 4)
+    assert shape(fp8, 4096, 3840) == (128, 4, 2)
+    assert shape(fp8, 4096, 5120) == (160, 4, 2)
+    assert shape(fp8, 4096, 7168) == (128, 8, 1)
+    assert shape(fp8, 8192, 7168) == (224, 4, 2)
+    assert shape(fp8, 32768, 5120) == (160, 4, 3)
+    assert rn.plan_launch(fp8, BF, 8192, 3840)["grid"] == 4096  # uncapped
+    for op in (fused, fp8):
         assert shape(op, 32768, 4096) == (128, 4, 4)
-        assert shape(op, 32768, 8192) == (256, 4, 2)
-        assert shape(op, 4096, 5120) == (160, 4, 2)
+        assert rn.plan_launch(op, BF, 65536, 4096)["grid"] == 65536 // 4
+        assert rn.plan_launch(op, BF, 4096, 4096)["grid"] <= 16 * 148
+    assert rn.plan_launch("rms_norm", BF, 65536, 4096)["grid"] == 16 * 148
+    # rows that would take 512 threads at four vectors: eight, one row per block
+    for T in (4096, 65536):
+        assert shape("rms_norm", T, 16384) == (256, 8, 1)
+        assert shape(fp8, T, 16384) == (256, 8, 1)
+        assert shape(fused, T, 16384) == (512, 4, 1)
     assert shape("rms_norm", 8192, 3840) == (128, 4, 2)
     assert shape("rms_norm", 32768, 4096) == (128, 4, 2)
     assert shape("rms_norm", 32768, 2048) == (64, 4, 4)

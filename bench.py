@@ -9,9 +9,12 @@ weight = 1 + N(0,0.1), eps 1e-6) through
 Metric: algorithmic HBM GB/s of the step (bytes every element must move,
 weight counted once per launch), its fraction of the HBM roofline, and rows/s.
 
-Timing: W untimed warm-up steps, then K steps bracketed by a barrier and a
-device synchronize, timed with CUDA events on the launching stream; per-kernel
-durations from event pairs around each launch. L2: launches rotate over
+Timing: W untimed warm-up steps, then R (default 30) timed passes of exactly
+K steps, each bracketed by a barrier and a device synchronize and timed with
+CUDA events on the launching stream; the line reports the median pass with
+the fastest and slowest, and an NVML clock sample taken during each pass.
+Per-kernel durations: each op alone, K launches back to back between one
+event pair, median over R such passes. L2: launches rotate over
 buffer sets totalling >= 4x the L2 size, so no launch reads data the previous
 launches left in L2. Under torchrun each rank runs an independent replica
 (no collective on the data path; the path has no exchange step) and rank 0
@@ -158,6 +161,19 @@ class ClockSampler:
                 return
             self._stop.wait(self.period)
 
+    def sample_now(self):
+        """One SM clock reading now (MHz), also kept with the polled samples."""
+        if self.nv is None:
+            return None
+        try:
+            mhz = self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM)
+            bits = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+        except Exception as e:
+            self.err = f"{type(e).__name__}: {e}"
+            return None
+        self.samples.append((mhz, bits))
+        return mhz
+
     def start(self):
         import threading
         if self.nv is None:
@@ -279,7 +295,8 @@ def run_reference(args, world, rank):
         total += dt
     nbytes = step_bytes(rows, H_PREFILL) * args.steps
     value = nbytes / total / 1e9
-    sample = (f"{rows} of {T_PREFILL} rows of the prefill batch per step, both ops, fp64 C oracle "
+    what = "all" if rows == T_PREFILL else f"{rows} of"
+    sample = (f"{what} {T_PREFILL} rows of the prefill batch per step, both ops, fp64 C oracle "
               f"on {cores} host threads")
     line = {
         "impl": "reference", "metric": METRIC, "value": round(value, 4), "unit": "GB/s",
@@ -287,7 +304,8 @@ def run_reference(args, world, rank):
         "ms_per_step": round(total / args.steps * 1e3, 3), "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "rows_per_s": round(rows * args.steps / total, 2),
-        "config": dict(step_config(wl.eps), sample_rows_per_step=rows),
+        "config": step_config(wl.eps) if rows == T_PREFILL else
+        dict(step_config(wl.eps), sample_rows_per_step=rows),
         "cpu_baseline": {"value": round(value, 4), "unit": "GB/s", "cores": cores,
                          "kind": "oracle", "sample": sample},
         "e2e": {"value": round(value, 4), "unit": "GB/s", "h2d_bytes_per_step": 0,
@@ -349,21 +367,31 @@ def run_ours(args, world, rank, local):
     torch.cuda.synchronize(device)
 
     K = args.steps
-    # Pass A (the headline): K steps, events only at the two ends.
+    R = max(1, args.repeats)
+    # Pass A (the headline): R timed passes of exactly K steps each, each
+    # bracketed by a barrier and a device synchronize, events only at the two
+    # ends of a pass, one NVML clock sample taken while the pass runs (after
+    # its launches are queued, before the synchronize) besides the background
+    # poller. The line reports the median pass (max over ranks per pass).
     clocks = ClockSampler(device)
     e_start, e_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    barrier(world)
-    torch.cuda.synchronize(device)
+    pass_ms, pass_mhz = [], []
     clocks.start()
-    e_start.record(stream)
-    for i in range(K):
-        launch(i, 0)
-        launch(i, 1)
-    e_end.record(stream)
-    torch.cuda.synchronize(device)
+    for rep in range(R):
+        barrier(world)
+        torch.cuda.synchronize(device)
+        e_start.record(stream)
+        for i in range(K):
+            launch(i, 0)
+            launch(i, 1)
+        e_end.record(stream)
+        pass_mhz.append(clocks.sample_now())
+        torch.cuda.synchronize(device)
+        barrier(world)
+        pass_ms.append(max_over_ranks(e_start.elapsed_time(e_end), world, device))
     clk = clocks.stop()
-    barrier(world)
-    total_ms = max_over_ranks(e_start.elapsed_time(e_end), world, device)
+    clk["per_pass_sm_mhz"] = pass_mhz
+    total_ms = statistics.median(pass_ms)
 
     # Pass B: each op alone, K launches back to back on the step's rotating
     # buffer sets, one event pair around the K launches: that kernel's
@@ -374,15 +402,18 @@ def run_ours(args, world, rank, local):
     per_op_ms = []
     for k in (0, 1):
         ea, eb = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        barrier(world)
-        torch.cuda.synchronize(device)
-        ea.record(stream)
-        for i in range(K):
-            launch(i, k)
-        eb.record(stream)
-        torch.cuda.synchronize(device)
-        barrier(world)
-        per_op_ms.append(max_over_ranks(ea.elapsed_time(eb), world, device) / K)
+        reps = []
+        for rep in range(R):
+            barrier(world)
+            torch.cuda.synchronize(device)
+            ea.record(stream)
+            for i in range(K):
+                launch(i, k)
+            eb.record(stream)
+            torch.cuda.synchronize(device)
+            barrier(world)
+            reps.append(max_over_ranks(ea.elapsed_time(eb), world, device) / K)
+        per_op_ms.append(statistics.median(reps))
 
     # end to end through the public API with host buffers: pinned H2D of each
     # launch's inputs, the two launches, D2H of every output, all timed.
@@ -403,6 +434,13 @@ def run_ours(args, world, rank, local):
     line = {
         "metric": METRIC, "value": round(value, 2), "unit": "GB/s", "n_gpus": world,
         "steps": K, "warmup": args.warmup, "ms_per_step": round(total_ms / K, 5),
+        "repeats": {"passes": R, "steps_per_pass": K,
+                    "ms_per_step_median": round(total_ms / K, 5),
+                    "ms_per_step_min": round(min(pass_ms) / K, 5),
+                    "ms_per_step_max": round(max(pass_ms) / K, 5),
+                    "value_min": round(b_step * K * world / (max(pass_ms) / 1e3) / 1e9, 2),
+                    "value_max": round(b_step * K * world / (min(pass_ms) / 1e3) / 1e9, 2),
+                    "how": "value and ms_per_step are the median of the passes"},
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic",
         "rows_per_s": round(T * K * world / (total_ms / 1e3), 1),
@@ -413,7 +451,8 @@ def run_ours(args, world, rank, local):
             l2=f"rotating {n_sets} buffer sets ({n_sets * set_bytes(T, H) / 1e6:.0f} MB, "
                f">= 4x L2 of {l2 / 1e6:.0f} MB); no L2 flush",
             plans={op: rn.plan_launch(op, torch.bfloat16, T, H) for op in STEP_OPS}),
-        "per_kernel_how": f"each op alone, {K} launches back to back, events at the ends",
+        "per_kernel_how": f"each op alone, {K} launches back to back, events at the ends; "
+                          f"median of {R} such passes",
         "per_kernel_ms": {"fused_add_rms_norm": round(dom_ms, 5),
                           "fused_add_rms_norm_fp8": round(fp8_ms, 5)},
         "per_kernel_gbs": {"fused_add_rms_norm": round(achieved, 1),
@@ -427,7 +466,9 @@ def run_ours(args, world, rank, local):
                      "traffic": traffic},
         "cpu_baseline": cpu,
         "e2e": e2e,
-        "gpu_launches": 2 * K,
+        "gpu_launches": 2 * K * R,
+        "gpu_launches_how": "launches inside the R timed step passes (the per-kernel "
+                            "passes and the e2e pass launch more)",
         "clocks": clk,
     }
     print(json.dumps(line), flush=True)
@@ -896,8 +937,10 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="skip the oracle timing (for profiler runs)")
-    ap.add_argument("--reference-rows", type=int, default=1024,
-                    help="rows of the prefill batch per reference (oracle) step")
+    ap.add_argument("--reference-rows", type=int, default=T_PREFILL,
+                    help="rows of the prefill batch per reference (oracle) step (default: all)")
+    ap.add_argument("--repeats", type=int, default=30,
+                    help="timed passes of K steps each; the line reports their median")
     ap.add_argument("--sweep-out", default=None,
                     help="instead of the step benchmark, time every workload cell and write "
                          "one JSON line per cell to this file")

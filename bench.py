@@ -545,6 +545,10 @@ def run_e2e(args, rn, wl, S, device, stream, world=1):
 
 # ----------------------------------------------------------------------------- sweep
 
+# Row counts of the --sweep-scan series (inputs of the "sweep" workload).
+SCAN_T = (256, 512, 1024, 2048, 4096, 8192, 16384, 32768, 65536)
+
+
 def sweep_cells():
     """Every (workload, op, dtype, T, H) cell of the named workloads."""
     cells = [("small", "rms_norm", "bf16", 8, 512)]
@@ -566,9 +570,10 @@ def sweep_cells():
 
 
 def time_cell(rn, name, op, dtype, T, H, iters, device, mem_cap_bytes=24 << 30):
-    """Median-free mean time per launch over `iters` launches that rotate
-    over buffer sets totalling >= 4x L2 (capped by memory), eager stream
-    launches; plus CUDA-graph replay time for launches under 30 us."""
+    """Mean time per launch over `iters` eager stream launches that rotate
+    over buffer sets totalling >= 4x L2 (capped by memory), and the device
+    time per launch under CUDA-graph replay (about 4 ms of launches per
+    graph, median of 5 replays), which excludes the host's per-call cost."""
     wl = synth.make_inputs(name, op, dtype, T, H, device=device)
     dt = wl.dtype
     l2 = torch.cuda.get_device_properties(device).L2_cache_size
@@ -604,6 +609,8 @@ def time_cell(rn, name, op, dtype, T, H, iters, device, mem_cap_bytes=24 << 30):
     for i in range(5):
         launch(i)
     torch.cuda.synchronize(device)
+    clocks = ClockSampler(device, period_s=0.002)
+    clocks.start()
     e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     e0.record()
     for i in range(iters):
@@ -611,27 +618,29 @@ def time_cell(rn, name, op, dtype, T, H, iters, device, mem_cap_bytes=24 << 30):
     e1.record()
     torch.cuda.synchronize(device)
     us = e0.elapsed_time(e1) / iters * 1e3
-    graph_us = None
-    if us < 30:
-        g = torch.cuda.CUDAGraph()
-        st = torch.cuda.Stream(device)
-        with torch.cuda.stream(st):
-            launch(0)
-            torch.cuda.synchronize(device)
-            with torch.cuda.graph(g, stream=st):
-                for i in range(100):
-                    launch(i)
+    nl = max(10, min(100, int(4000 / max(us, 1.0))))
+    g = torch.cuda.CUDAGraph()
+    st = torch.cuda.Stream(device)
+    with torch.cuda.stream(st):
+        launch(0)
         torch.cuda.synchronize(device)
-        g.replay()
-        torch.cuda.synchronize(device)
+        with torch.cuda.graph(g, stream=st):
+            for i in range(nl):
+                launch(i)
+    torch.cuda.synchronize(device)
+    g.replay()
+    torch.cuda.synchronize(device)
+    reps = []
+    for _ in range(5):
         e0.record()
-        for _ in range(5):
-            g.replay()
+        g.replay()
         e1.record()
         torch.cuda.synchronize(device)
-        graph_us = e0.elapsed_time(e1) / 500 * 1e3
-        del g
-    plan = rn.plan_launch(op, dt, T, H)
+        reps.append(e0.elapsed_time(e1) / nl * 1e3)
+    graph_us = statistics.median(reps)
+    del g
+    clk = clocks.stop()
+    plan = dict(rn.plan_launch(op, dt, T, H), sm_mhz=clk["sm_mhz"], clock_reasons=clk["reasons"])
     del sets
     torch.cuda.empty_cache()
     return us, graph_us, plan, n
@@ -867,9 +876,29 @@ def run_sweep(args, world, rank, local):
                "frac_of_measured": round(nbytes / best / 1e3 / peak, 4),
                "bytes": nbytes, "buffer_sets": nsets,
                "kernel": {0: "vector", 1: "scalar", 2: "staged"}[plan["kernel"]],
-               "tpr": plan["threads_per_row"], "vpt": plan["vectors_per_thread"]}
+               "tpr": plan["threads_per_row"], "vpt": plan["vectors_per_thread"],
+               "rpc": plan["rows_per_cta"], "grid": plan["grid"],
+               "sm_mhz": plan["sm_mhz"], "clock_reasons": plan["clock_reasons"]}
         out.write(json.dumps(rec) + "\n")
         out.flush()
+    if args.sweep_scan:
+        # the fused ops over a range of row counts at fixed widths: time per
+        # launch against bytes separates the per-launch fixed cost from the
+        # streaming rate
+        for H in (2048, 4096):
+            for op in ("fused_add_rms_norm", "fused_add_rms_norm_fp8"):
+                for T in SCAN_T:
+                    us, gus, plan, nsets = time_cell(rn, "sweep", op, "bf16", T, H,
+                                                     args.sweep_iters, device)
+                    nbytes = op_bytes(op, T, H)
+                    out.write(json.dumps({
+                        "workload": "scan", "op": op, "dtype": "bf16", "T": T, "H": H,
+                        "us": round(us, 3), "graph_us": round(gus, 3), "bytes": nbytes,
+                        "graph_gbs": round(nbytes / gus / 1e3, 1),
+                        "tpr": plan["threads_per_row"], "vpt": plan["vectors_per_thread"],
+                        "rpc": plan["rows_per_cta"], "grid": plan["grid"],
+                        "sm_mhz": plan["sm_mhz"], "clock_reasons": plan["clock_reasons"]}) + "\n")
+                    out.flush()
     tp_cells = [(fp8, W, T, H, algo) for fp8 in (False, True) for W in synth.TP_W
                 for T in synth.TP_T for H in (3840,)
                 for algo in (("one_shot", "two_shot") if W >= 3 else ("one_shot",))
@@ -945,6 +974,8 @@ def main():
                     help="instead of the step benchmark, time every workload cell and write "
                          "one JSON line per cell to this file")
     ap.add_argument("--sweep-iters", type=int, default=50)
+    ap.add_argument("--sweep-scan", action="store_true",
+                    help="also time the fused ops at H = 2048 and 4096 over T = 256 ... 65536")
     ap.add_argument("--sweep-gemm-configs", action="store_true",
                     help="also time every GEMM tile configuration, forced, on every GEMM cell")
     ap.add_argument("--sweep-filter", default=None,

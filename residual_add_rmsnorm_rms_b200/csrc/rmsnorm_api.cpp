@@ -267,7 +267,7 @@ long long default_grid_cap(int op, int64_t T, int num_sms) {
     return static_cast<long long>(kVectorBlocksPerSmCap) * num_sms;
 }
 
-bool auto_vector_plan(int op, int64_t T, int64_t H, int num_sms, rn_plan* p) {
+bool auto_vector_plan(int op, int dt, int64_t T, int64_t H, int num_sms, rn_plan* p) {
     const int64_t nvec = H / 8;
     auto idle_of = [&](int tpr, int vpt) {
         const int64_t slots = static_cast<int64_t>(tpr) * vpt;
@@ -279,14 +279,18 @@ bool auto_vector_plan(int op, int64_t T, int64_t H, int num_sms, rn_plan* p) {
     if (many_rows) {
         // Eight vectors per thread, one row per block of 128-256 threads:
         // half the warps per row of the four-vector plan, so half the
-        // cross-warp reduction. Taken by rms_norm and the fp8 op on rows
-        // that would need 512 threads at four vectors (H = 16384: 2-5 %
-        // faster at T = 4096-65536), and by the fp8 op below kFusedManyRows
-        // rows on rows of 128 or more threads at eight vectors (T = 4096:
-        // H = 7168 4.4 % faster, 8192 2 %; from T = 8192 on, 5-10 % slower).
+        // cross-warp reduction. Taken by rms_norm on rows that would need 512
+        // threads at four vectors (H = 16384: 2-5 % faster at T =
+        // 4096-65536, both formats), and by the bf16 fp8 op on such rows and,
+        // below kFusedManyRows rows, on rows of 128 or more threads at eight
+        // vectors (T = 4096: H = 7168 4.4 % faster, 8192 2 %; from T = 8192
+        // on, 5-10 % slower). The fp16 fp8 op, whose fp16 -> fp32 widening
+        // costs more issue slots than bf16's shifts, keeps four vectors (4-7 %
+        // faster at T = 4096, H = 7168-16384).
         const int tpr8 = tpr_for(nvec, 8);
-        const bool wide = tpr4 >= 512 && (op == rn::kRmsNorm || op == rn::kFusedAddFp8);
-        const bool fp8_few = op == rn::kFusedAddFp8 && T < kFusedManyRows && tpr8 >= 128;
+        const bool fp8_bf16 = op == rn::kFusedAddFp8 && dt == rn::kBF16;
+        const bool wide = tpr4 >= 512 && (op == rn::kRmsNorm || fp8_bf16);
+        const bool fp8_few = fp8_bf16 && T < kFusedManyRows && tpr8 >= 128;
         if ((wide || fp8_few) && tpr8 <= rn::max_block_for_vpt(8) && idle_of(tpr8, 8) <= 1.0 / 8) {
             fill_vector_plan(tpr8, 8, T, p, 1);
             return true;
@@ -326,15 +330,15 @@ bool auto_vector_plan(int op, int64_t T, int64_t H, int num_sms, rn_plan* p) {
     return false;
 }
 
-rn_status plan_shape(int op, int64_t T, int64_t H, bool vector_ok, int num_sms, rn_plan* p,
-                     bool allow_staged);
+rn_status plan_shape(int op, int dt, int64_t T, int64_t H, bool vector_ok, int num_sms,
+                     rn_plan* p, bool allow_staged);
 
 // The launch plan: the kernel and its shape, then the grid cap (the kernels
 // stride over the rows a capped grid does not cover). `allow_staged` is false
 // for kernels that have no staged form.
-rn_status plan_impl(int op, int64_t T, int64_t H, bool vector_ok, int num_sms, rn_plan* p,
+rn_status plan_impl(int op, int dt, int64_t T, int64_t H, bool vector_ok, int num_sms, rn_plan* p,
                     bool allow_staged = true) {
-    const rn_status st = plan_shape(op, T, H, vector_ok, num_sms, p, allow_staged);
+    const rn_status st = plan_shape(op, dt, T, H, vector_ok, num_sms, p, allow_staged);
     if (st != RN_OK) return st;
     long long cap = g_max_grid.load();
     if (cap == 0 && p->kernel == RN_KERNEL_VECTOR) cap = default_grid_cap(op, T, num_sms);
@@ -343,8 +347,8 @@ rn_status plan_impl(int op, int64_t T, int64_t H, bool vector_ok, int num_sms, r
     return RN_OK;
 }
 
-rn_status plan_shape(int op, int64_t T, int64_t H, bool vector_ok, int num_sms, rn_plan* p,
-                     bool allow_staged) {
+rn_status plan_shape(int op, int dt, int64_t T, int64_t H, bool vector_ok, int num_sms,
+                     rn_plan* p, bool allow_staged) {
     if (H < 1 || T < 0) return RN_ERR_SHAPE;
     std::memset(p, 0, sizeof *p);
     if (!vector_ok || H % 8 != 0) {
@@ -368,7 +372,7 @@ rn_status plan_shape(int op, int64_t T, int64_t H, bool vector_ok, int num_sms, 
     }
     // The STAGED kernel is chosen only when forced: measured on B200 it trails
     // the VECTOR kernel at every shape tried (T up to 65536, H 2048..16384).
-    if (!auto_vector_plan(op, T, H, num_sms, p)) fill_scalar_plan(T, p);
+    if (!auto_vector_plan(op, dt, T, H, num_sms, p)) fill_scalar_plan(T, p);
     return RN_OK;
 }
 
@@ -523,7 +527,7 @@ rn_status check_pointers_and_plan(int op, const Common& c, int num_sms, rn_plan*
     if (op != rn::kFusedAddFp8) vector_ok = vector_ok && aligned(c.out.ptr, 16);
     if (op != rn::kRmsNorm) vector_ok = vector_ok && aligned(c.res.ptr, 16);
     if (op == rn::kFusedAddFp8) vector_ok = vector_ok && aligned(c.q.ptr, 8);
-    rn_status st = plan_impl(op, T, H, vector_ok, num_sms, plan);
+    rn_status st = plan_impl(op, c.dt, T, H, vector_ok, num_sms, plan);
     if (st != RN_OK) return st;
 
     return RN_OK;
@@ -649,7 +653,9 @@ rn_status rn_silu_and_mul_fp8(const rn_tensor* q, const rn_tensor* scale, const 
     // The row mapping of the fused norm ops on I-wide rows (rows per block as
     // for the fp8 op): per output element it moves 2 x 2 bytes in and 1 byte
     // out, within a few bytes of that op.
-    if ((st = plan_impl(rn::kSwigluFp8, fx.T, I, vector_ok, device_sms(), &plan, false)) != RN_OK)
+    const int sdt = x->dtype == RN_BF16 ? rn::kBF16 : rn::kF16;
+    if ((st = plan_impl(rn::kSwigluFp8, sdt, fx.T, I, vector_ok, device_sms(), &plan, false)) !=
+        RN_OK)
         return st;
     rn::SwigluArgs a{fx.ptr, reinterpret_cast<uint8_t*>(fq.ptr), reinterpret_cast<float*>(fs.ptr),
                      fx.T, I};
@@ -1060,7 +1066,7 @@ rn_status run_host(int op, const rn_tensor* o, const rn_tensor* sc, const rn_ten
         a.H = H;
         a.eps = eps;
         rn_plan plan;
-        st = plan_impl(op, rows, H, vector_ok, num_sms, &plan);
+        st = plan_impl(op, c.dt, rows, H, vector_ok, num_sms, &plan);
         if (st != RN_OK) return st;
         // no programmatic dependent launch: the kernel follows copies
         st = launch_plan(op, c.dt, a, plan, false, pair_ok(op, H, a.x, a.residual, a.out, a.q),
@@ -1210,9 +1216,10 @@ rn_status rn_plan_launch(int32_t op, int32_t dtype, int64_t T, int64_t H, int32_
     if (!plan) return RN_ERR_NULL;
     if (op < 0 || op > 3) return RN_ERR_CONFIG;
     if (!is16(dtype)) return RN_ERR_DTYPE;
+    const int dt = dtype == RN_BF16 ? rn::kBF16 : rn::kF16;
     if (op == RN_OP_SILU_AND_MUL_FP8)
-        return plan_impl(rn::kSwigluFp8, T, H, vector_ok != 0, kDefaultSms, plan, false);
-    return plan_impl(op, T, H, vector_ok != 0, kDefaultSms, plan);
+        return plan_impl(rn::kSwigluFp8, dt, T, H, vector_ok != 0, kDefaultSms, plan, false);
+    return plan_impl(op, dt, T, H, vector_ok != 0, kDefaultSms, plan);
 }
 
 rn_status rn_force_staged(int32_t ctas_per_sm, int32_t stages, int32_t threads) {

@@ -316,6 +316,15 @@ def test_planner_measured_choices():
         assert shape("rms_norm", T, 16384) == (256, 8, 1)
         assert shape(fp8, T, 16384) == (256, 8, 1)
         assert shape(fused, T, 16384) == (512, 4, 1)
+    # fp16: the fp8 op keeps four vectors per thread (its widening costs more)
+    def shape16(op, T, H):
+        p = rn.plan_launch(op, F16, T, H)
+        return p["threads_per_row"], p["vectors_per_thread"], p["rows_per_cta"]
+    assert shape16(fp8, 4096, 7168) == (224, 4, 2)
+    assert shape16(fp8, 4096, 16384) == (512, 4, 1)
+    assert shape16(fp8, 65536, 16384) == (512, 4, 1)
+    assert shape16("rms_norm", 4096, 16384) == (256, 8, 1)
+    assert shape16(fused, 8192, 3840) == shape(fused, 8192, 3840)
     assert shape("rms_norm", 8192, 3840) == (128, 4, 2)
     assert shape("rms_norm", 32768, 4096) == (128, 4, 2)
     assert shape("rms_norm", 32768, 2048) == (64, 4, 4)

@@ -477,12 +477,14 @@ __global__ void __launch_bounds__(kArMaxBlock)
         allreduce_rows<T, VPT, kW, kFp8, false, kTwoShot>(a, tpr, rpc, red);
 }
 
-// Groups of four or eight ranks: the same kernel held to 80 registers, so
-// three 256-thread blocks fit an SM instead of two (the rank-order reduction
-// otherwise keeps every rank's vectors live: ~125 registers). Measured on one
-// device, [8192 x 3840] bf16: 8 ranks two-shot 636 -> 557 us, one-shot 1672
-// -> 1320 us; 4 ranks two-shot 329 -> 297 us (a few spilled words). Two ranks
-// keep the 128-register bound (6 % slower at 80).
+// Groups of four or eight ranks on many rows: the same kernel held to 80
+// registers, so three 256-thread blocks fit an SM instead of two (the
+// rank-order reduction otherwise keeps every rank's vectors live: ~125
+// registers). Measured on one device, [8192 x 3840] bf16: 8 ranks two-shot
+// 636 -> 557 us, one-shot 1672 -> 1346 us; 4 ranks two-shot 329 -> 295 us.
+// Its few spilled words cost more than the occupancy gains on a handful of
+// rows (8 ranks, T = 64: 17.7 -> 22.0 us), and two ranks are 6 % slower at 80
+// at any size, so the host picks it only for kW >= 4 and many rows.
 template <typename T, int VPT, int kW, bool kFp8, bool kTwoShot>
 __global__ void __maxnreg__(80) rn_allreduce_wide_kernel(const ArArgs a, const int tpr,
                                                            const int rpc) {
@@ -496,20 +498,20 @@ __global__ void __maxnreg__(80) rn_allreduce_wide_kernel(const ArArgs a, const i
 using ArKernel = void (*)(const ArArgs, const int, const int);
 
 template <typename T, int VPT, int kW, bool kFp8, bool kTwoShot>
-ArKernel pick_kernel() {
-    if constexpr (kW >= 4)
-        return rn_allreduce_wide_kernel<T, VPT, kW, kFp8, kTwoShot>;
-    else
-        return rn_allreduce_kernel<T, VPT, kW, kFp8, kTwoShot>;
+ArKernel pick_kernel(bool wide) {
+    if constexpr (kW >= 4) {
+        if (wide) return rn_allreduce_wide_kernel<T, VPT, kW, kFp8, kTwoShot>;
+    }
+    return rn_allreduce_kernel<T, VPT, kW, kFp8, kTwoShot>;
 }
 
 template <typename T, int kW, bool kFp8, bool kTwoShot>
-ArKernel pick_vpt(int vpt) {
+ArKernel pick_vpt(int vpt, bool wide) {
     switch (vpt) {
-        case 1: return pick_kernel<T, 1, kW, kFp8, kTwoShot>();
-        case 2: return pick_kernel<T, 2, kW, kFp8, kTwoShot>();
-        case 4: return pick_kernel<T, 4, kW, kFp8, kTwoShot>();
-        case 8: return pick_kernel<T, 8, kW, kFp8, kTwoShot>();
+        case 1: return pick_kernel<T, 1, kW, kFp8, kTwoShot>(wide);
+        case 2: return pick_kernel<T, 2, kW, kFp8, kTwoShot>(wide);
+        case 4: return pick_kernel<T, 4, kW, kFp8, kTwoShot>(wide);
+        case 8: return pick_kernel<T, 8, kW, kFp8, kTwoShot>(wide);
         default: return nullptr;
     }
 }
@@ -517,26 +519,26 @@ ArKernel pick_vpt(int vpt) {
 // Two-shot kernels exist for groups of 3 to 8 ranks (it moves more data than
 // one-shot with two ranks).
 template <typename T, bool kFp8>
-ArKernel pick_w(int world, int vpt, bool two_shot) {
+ArKernel pick_w(int world, int vpt, bool two_shot, bool wide) {
     if (two_shot) {
         if (world < 3) return nullptr;
-        if (world <= 4) return pick_vpt<T, 4, kFp8, true>(vpt);
-        return pick_vpt<T, 8, kFp8, true>(vpt);
+        if (world <= 4) return pick_vpt<T, 4, kFp8, true>(vpt, wide);
+        return pick_vpt<T, 8, kFp8, true>(vpt, wide);
     }
-    if (world == 1) return pick_vpt<T, 1, kFp8, false>(vpt);
-    if (world == 2) return pick_vpt<T, 2, kFp8, false>(vpt);
-    if (world <= 4) return pick_vpt<T, 4, kFp8, false>(vpt);
-    return pick_vpt<T, 8, kFp8, false>(vpt);
+    if (world == 1) return pick_vpt<T, 1, kFp8, false>(vpt, wide);
+    if (world == 2) return pick_vpt<T, 2, kFp8, false>(vpt, wide);
+    if (world <= 4) return pick_vpt<T, 4, kFp8, false>(vpt, wide);
+    return pick_vpt<T, 8, kFp8, false>(vpt, wide);
 }
 
-ArKernel pick(int dtype, bool fp8, int world, int vpt, bool two_shot) {
+ArKernel pick(int dtype, bool fp8, int world, const ArLaunch& l) {
     if (world < 1 || world > kArMaxWorld) return nullptr;
     if (dtype == kBF16)
-        return fp8 ? pick_w<__nv_bfloat16, true>(world, vpt, two_shot)
-                   : pick_w<__nv_bfloat16, false>(world, vpt, two_shot);
+        return fp8 ? pick_w<__nv_bfloat16, true>(world, l.vpt, l.two_shot, l.wide)
+                   : pick_w<__nv_bfloat16, false>(world, l.vpt, l.two_shot, l.wide);
     if (dtype == kF16)
-        return fp8 ? pick_w<__half, true>(world, vpt, two_shot)
-                   : pick_w<__half, false>(world, vpt, two_shot);
+        return fp8 ? pick_w<__half, true>(world, l.vpt, l.two_shot, l.wide)
+                   : pick_w<__half, false>(world, l.vpt, l.two_shot, l.wide);
     return nullptr;
 }
 
@@ -544,7 +546,7 @@ ArKernel pick(int dtype, bool fp8, int world, int vpt, bool two_shot) {
 
 cudaError_t allreduce_blocks_per_sm(int dtype, bool fp8, int world, const ArLaunch& l,
                                     int* blocks) {
-    const ArKernel k = pick(dtype, fp8, world, l.vpt, l.two_shot);
+    const ArKernel k = pick(dtype, fp8, world, l);
     if (!k) return cudaErrorInvalidValue;
     return cudaOccupancyMaxActiveBlocksPerMultiprocessor(blocks, k, l.block,
                                                          static_cast<size_t>(l.smem));
@@ -552,7 +554,7 @@ cudaError_t allreduce_blocks_per_sm(int dtype, bool fp8, int world, const ArLaun
 
 cudaError_t launch_allreduce(int dtype, bool fp8, const ArArgs& a, const ArLaunch& l,
                              cudaStream_t s) {
-    const ArKernel k = pick(dtype, fp8, a.world, l.vpt, l.two_shot);
+    const ArKernel k = pick(dtype, fp8, a.world, l);
     if (!k) return cudaErrorInvalidValue;
     cudaLaunchConfig_t cfg = {};
     cfg.gridDim = dim3(static_cast<unsigned>(l.grid_x), static_cast<unsigned>(l.local_ranks));

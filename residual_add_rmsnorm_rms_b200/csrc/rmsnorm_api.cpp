@@ -781,6 +781,14 @@ rn_status ar_shape(int64_t H, rn::ArLaunch* l) {
 // at the cost of a second exchange barrier (a few microseconds). Two-shot is
 // taken from four ranks on, once it saves at least 2.3 MB of peer reads per
 // rank: about 3 us at the 770 GB/s a B200 peer copy reaches over NVLink.
+// Rows from which groups of three to eight ranks run the all-reduce kernel
+// held to 80 registers (allreduce_kernels.cu, rn_allreduce_wide_kernel), by
+// algorithm. Measured on one device (H = 3840, 4 and 8 ranks, both outputs):
+// one-shot gains 2-31 % from 256 rows on and loses up to 10 % at 64; two-shot
+// loses 2-12 % up to 512 rows, breaks even at 1024 and gains 7-15 % from 2048.
+constexpr int64_t kArWideRowsOneShot = 256;
+constexpr int64_t kArWideRowsTwoShot = 2048;
+
 bool ar_two_shot_pays(int W, int64_t T, int64_t H) {
     if (W < 4) return false;
     const double th = static_cast<double>(T) * static_cast<double>(H);
@@ -860,6 +868,7 @@ rn_status run_allreduce(bool fp8, const rn_tensor* o, const rn_tensor* sc, const
     a.H = H;
     a.eps = eps;
     l.local_ranks = L;
+    l.wide = comm->world >= 3 && T >= (l.two_shot ? kArWideRowsTwoShot : kArWideRowsOneShot);
     int per_sm = 0;
     cudaError_t e = rn::allreduce_blocks_per_sm(c.dt, fp8, comm->world, l, &per_sm);
     if (e == cudaSuccess) {

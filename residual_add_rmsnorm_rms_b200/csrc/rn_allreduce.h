@@ -42,6 +42,7 @@ struct ArLaunch {
     int grid_x;       // blocks per rank (the same on every rank)
     int local_ranks;  // gridDim.y
     bool two_shot;    // reduce-scatter of row slices + gather of finished rows
+    bool wide = false;  // groups of 4-8 ranks: the 80-register kernel (more blocks per SM)
 };
 
 // Resident blocks per SM of the all-reduce kernel for this shape.

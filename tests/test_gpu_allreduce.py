@@ -91,8 +91,10 @@ def _check(fp8, got, wl, dtype, rows=None):
     return stats
 
 
+# (4, 2048, 1024) and (8, 256, 3840) run the 80-register kernels of groups of
+# 4-8 ranks on many rows (two-shot from 2048 rows, one-shot from 256).
 CASES = [(1, 1, 512), (2, 7, 512), (2, 300, 3840), (4, 64, 4096), (8, 1, 3840),
-         (8, 256, 3840), (3, 33, 1032), (8, 5, 32768), (5, 129, 24)]
+         (8, 256, 3840), (3, 33, 1032), (8, 5, 32768), (5, 129, 24), (4, 2048, 1024)]
 
 
 @pytest.mark.parametrize("W,T,H", CASES)

@@ -41,6 +41,7 @@
 #include <cuda_fp16.h>
 
 #include <cstdint>
+#include <type_traits>
 #include <utility>
 
 #include "rn_device.cuh"
@@ -67,6 +68,12 @@ __device__ __forceinline__ void vector_rows(const Args& a, const int tpr, const 
     static_assert(!kPair || VPT % 2 == 0, "pairs need an even vector count");
     constexpr bool kFused = OP != kRmsNorm;
     constexpr bool kFp8 = OP == kFusedAddFp8;
+    // bf16 rms_norm widens nothing: squares and products straight from the
+    // 16-bit values with the mixed-precision fma (rn_vec8.cuh). fp16 keeps
+    // widening: with the mixed fma, rms_norm no longer reproduced the fused
+    // op's output bit for bit on fp16 rows (they hold subnormals; bf16 rows
+    // practically never do), so its exactness there is not established.
+    constexpr bool kMixed = OP == kRmsNorm && std::is_same_v<T, __nv_bfloat16>;
 
     const int row_in_cta = threadIdx.x / tpr;
     const int lr = threadIdx.x - row_in_cta * tpr;
@@ -132,7 +139,7 @@ __device__ __forceinline__ void vector_rows(const Args& a, const int tpr, const 
         float pm = 0.f;
 #pragma unroll
         for (int k = 0; k < VPT; ++k) {
-            acc = ssq8<T>(v[k], acc);
+            acc = ssq8<T, kMixed>(v[k], acc);
             if constexpr (kFp8) {
                 const int j = vec_index<kPair>(lr, k, tpr);
                 uint4 w = make_uint4(0, 0, 0, 0);
@@ -178,10 +185,10 @@ __device__ __forceinline__ void vector_rows(const Args& a, const int tpr, const 
                 if constexpr (kPair) {
                     uint4 w1 = make_uint4(0, 0, 0, 0);
                     if constexpr (kHasW) w1 = __ldg(wv + j + 1);
-                    st_v8(orow + j, scale8<T, kHasW>(v[k], w, inv2),
-                          scale8<T, kHasW>(v[k + 1], w1, inv2));
+                    st_v8(orow + j, scale8<T, kHasW, kMixed>(v[k], w, inv2),
+                          scale8<T, kHasW, kMixed>(v[k + 1], w1, inv2));
                 } else {
-                    st_v4(orow + j, scale8<T, kHasW>(v[k], w, inv2));
+                    st_v4(orow + j, scale8<T, kHasW, kMixed>(v[k], w, inv2));
                 }
             }
         } else {

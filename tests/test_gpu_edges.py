@@ -304,6 +304,40 @@ def test_fused_equals_rms_norm_of_written_back_residual_on_gpu():
         assert torch.equal(out.view(torch.int16), out2.view(torch.int16))
 
 
+def test_bf16_rms_norm_equals_fused_on_subnormals_and_extremes():
+    """bf16 rms_norm squares and weights its inputs with the mixed-precision
+    fma (16-bit operands, fp32 result); the fused op widens them first.
+    rms_norm of the written-back residual must equal the fused op's output
+    bit for bit, here on rows mixing normal values, bf16 subnormals and
+    values near 1e15 (squares stay inside fp32, the supported range), with and
+    without a weight. (With x = 0 the written-back residual is r itself
+    except that -0 becomes +0.)"""
+    g = torch.Generator().manual_seed(17)
+    T, H = 64, 4096
+    r = torch.randn(T, H, generator=g)
+    sub = torch.rand(T, H, generator=g) < 0.1
+    r[sub] = torch.randn(int(sub.sum()), generator=g) * 1e-39   # bf16 subnormals
+    big = torch.rand(T, H, generator=g) < 0.01
+    r[big] = torch.randn(int(big.sum()), generator=g) * 1e15
+    r[7] = torch.randn(H, generator=g) * 1e-39                   # a row of subnormals only
+    r = r.bfloat16()
+    assert ((r.abs() < 2 ** -126) & (r != 0)).sum() > 1000
+    w = synth.weight(H, torch.bfloat16, g, "cpu")
+    for weight in (w, None):
+        x = torch.zeros(T, H, dtype=torch.bfloat16, device="cuda")
+        rr = r.cuda().clone()
+        out = torch.empty_like(x)
+        rn.fused_add_rms_norm(out, x, rr, None if weight is None else weight.cuda(), 1e-30)
+        out2 = torch.empty_like(x)
+        rn.rms_norm(out2, rr, None if weight is None else weight.cuda(), 1e-30)
+        torch.cuda.synchronize()
+        assert torch.equal(out.view(torch.int16), out2.view(torch.int16))
+        want = oracle_run("fused_add_rms_norm", x.cpu(), r, weight, 1e-30, "bf16")
+        compare("fused_add_rms_norm", {"out": out, "residual": rr}, want, "bf16")
+        compare("rms_norm", {"out": out2},
+                oracle_run("rms_norm", rr.cpu(), None, weight, 1e-30, "bf16"), "bf16")
+
+
 def test_non_default_stream():
     wl = synth.make_inputs("decode", "fused_add_rms_norm", "bf16", 64, 4096)
     s = torch.cuda.Stream()

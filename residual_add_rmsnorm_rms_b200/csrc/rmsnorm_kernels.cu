@@ -68,12 +68,14 @@ __device__ __forceinline__ void vector_rows(const Args& a, const int tpr, const 
     static_assert(!kPair || VPT % 2 == 0, "pairs need an even vector count");
     constexpr bool kFused = OP != kRmsNorm;
     constexpr bool kFp8 = OP == kFusedAddFp8;
-    // bf16 rms_norm widens nothing: squares and products straight from the
-    // 16-bit values with the mixed-precision fma (rn_vec8.cuh). fp16 keeps
-    // widening: with the mixed fma, rms_norm no longer reproduced the fused
-    // op's output bit for bit on fp16 rows (they hold subnormals; bf16 rows
-    // practically never do), so its exactness there is not established.
-    constexpr bool kMixed = OP == kRmsNorm && std::is_same_v<T, __nv_bfloat16>;
+    // bf16 rms_norm at four or more vectors per thread widens nothing:
+    // squares and products straight from the 16-bit values with the
+    // mixed-precision fma (rn_vec8.cuh; 3-14 % faster on T >= 4096). fp16
+    // keeps widening: with the mixed fma, rms_norm no longer reproduced the
+    // fused op's output bit for bit on fp16 rows, so its exactness there is
+    // not established. The one- and two-vector shapes of decode-sized rows
+    // keep widening too (two vectors per thread: up to 27 % slower with it).
+    constexpr bool kMixed = OP == kRmsNorm && std::is_same_v<T, __nv_bfloat16> && VPT >= 4;
 
     const int row_in_cta = threadIdx.x / tpr;
     const int lr = threadIdx.x - row_in_cta * tpr;

@@ -285,6 +285,15 @@ def run_reference(args, world, rank):
     import oracle
     cores = oracle.usable_cores()
     rows = args.reference_rows
+    if rows <= 0:
+        # time a probe of 256 rows, then take the whole batch if all steps fit
+        # the budget, else the largest sample that does (whole multiples of 64)
+        probe = synth.make_inputs("prefill", "fused_add_rms_norm", "bf16", 256, H_PREFILL)
+        dt, _, _ = oracle_step_sample(256, cores, (probe.x, probe.residual, probe.weight,
+                                                   probe.eps))
+        per_row = dt / 256
+        fit = int(args.reference_budget_s / (max(1, args.steps + args.warmup) * per_row))
+        rows = T_PREFILL if fit >= T_PREFILL else max(64, fit // 64 * 64)
     wl = synth.make_inputs("prefill", "fused_add_rms_norm", "bf16", rows, H_PREFILL)
     inp = (wl.x, wl.residual, wl.weight, wl.eps)
     for _ in range(args.warmup):
@@ -966,8 +975,12 @@ def main():
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true",
                     help="skip the oracle timing (for profiler runs)")
-    ap.add_argument("--reference-rows", type=int, default=T_PREFILL,
-                    help="rows of the prefill batch per reference (oracle) step (default: all)")
+    ap.add_argument("--reference-rows", type=int, default=0,
+                    help="rows of the prefill batch per reference (oracle) step; 0 (default): "
+                         "all of them when the warm-up and timed steps fit the time budget, "
+                         "else the largest sample that does")
+    ap.add_argument("--reference-budget-s", type=float, default=120.0,
+                    help="host-time budget of the whole reference run when --reference-rows is 0")
     ap.add_argument("--repeats", type=int, default=30,
                     help="timed passes of K steps each; the line reports their median")
     ap.add_argument("--sweep-out", default=None,

@@ -505,8 +505,10 @@ RN_API rn_status rn_force_staged(int32_t ctas_per_sm, int32_t stages, int32_t th
  * launching while the previous kernel in the stream drains; it waits for that
  * kernel to complete before touching memory), 0 launches plainly, -1 restores
  * the library default; max_grid > 0 caps the blocks launched (the kernels
- * stride over the remaining rows), 0 removes the cap. RN_ERR_CONFIG for other
- * values. Not thread-safe with concurrent launches. */
+ * stride over the remaining rows), 0 restores the library's default cap (16
+ * blocks per SM; none for the fused ops on 8192 rows or more and the SwiGLU
+ * kernel on 4096 or more, whose blocks then take one row group each).
+ * RN_ERR_CONFIG for other values. Not thread-safe with concurrent launches. */
 RN_API rn_status rn_set_launch_options(int32_t pdl, int64_t max_grid);
 
 /* L2 prefetch across the kernel boundary for every later call in the

@@ -484,7 +484,8 @@ def force_staged(ctas_per_sm: int, stages: int, threads: int) -> None:
 
 
 def set_launch_options(pdl: int = -1, max_grid: int = 0) -> None:
-    """Tuning hook: pdl 1/0/-1 (on/off/default) and a cap on blocks launched (0 = none)."""
+    """Tuning hook: pdl 1/0/-1 (on/off/default) and a cap on blocks launched
+    (0 = the library's default cap)."""
     _check(lib.rn_set_launch_options(pdl, max_grid), "rn_set_launch_options")
 
 

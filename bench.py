@@ -824,31 +824,35 @@ def time_tp_cell(rn, fp8, W, T, H, iters, device, algorithm="one_shot"):
 def time_chain_cell(rn, T, iters, device, pdl):
     """The decode chain of one layer input: fused_add_rms_norm_fp8 on [T x
     3840] bf16, then the row-wise fp8 GEMM of its codes and per-token scales
-    with the 8192 x 3840 Gemma 4 12B weight. Mean time per chain over `iters`
-    chains under CUDA-graph replay (device time), with or without
+    with the 8192 x 3840 Gemma 4 12B weight. Every chain takes the next of
+    several weights (together >= 4x L2), as each layer of a model has its own,
+    so the weight is read from DRAM and not from L2. Mean time per chain over
+    `iters` chains under CUDA-graph replay (device time), with or without
     programmatic dependent launch between the kernels."""
     H, N = 3840, 8192
     wl = synth.make_inputs("decode", "fused_add_rms_norm_fp8", "bf16", T, H, device=device)
     g = torch.Generator(device=device).manual_seed(T)
-    b = (torch.randn(N, H, generator=g, device=device) * 40).clamp_(-448, 448).to(torch.float8_e4m3fn)
-    sb = torch.rand(N, generator=g, device=device) * 0.01
+    n_w = math.ceil(4 * torch.cuda.get_device_properties(device).L2_cache_size / (N * H)) + 1
+    bs = [(torch.randn(N, H, generator=g, device=device) * 40).clamp_(-448, 448)
+          .to(torch.float8_e4m3fn) for _ in range(n_w)]
+    sbs = [torch.rand(N, generator=g, device=device) * 0.01 for _ in range(n_w)]
     q = torch.empty(T, H, dtype=torch.float8_e4m3fn, device=device)
     sc = torch.empty(T, dtype=torch.float32, device=device)
     d = torch.empty(T, N, dtype=torch.bfloat16, device=device)
     r = wl.residual.clone()
     rn.set_launch_options(pdl=1 if pdl else 0)
     try:
-        def chain():
+        def chain(i):
             rn.fused_add_rms_norm_fp8(q, sc, wl.x, r, wl.weight, wl.eps)
-            rn.fp8_rowwise_gemm(d, q, b, sc, sb)
+            rn.fp8_rowwise_gemm(d, q, bs[i % n_w], sc, sbs[i % n_w])
         st = torch.cuda.Stream(device)
         with torch.cuda.stream(st):
-            chain()
+            chain(0)
             torch.cuda.synchronize(device)
             gr = torch.cuda.CUDAGraph()
             with torch.cuda.graph(gr, stream=st):
-                for _ in range(iters):
-                    chain()
+                for i in range(iters):
+                    chain(i)
         gr.replay()
         torch.cuda.synchronize(device)
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)

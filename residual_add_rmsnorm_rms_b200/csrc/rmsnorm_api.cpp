@@ -29,6 +29,16 @@ static_assert(RN_ALLREDUCE_SIGNAL_BYTES == rn::kArSignalBytes,
               "RN_ALLREDUCE_SIGNAL_BYTES differs from the signal pad layout");
 static_assert(RN_ALLREDUCE_MAX_WORLD == rn::kArMaxWorld,
               "RN_ALLREDUCE_MAX_WORLD differs from the kernels' group limit");
+// (unary + compares the two enums as integers)
+static_assert(+RN_GEMM_TOK128_CH128 == +rn::kGemmTok128Ch128 &&
+                  +RN_GEMM_CH128_TOK16 == +rn::kGemmCh128Tok16 &&
+                  +RN_GEMM_CH128_TOK32 == +rn::kGemmCh128Tok32 &&
+                  +RN_GEMM_CH128_TOK64 == +rn::kGemmCh128Tok64 &&
+                  +RN_GEMM_CH64_TOK16 == +rn::kGemmCh64Tok16 &&
+                  +RN_GEMM_CH64_TOK32 == +rn::kGemmCh64Tok32 &&
+                  +RN_GEMM_CH64_TOK64 == +rn::kGemmCh64Tok64 &&
+                  +RN_GEMM_TOK128_CH256 == +rn::kGemmTok128Ch256 && rn::kNumGemmConfigs == 8,
+              "rn_gemm_config must match the GEMM dispatch");
 
 namespace {
 

@@ -3,7 +3,8 @@
 Ragged hidden sizes (scalar kernel), idle vector slots, every compiled
 vectors-per-thread width and threads-per-row shape (forced), misaligned bases,
 rows aligned for 16-byte but not 32-byte accesses,
-T == 0, in-place out == x, no weight, N-D views, zero rows, fp16 subnormal
+T == 0, tensors of more than 2^31 elements, in-place out == x, no weight,
+N-D views, zero rows, fp16 subnormal
 inputs, determinism, the structural identity fused(x, r).out ==
 rms_norm(r'), non-default streams and validation errors on real tensors.
 """
@@ -14,7 +15,7 @@ import torch
 import synth
 import residual_add_rmsnorm_rms_b200 as rn
 from tests.cmp_util import bits16
-from tests.gpu_util import compare, gpu_run, oracle_run
+from tests.gpu_util import compare, gpu_run, oracle_run, sample_rows
 
 pytestmark = pytest.mark.gpu
 OPS = ["rms_norm", "fused_add_rms_norm", "fused_add_rms_norm_fp8"]
@@ -67,6 +68,34 @@ def test_large_hidden_sizes(op):
     for H in (32768, 40000, 131072 + 8):
         x, r, w = _inputs(3, H, "bf16", seed=H)
         _check(op, x, r, w, 1e-6, "bf16")
+
+
+# More than 2^31 elements per tensor: element indices and byte offsets past
+# 32 bits. 4.6 GB per 16-bit tensor.
+BIG_T = 139264
+
+
+@pytest.mark.parametrize("H", [16384, 16383], ids=["vector", "scalar"])
+@pytest.mark.parametrize("op", OPS)
+def test_more_than_2_31_elements(op, H):
+    """The automatic plan on [139264 x H] bf16 (H = 16383 takes the scalar
+    kernel); the oracle checks a row sample that includes the rows around
+    element 2^31 and the last rows."""
+    wl = synth.make_inputs("sweep", op, "bf16", BIG_T, H, device="cuda")
+    edge = (1 << 31) // H
+    rows = np.unique(np.concatenate([sample_rows(BIG_T, k=64),
+                                     [edge - 1, edge, edge + 1, BIG_T - 2, BIG_T - 1]]))
+    ridx = torch.from_numpy(rows).cuda()
+    x_s = wl.x.index_select(0, ridx).cpu()
+    r_s = None if wl.residual is None else wl.residual.index_select(0, ridx).cpu()
+    got = gpu_run(op, wl.x, wl.residual, wl.weight, wl.eps)
+    got = {k: (v.index_select(0, ridx) if v.dim() and v.shape[0] == BIG_T else v)
+           for k, v in got.items()}
+    torch.cuda.synchronize()
+    want = oracle_run(op, x_s, r_s, wl.weight.cpu(), wl.eps, "bf16")
+    compare(op, got, want, "bf16")
+    del wl, got
+    torch.cuda.empty_cache()
 
 
 def _tpr_for(nvec, vpt):

@@ -82,6 +82,21 @@ def test_swiglu_workload(T, dtype):
         print(_check(xs, q, s, dtype, rows=rows))
 
 
+def test_swiglu_more_than_2_31_elements():
+    """x of [69632 x 2 * 16384] bf16 (2.3e9 elements; row 65536 starts at
+    element 2^31): a row sample including the rows around that element and
+    the last row."""
+    T, I = 69632, 16384
+    wl = synth.make_inputs("swiglu", "silu_and_mul_fp8", "bf16", T, I, device="cuda")
+    edge = (1 << 31) // (2 * I)
+    rows = np.unique(np.concatenate([sample_rows(T, k=64), [edge - 1, edge, edge + 1, T - 1]]))
+    q, s = _gpu(wl.x)
+    xs = wl.x.index_select(0, torch.from_numpy(rows).cuda()).cpu()
+    print(_check(xs, q, s, "bf16", rows=rows))
+    del wl, q, s
+    torch.cuda.empty_cache()
+
+
 @pytest.mark.parametrize("I", [8, 1000, 1004, 4096, 15360, 40000])
 def test_swiglu_shapes_and_scalar_path(I):
     """Ragged I (scalar kernel), narrow and wide rows."""

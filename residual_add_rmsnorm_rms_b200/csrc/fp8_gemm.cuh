@@ -35,6 +35,7 @@
 // so they round identically.
 #pragma once
 
+#include <atomic>
 #include <cstdint>
 #include <type_traits>
 
@@ -59,6 +60,7 @@ using ElementAB = cutlass::float_e4m3_t;
 using ElementD = cutlass::bfloat16_t;
 constexpr int kAlignAB = 16;  // elements: 16 bytes of e4m3 per TMA row granule
 constexpr int kAlignD = 8;    // elements: 16 bytes of bf16
+constexpr int kGemmMaxDevices = 64;
 
 template <class MmaTile, bool kSwapAB>
 struct RowwiseGemm {
@@ -124,12 +126,24 @@ struct RowwiseGemm {
             {}};
         args.hw_info.device_id = g.device;
         args.hw_info.sm_count = g.num_sms;
-        Gemm gemm;
-        if (gemm.can_implement(args) != cutlass::Status::kSuccess) return cudaErrorInvalidValue;
+        if (Gemm::can_implement(args) != cutlass::Status::kSuccess) return cudaErrorInvalidValue;
         if (Gemm::get_workspace_size(args) != 0) return cudaErrorInvalidValue;  // none by design
-        if (gemm.initialize(args, nullptr, stream) != cutlass::Status::kSuccess)
+        if (Kernel::initialize_workspace(args, nullptr, stream) != cutlass::Status::kSuccess)
             return cudaErrorInvalidConfiguration;
-        if (gemm.run(stream, nullptr, g.pdl) != cutlass::Status::kSuccess)
+        typename Gemm::Params params = Kernel::to_underlying_arguments(args, nullptr);
+        // The adapter's initialize() sets the kernel's dynamic shared memory
+        // limit on every call; here it is set once per device and CUDA context
+        // (and on every call when the context id is unknown).
+        static std::atomic<unsigned long long> ready[kGemmMaxDevices];
+        const bool known = g.ctx_id != 0 && g.device >= 0 && g.device < kGemmMaxDevices;
+        if (!known || ready[g.device].load(std::memory_order_relaxed) != g.ctx_id) {
+            const cudaError_t e = cudaFuncSetAttribute(
+                cutlass::device_kernel<Kernel>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                static_cast<int>(Kernel::SharedStorageSize));
+            if (e != cudaSuccess) return e;
+            if (known) ready[g.device].store(g.ctx_id, std::memory_order_relaxed);
+        }
+        if (Gemm::run(params, stream, nullptr, g.pdl) != cutlass::Status::kSuccess)
             return cudaErrorLaunchFailure;
         return cudaGetLastError();
     }

@@ -618,6 +618,8 @@ rn_status run(int op, const rn_tensor* o, const rn_tensor* sc, const rn_tensor* 
                        pair_ok(op, a.H, a.x, a.residual, a.out, a.q), stream);
 }
 
+bool current_context_id(unsigned long long* id);  // below
+
 }  // namespace
 
 extern "C" {
@@ -727,6 +729,7 @@ rn_status rn_fp8_rowwise_gemm(const rn_tensor* d, const rn_tensor* a, const rn_t
                        device_sms(), 0, false};
         g.config = gemm_config(M, N, g.num_sms);
         g.pdl = g_pdl.load() < 0 ? kPdlDefault : g_pdl.load() == 1;
+        if (!current_context_id(&g.ctx_id)) g.ctx_id = 0;
         e = rn::launch_fp8_rowwise_gemm(g, static_cast<cudaStream_t>(stream));
     }
     if (e != cudaSuccess) {

@@ -20,6 +20,7 @@ struct GemmArgs {
     int num_sms;
     int config;           // GemmConfig: tile shape and orientation
     bool pdl;             // launch with programmatic dependent launch
+    unsigned long long ctx_id = 0;  // id of the current CUDA context (0: unknown)
 };
 
 // Tile configurations of the fp8 GEMM (values of rn_gemm_config in the public

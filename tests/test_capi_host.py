@@ -442,3 +442,44 @@ def test_status_strings():
     for code, name in rn.STATUS.items():
         assert rn.status_string(code)
     assert rn.status_string(999) == "unknown status"
+
+
+def test_host_logic_from_many_threads():
+    """rn_validate and rn_plan_launch from eight threads at once give the
+    results of the same calls made serially (pure host logic, per-thread
+    descriptor caches in the binding)."""
+    import threading
+    shapes = [(op, T, H) for op in ("rms_norm", "fused_add_rms_norm", "fused_add_rms_norm_fp8")
+              for T in (1, 7, 4096) for H in (8, 3840, 16384, 4100)]
+
+    def run_all():
+        out = []
+        for op, T, H in shapes:
+            x = torch.empty(T, H, dtype=torch.bfloat16)
+            o = (torch.empty(T, H, dtype=torch.float8_e4m3fn) if op.endswith("fp8")
+                 else torch.empty_like(x))
+            sc = torch.empty(T, dtype=torch.float32) if op.endswith("fp8") else None
+            r = None if op == "rms_norm" else torch.empty_like(x)
+            st, plan = rn.validate(op, o, x, residual=r, weight=torch.empty(H, dtype=torch.bfloat16),
+                                   scale=sc)
+            out.append((st, tuple(sorted(plan.items())),
+                        tuple(sorted(rn.plan_launch(op, torch.bfloat16, T, H).items()))))
+        return out
+
+    want = run_all()
+    got, errors = [None] * 8, []
+
+    def worker(i):
+        try:
+            got[i] = [run_all() for _ in range(3)]
+        except Exception as e:  # noqa: BLE001
+            errors.append(repr(e))
+
+    threads = [threading.Thread(target=worker, args=(i,)) for i in range(8)]
+    for t in threads:
+        t.start()
+    for t in threads:
+        t.join(timeout=120)
+    assert not errors, errors
+    for g in got:
+        assert all(r == want for r in g)

@@ -9,12 +9,14 @@ weight = 1 + N(0,0.1), eps 1e-6) through
 Metric: algorithmic HBM GB/s of the step (bytes every element must move,
 weight counted once per launch), its fraction of the HBM roofline, and rows/s.
 
-Timing: W untimed warm-up steps, then R (default 30) timed passes of exactly
-K steps, each bracketed by a barrier and a device synchronize and timed with
-CUDA events on the launching stream; the line reports the median pass with
-the fastest and slowest, and an NVML clock sample taken during each pass.
-Per-kernel durations: each op alone, K launches back to back between one
-event pair, median over R such passes. L2: launches rotate over
+Timing: W untimed warm-up steps; the K steps' launches are recorded once into
+a CUDA graph (--eager: issued one by one instead), then R (default 30) timed
+passes, each one replay of exactly K steps, bracketed by a barrier and a
+device synchronize and timed with CUDA events on the launching stream; the
+line reports the median pass with the fastest and slowest, and an NVML clock
+sample taken during each pass. Per-kernel durations: each op alone, K
+launches back to back (one graph replay) between one event pair, median over
+R such passes. L2: launches rotate over
 buffer sets totalling >= 4x the L2 size, so no launch reads data the previous
 launches left in L2. Under torchrun each rank runs an independent replica
 (no collective on the data path; the path has no exchange step) and rank 0

@@ -618,7 +618,8 @@ rn_status run(int op, const rn_tensor* o, const rn_tensor* sc, const rn_tensor* 
                        pair_ok(op, a.H, a.x, a.residual, a.out, a.q), stream);
 }
 
-bool current_context_id(unsigned long long* id);  // below
+// The current CUDA context's unique id (defined with the local all-reduce state).
+bool current_context_id(unsigned long long* id);
 
 }  // namespace
 

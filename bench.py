@@ -386,6 +386,8 @@ def run_ours(args, world, rank, local):
     # replayed on `stream`, as a decoder layer's kernels run in production
     # (programmatic dependent launch keeps its overlap between the graph's
     # kernel nodes); with --eager, the same launches issued one by one.
+    graphs = []  # kept alive until the buffer sets are released
+
     def sequence(ops):
         def run(st=None):
             for i in range(K):
@@ -407,7 +409,6 @@ def run_ours(args, world, rank, local):
                 g.replay()
         return replay
 
-    graphs = []
     seq_step, seq_ops = sequence((0, 1)), [sequence((0,)), sequence((1,))]
     seq_step()  # one untimed run of each recorded sequence
     for f in seq_ops:

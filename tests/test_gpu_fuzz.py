@@ -6,7 +6,8 @@ bytes (16- but not 32-byte aligned rows), and out == x in place. Each case
 meets the oracle tolerances (residual bit-exact, outputs within 1 ulp, codes
 within 1, scales within 1e-6); the fraction of e4m3 codes that differ is
 bounded over all the fp8 cases together (<= 0.1 %), as for one workload.
-The fused SwiGLU + FP8 op gets the same treatment on random [T x 2I] rows."""
+The fused SwiGLU + FP8 op gets the same treatment on random [T x 2I] rows,
+and the fp8 GEMM on random M x N x K with its automatic tile choice."""
 import numpy as np
 import pytest
 import torch
@@ -139,3 +140,20 @@ def test_fuzz_swiglu():
         gs = s.cpu().numpy().astype(np.float64)
         assert (np.abs(gs - ws) <= SCALE_RTOL * np.abs(ws)).all(), (c, T, I, dtype)
     assert diff / total <= FP8_MAX_MISMATCH_FRAC, diff / total
+
+
+def test_fuzz_fp8_gemm():
+    """fp8_rowwise_gemm with the automatic tile configuration on random M x N x
+    K (N a multiple of 8, K of 16), checked in full against the oracle with
+    the derived per-element bound of the GEMM tests."""
+    from tests.test_gpu_fp8_gemm import _check, _operands
+    rng = np.random.default_rng(2024)
+    for c in range(30):
+        M = int(rng.integers(1, 301))
+        N = 8 * int(rng.integers(1, 257))
+        K = 16 * int(rng.integers(1, 129))
+        a, b, sa, sb = _operands(M, N, K, seed=900 + c)
+        d = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+        rn.fp8_rowwise_gemm(d, a.cuda(), b.cuda(), sa.cuda(), sb.cuda())
+        torch.cuda.synchronize()
+        _check(d, codes8(a), codes8(b), sa.numpy(), sb.numpy())

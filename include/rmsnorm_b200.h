@@ -28,9 +28,11 @@
  *    library allocates nothing and keeps no pointer after returning. Its
  *    only global state:
  *    the test and tuning overrides (rn_force_plan, rn_force_staged,
- *    rn_set_launch_options, rn_fp8_gemm_force_config), the thread-local
- *    error text, the device error flags (rn_device_errors) and the static
- *    exchange memory of rn_allreduce_fused_add_rms_norm_local.
+ *    rn_set_launch_options, rn_set_prefetch, rn_fp8_gemm_force_config), the
+ *    thread-local error text, the device error flags (rn_device_errors), the
+ *    static exchange memory of rn_allreduce_fused_add_rms_norm_local, and,
+ *    per device, the id of the CUDA context in which each GEMM kernel's
+ *    shared-memory limit was last set.
  *  - Views. A tensor is described by rn_tensor (pointer, dtype, sizes and
  *    strides in ELEMENTS). It must flatten to a dense [T x H] matrix for free:
  *    the last stride is 1 and each leading dimension of size != 1 has the

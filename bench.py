@@ -388,6 +388,8 @@ def run_ours(args, world, rank, local):
     # kernel nodes); with --eager, the same launches issued one by one.
     graphs = []  # kept alive until the buffer sets are released
 
+    timed_how = []
+
     def sequence(ops):
         def run(st=None):
             for i in range(K):
@@ -398,10 +400,15 @@ def run_ours(args, world, rank, local):
         side = torch.cuda.Stream(device)
         side.wait_stream(stream)
         g = torch.cuda.CUDAGraph()
-        with torch.cuda.stream(side):
-            with torch.cuda.graph(g, stream=side):
-                run(side)
-        torch.cuda.synchronize(device)
+        try:
+            with torch.cuda.stream(side):
+                with torch.cuda.graph(g, stream=side):
+                    run(side)
+            torch.cuda.synchronize(device)
+        except RuntimeError as e:  # no graph on this setup: time the launches one by one
+            torch.cuda.synchronize(device)
+            timed_how.append(f"eager launches (CUDA-graph capture failed: {str(e)[:120]})")
+            return run
         graphs.append(g)
 
         def replay():
@@ -498,7 +505,7 @@ def run_ours(args, world, rank, local):
         "per_kernel_how": f"each op alone, {K} launches back to back "
                           f"({'eager' if args.eager else 'one CUDA-graph replay'}), events at the "
                           f"ends; median of {R} such passes",
-        "timed": ("eager launches" if args.eager else
+        "timed": (timed_how[0] if timed_how else "eager launches" if args.eager else
                   "CUDA-graph replay of the K-step launch sequence (recorded once per run)"),
         "per_kernel_ms": {"fused_add_rms_norm": round(dom_ms, 5),
                           "fused_add_rms_norm_fp8": round(fp8_ms, 5)},

@@ -172,3 +172,42 @@ def test_gemm_validation():
     empty = torch.empty(0, 32, dtype=torch.float8_e4m3fn, device="cuda")
     rn.fp8_rowwise_gemm(torch.empty(0, 16, dtype=torch.bfloat16, device="cuda"), empty, b,
                         torch.empty(0, device="cuda"), sb)
+
+
+_CAPTURE_FIRST = r"""
+import torch, residual_add_rmsnorm_rms_b200 as rn
+torch.cuda.init()
+g = torch.Generator(device="cuda").manual_seed(3)
+M, N, K = 16, 3840, 4096
+a = (torch.randn(M, K, generator=g, device="cuda") * 40).clamp_(-448, 448).to(torch.float8_e4m3fn)
+b = (torch.randn(N, K, generator=g, device="cuda") * 40).clamp_(-448, 448).to(torch.float8_e4m3fn)
+sa = torch.rand(M, generator=g, device="cuda") * 0.01 + 1e-3
+sb = torch.rand(N, generator=g, device="cuda") * 0.01 + 1e-3
+d_graph = torch.empty(M, N, dtype=torch.bfloat16, device="cuda")
+st = torch.cuda.Stream()
+graph = torch.cuda.CUDAGraph()
+with torch.cuda.stream(st):
+    with torch.cuda.graph(graph, stream=st):  # the process's first GEMM call
+        rn.fp8_rowwise_gemm(d_graph, a, b, sa, sb)
+graph.replay()
+torch.cuda.synchronize()
+d = torch.empty_like(d_graph)
+rn.fp8_rowwise_gemm(d, a, b, sa, sb)
+torch.cuda.synchronize()
+assert torch.equal(d.view(torch.int16), d_graph.view(torch.int16))
+assert rn.device_errors() == 0
+print("ok")
+"""
+
+
+def test_gemm_first_call_inside_graph_capture():
+    """A process whose first GEMM call is recorded into a CUDA graph (the
+    kernel's shared-memory limit is then set during the capture) replays it
+    to the same bits as an eager call."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    out = subprocess.run([sys.executable, "-c", _CAPTURE_FIRST], cwd=root, capture_output=True,
+                         text=True, timeout=300, env=dict(os.environ, PYTHONPATH=root))
+    assert out.returncode == 0 and out.stdout.strip().endswith("ok"), out.stderr[-2000:]
